@@ -1,0 +1,163 @@
+"""Pins of the oracle's dispatch (bf16 copy, fp8 1x128 quantisation) and
+combine (router-weighted sum): hand-worked fixtures, the quantisation error
+bound of E4M3, sign symmetry, Higham's bound for recursive summation against
+a binary64 recomputation, and the dispatch -> identity expert -> combine
+invariant (the weight-scaled input)."""
+import numpy as np
+import pytest
+import torch
+
+from conftest import load_golden
+from harness import inputs
+
+U = 2.0 ** -24  # binary32 unit roundoff
+
+
+def _bits(t):
+    return inputs.bf16_bits(t)
+
+
+def _f(bits):
+    return inputs.bits_to_bf16(bits).float().numpy()
+
+
+# ----------------------------------------------------------------- dispatch
+
+def test_dispatch_bf16_copies_rows_and_leaves_others(oracle_mod):
+    cfg = inputs.CONFIGS["tiny"]
+    idx, _ = oracle_mod.route(inputs.make_logits(cfg).numpy(), cfg.k)
+    lay = oracle_mod.layout(idx, cfg.E, cfg.R)
+    x = _bits(inputs.make_x(cfg))
+    rows = cfg.T * cfg.k + 3                      # 3 spare rows: canaries
+    canary = np.full((rows, cfg.H), 0xBEEF, np.uint16)
+    out = oracle_mod.dispatch_bf16(x, lay["dispatch_pos"], rows, canary.copy())
+    for g in range(cfg.T):
+        for j in range(cfg.k):
+            assert np.array_equal(out[lay["dispatch_pos"][g, j]], x[g])
+    assert np.all(out[cfg.T * cfg.k:] == 0xBEEF)
+
+
+def test_fp8_block_hand_example(oracle_mod):
+    fx = load_golden("fp8_block_hand.json")
+    b0 = torch.tensor([i / 127 for i in range(128)], dtype=torch.float64).to(torch.bfloat16)
+    x = torch.cat([b0, -b0, torch.zeros(128, dtype=torch.bfloat16)]).reshape(1, fx["H"])
+    q, s = oracle_mod.quantize_tokens(_bits(x), [0])
+    inv448 = np.float32(1.0 / 448.0)            # nearest binary32 to 1/448
+    assert s[0].tolist() == [inv448, inv448, 1.0]
+    blocks = {"b0": 0, "b1": 1, "b2": 2}
+    for b, i, code in fx["expect"]["codes"]:
+        assert q[0, blocks[b] * 128 + i] == int(code, 16), (b, i)
+
+
+def test_fp8_exact_tie_pins_true_division(oracle_mod):
+    tb = load_golden("fp8_block_hand.json")["tie_block"]
+    x = torch.zeros(1, 128, dtype=torch.float64)
+    x[0, :2] = torch.tensor(tb["x"], dtype=torch.float64)
+    q, s = oracle_mod.quantize_tokens(_bits(x.to(torch.bfloat16)), [0])
+    assert s[0, 0] == np.float32(tb["scale"])
+    assert [int(c) for c in q[0, :3]] == [int(c, 16) for c in tb["codes"]]
+
+
+def test_fp8_properties_on_workload_rows(oracle_mod):
+    cfg = inputs.CONFIGS["dsv3"]
+    x = inputs.make_x(cfg)[:64]
+    q, s = oracle_mod.quantize_tokens(_bits(x), np.arange(64))
+    S = cfg.H // 128
+    mag = q & 0x7F
+    assert np.all(mag.reshape(64, S, 128).max(2) == 0x7E)   # amax maps to 448
+    assert np.all(s > 0)
+    # |dequant - x| <= max(2^-4 |x|, s 2^-10) (half an E4M3 ulp), plus the
+    # binary32 roundings of x/s and of the dequantising product
+    xf = x.float().numpy().reshape(64, S, 128)
+    deq = (oracle_mod.e4m3_decode(q).reshape(64, S, 128).astype(np.float64)
+           * s.reshape(64, S, 1))
+    bound = np.maximum(2.0 ** -4 * np.abs(xf), s.reshape(64, S, 1) * 2.0 ** -10) * (1 + 4 * U)
+    assert np.all(np.abs(deq - xf) <= bound)
+    # sign symmetry: -x gives the same scales and codes with the sign flipped
+    qn, sn = oracle_mod.quantize_tokens(_bits(-x), np.arange(64))
+    assert np.array_equal(sn, s)
+    assert np.array_equal(qn, q ^ 0x80)
+
+
+def test_fp8_dispatch_writes_each_token_to_its_k_rows(oracle_mod):
+    cfg = inputs.CONFIGS["dsv3"]
+    T = 96
+    logits = inputs.make_logits(cfg)[:T].numpy()
+    idx, _ = oracle_mod.route(logits, cfg.k)
+    lay = oracle_mod.layout(idx, cfg.E, 1)
+    x = _bits(inputs.make_x(cfg)[:T])
+    q, s = oracle_mod.dispatch_fp8(x, lay["dispatch_pos"], T * cfg.k)
+    qt, st = oracle_mod.quantize_tokens(x, np.arange(T))
+    for g in range(T):
+        for j in range(cfg.k):
+            r = lay["dispatch_pos"][g, j]
+            assert np.array_equal(q[r], qt[g]) and np.array_equal(s[r], st[g])
+
+
+# ------------------------------------------------------------------ combine
+
+@pytest.mark.parametrize("case", load_golden("combine_hand.json")["cases"], ids=lambda c: c["name"])
+def test_combine_hand_cases(oracle_mod, case):
+    y = _bits(torch.tensor(case["y"], dtype=torch.float64).to(torch.bfloat16))
+    pos = np.array(case["dispatch_pos"], np.int32)
+    w = np.array(case["topk_w"], np.float32)
+    acc, out = oracle_mod.combine(y, pos, w)
+    assert acc[0].tolist() == case["acc"]
+    assert np.array_equal(out[0], oracle_mod.float_to_bf16_bits(acc[0]))
+
+
+@pytest.mark.parametrize("k", [1, 2, 8, 16])
+def test_combine_higham_bound_vs_binary64(oracle_mod, k):
+    """|acc - exact| <= gamma_k * sum_j |w_j y_j|, gamma_k = k u / (1 - k u)
+    (recursive summation of k rounded products)."""
+    T, H, rows = 64, 256, 64 * k
+    rng = np.random.default_rng(k)
+    pos = rng.permutation(rows).astype(np.int32).reshape(T, k)
+    w = rng.random((T, k)).astype(np.float32)
+    y = _bits(inputs.make_random_rows(rows, H, seed=k))
+    acc, out = oracle_mod.combine(y, pos, w)
+    yf = _f(y).astype(np.float64)
+    terms = w.astype(np.float64)[:, :, None] * yf[pos]          # [T][k][H]
+    exact = terms.sum(1)
+    gamma = k * U / (1 - k * U)
+    assert np.all(np.abs(acc - exact) <= gamma * np.abs(terms).sum(1))
+    # k = 1 with w = 1 is an exact copy
+    if k == 1:
+        acc1, out1 = oracle_mod.combine(y, pos, np.ones((T, 1), np.float32))
+        assert np.array_equal(out1, y[pos[:, 0]])
+
+
+def test_combine_token_subset_matches_full(oracle_mod):
+    T, H, k = 40, 128, 4
+    rng = np.random.default_rng(3)
+    pos = rng.permutation(T * k).astype(np.int32).reshape(T, k)
+    pos[5, 2] = -1
+    w = rng.random((T, k)).astype(np.float32)
+    y = _bits(inputs.make_random_rows(T * k, H, seed=4))
+    acc, out = oracle_mod.combine(y, pos, w)
+    sub = np.array([39, 5, 0, 17], np.int32)
+    acc_s, out_s = oracle_mod.combine(y, pos, w, tokens=sub)
+    assert np.array_equal(acc_s, acc[sub]) and np.array_equal(out_s, out[sub])
+
+
+@pytest.mark.parametrize("renormalize", [False, True])
+def test_dispatch_identity_combine_returns_weight_scaled_input(oracle_mod, renormalize):
+    """dispatch (bf16) -> identity expert -> combine gives bf16(x * sum_j w_j)
+    up to the summation bound; renormalised weights give back x within one
+    bf16 ulp plus that bound."""
+    cfg = inputs.CONFIGS["mixtral"]
+    logits = inputs.make_logits(cfg).numpy()
+    idx, w = oracle_mod.route(logits, cfg.k, renormalize=renormalize)
+    lay = oracle_mod.layout(idx, cfg.E, cfg.R)
+    x = _bits(inputs.make_x(cfg))
+    recv = oracle_mod.dispatch_bf16(x, lay["dispatch_pos"], cfg.T * cfg.k)
+    acc, out = oracle_mod.combine(recv, lay["dispatch_pos"], w)
+    xf = _f(x).astype(np.float64)
+    wsum = w.astype(np.float64).sum(1, keepdims=True)
+    target = xf * wsum
+    gamma = cfg.k * U / (1 - cfg.k * U)
+    assert np.all(np.abs(acc - target) <= gamma * np.abs(target) + 1e-45)
+    if renormalize:
+        outf = _f(out).astype(np.float64)
+        ulp = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(xf), 2.0 ** -126))) - 7)
+        assert np.all(np.abs(outf - xf) <= ulp + cfg.k * 2 ** -23 * np.abs(xf))
