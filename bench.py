@@ -1,0 +1,492 @@
+#!/usr/bin/env python
+"""Benchmark of the MoE route -> layout -> dispatch -> combine path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config dsv3]
+                    [--impl ours|reference]
+
+One step = one pass of the whole path over one batch of seeded synthetic
+input: moe_route_topk, moe_dispatch_layout, moe_dispatch_fp8 (or _bf16) and
+moe_combine_bf16.  The stand-in expert between dispatch and combine is not
+part of the path (it needs trained weights): its outputs are prepared once,
+before timing, and stay resident, as a grouped GEMM would leave them.
+
+Timing: W untimed warm-up steps, then exactly K timed steps between a
+barrier + device synchronise on both sides.  Before every step a 512 MiB
+buffer is written to flush L2 (126 MB) outside the timed events; each step
+and each stage is timed with CUDA events on the stream the kernels run on.
+Clocks and throttle reasons are sampled with nvidia-smi during the timed
+region.  With N > 1 (torchrun) every rank runs an independent replica (the
+path does not shard: no data-path collective); the reported time is the
+maximum over ranks and `value` the bytes of all ranks over that time.
+
+`value` is the effective HBM bandwidth of a step: the algorithmic bytes the
+path must move (each token read once, each row written once, see
+algorithmic_bytes) divided by the step time.  The reference arm
+(--impl reference) times the oracle, a plain single-threaded CPU program,
+on the same workload and metric.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime as _dt
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from harness import experts, inputs  # noqa: E402
+
+METRIC = "dispatch+combine µs/layer and effective HBM GB/s (% of B200 roofline), 1 GPU"
+SPEC_HBM_GBS = 8000.0          # B200 HBM3e bandwidth the roofline target is quoted against
+FALLBACK_HBM_GBS = 6650.0      # earlier measured copy bandwidth on this machine
+L2_FLUSH_BYTES = 512 << 20
+KERNELS_PER_STEP = 5           # route, layout (2 kernels), dispatch, combine
+
+
+# --------------------------------------------------------------------------
+# algorithmic bytes
+# --------------------------------------------------------------------------
+
+def algorithmic_bytes(cfg: inputs.Config, rows: int, kept: int) -> dict:
+    """Minimal bytes each stage must move.  kept = slots that have a row
+    (T*k when nothing is dropped); rows = receive rows laid out."""
+    T, H, E, k, R = cfg.T, cfg.H, cfg.E, cfg.k, cfg.R
+    S = H // 128
+    route = T * E * 4 + T * k * 8
+    layout = T * k * 4 + E * 4 * (2 + R) + 4 + R * 4 + T * k * 4 + rows * 4
+    if cfg.dispatch == "fp8":
+        dispatch = T * H * 2 + T * k * 4 + kept * H + kept * S * 4
+    else:
+        dispatch = T * H * 2 + T * k * 4 + kept * H * 2
+    combine = kept * H * 2 + T * k * 8 + T * H * 2
+    return dict(route=route, layout=layout, dispatch=dispatch, combine=combine,
+                step=route + layout + dispatch + combine)
+
+
+def load_peak() -> tuple[float, str]:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def combine_traffic(cfg_name: str):
+    """DRAM bytes per launch of the combine kernel from the committed ncu
+    summary, or None when that summary is missing or the kernel source has
+    changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", f"combine_{cfg_name}_traffic.json")
+    src = os.path.join(ROOT, "combine_moe_route_08_b200", "csrc", "combine.cu")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+        with open(src, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
+    except (OSError, ValueError):
+        return None
+    if rec.get("source_sha256") != sha:
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+# --------------------------------------------------------------------------
+# clocks during the timed region
+# --------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.t0 = self.t1 = None
+        uuid = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            if not uuid.startswith("GPU-"):
+                uuid = "GPU-" + uuid
+        except Exception:
+            uuid = None
+        self.sel = uuid or str(device_index)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.sel, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def mark_start(self):
+        self.t0 = _dt.datetime.now()
+
+    def mark_end(self):
+        self.t1 = _dt.datetime.now()
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.1)
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        rows = []
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                ts = _dt.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f")
+            except ValueError:
+                continue
+            rows.append((ts, parts))
+        inside = [p for ts, p in rows if self.t0 and self.t1 and self.t0 <= ts <= self.t1]
+        use = inside or [p for _, p in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for p in use for n, v in zip(names, p[5:9]) if v.lower() == "active"})
+        sm = [float(p[1]) for p in use if p[1].replace(".", "").isdigit()]
+        smax = [float(p[2]) for p in use if p[2].replace(".", "").isdigit()]
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(use), "samples_in_timed_region": len(inside)}
+
+
+# --------------------------------------------------------------------------
+# multi-rank plumbing (replicas: only a barrier and a max of the timings)
+# --------------------------------------------------------------------------
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return world, rank, local
+
+
+def init_dist(world: int, backend: str):
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group(backend, timeout=_dt.timedelta(seconds=120))
+    return dist
+
+
+def barrier(world: int, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        if dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[device.index] if device is not None else None)
+        else:
+            dist.barrier()
+
+
+def max_over_ranks(values: list[float], world: int, device) -> list[float]:
+    """Element-wise maximum of per-rank timings (all ranks call this)."""
+    if world == 1:
+        return list(values)
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.cpu().tolist()
+
+
+# --------------------------------------------------------------------------
+# the oracle as CPU baseline / reference arm
+# --------------------------------------------------------------------------
+
+def oracle_step_on_sample(cfg: inputs.Config, wl: dict, tokens: int) -> tuple[float, int]:
+    """Run the oracle's route -> layout -> dispatch -> combine on the first
+    `tokens` tokens (whole logical ranks) of the workload; returns (seconds,
+    algorithmic bytes of that sample)."""
+    import oracle
+    sub = inputs.Config(cfg.name, cfg.index, tokens // cfg.R if tokens % cfg.R == 0 else tokens,
+                        cfg.R if tokens % cfg.R == 0 else 1, cfg.H, cfg.E, cfg.k, cfg.dispatch,
+                        cfg.layout, cfg.expert, cfg.zipf)
+    T = sub.T
+    logits = wl["logits_np"][:T]
+    xb = wl["x_bits"][:T]
+    t0 = time.perf_counter()
+    idx, w = oracle.route(logits, cfg.k)
+    lay = oracle.layout(idx, cfg.E, sub.R)
+    cap = 0
+    if cfg.layout == "padded":
+        cap = int(lay["expert_counts"].max())
+        lay = oracle.layout(idx, cfg.E, sub.R, cap)
+    rows = lay["recv_src"].shape[0]
+    pos = lay["dispatch_pos"]
+    if cfg.dispatch == "fp8":
+        oracle.dispatch_fp8(xb, pos, rows)
+    else:
+        oracle.dispatch_bf16(xb, pos, rows)
+    y = wl["y_bank_bits"]
+    pos_bank = np.where(pos >= 0, pos % y.shape[0], -1).astype(np.int32)
+    oracle.combine(y, pos_bank, w)
+    dt = time.perf_counter() - t0
+    kept = int(np.sum(pos >= 0))
+    return dt, algorithmic_bytes(sub, rows, kept)["step"]
+
+
+def cpu_inputs(cfg: inputs.Config) -> dict:
+    logits = inputs.make_logits(cfg)
+    x = inputs.make_x(cfg)
+    bank = inputs.make_row_bank(cfg.H, seed=cfg.seed * 10 + 2, n=min(cfg.T * cfg.k, 32768))
+    return dict(logits_np=logits.numpy(), x_bits=inputs.bf16_bits(x),
+                y_bank_bits=inputs.bf16_bits(bank))
+
+
+def cpu_baseline(cfg: inputs.Config, budget_s: float = 12.0) -> dict:
+    """The oracle as it stands, single-threaded, on whole-workload steps
+    repeated until about `budget_s` seconds of CPU work."""
+    wl = cpu_inputs(cfg)
+    total_t, total_b, n = 0.0, 0, 0
+    while n == 0 or total_t < budget_s:
+        dt, b = oracle_step_on_sample(cfg, wl, cfg.T)
+        total_t += dt
+        total_b += b
+        n += 1
+    return {"value": total_b / total_t / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "host_cores": os.cpu_count(),
+            "sample": f"{n} full {cfg.name} step(s) (T={cfg.T}), {total_t:.1f} s of CPU work, "
+                      f"1 thread of {os.cpu_count()} host cores",
+            "s_per_step": total_t / n}
+
+
+def run_reference(args) -> None:
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return  # the oracle runs on rank 0 only; other ranks exit without work
+    cfg = inputs.CONFIGS[args.config]
+    wl = cpu_inputs(cfg)
+    # size each step so that warm-up + timed steps fit in about two minutes
+    dt1, _ = oracle_step_on_sample(cfg, wl, cfg.R)           # one token per rank
+    per_token = dt1 / cfg.R
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    ranks = max(1, min(cfg.T_r, int(budget / per_token / cfg.R)))
+    tokens = ranks * cfg.R
+    for _ in range(args.warmup):
+        oracle_step_on_sample(cfg, wl, tokens)
+    tt, tb = 0.0, 0
+    for _ in range(args.steps):
+        dt, b = oracle_step_on_sample(cfg, wl, tokens)
+        tt += dt
+        tb += b
+    value = tb / tt / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * tt / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": cfg.describe(), "sample_tokens_per_step": tokens},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{tokens} of {cfg.T} tokens per step "
+                                   f"({ranks} per logical rank), 1 thread of {os.cpu_count()}"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------
+# our arm
+# --------------------------------------------------------------------------
+
+def run_ours(args) -> None:
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_dist(world, "nccl")
+    import combine_moe_route_08_b200 as moe
+
+    cfg = inputs.CONFIGS[args.config]
+    T, H, E, k, R = cfg.T, cfg.H, cfg.E, cfg.k, cfg.R
+    logits_h = inputs.make_logits(cfg)
+    x_h = inputs.make_x(cfg)
+    logits = logits_h.to(dev)
+    x = x_h.to(dev)
+    s = torch.cuda.Stream(dev)
+    ws = moe.Workspace(dev)
+
+    with torch.cuda.stream(s):
+        idx, w = moe.moe_route_topk(logits, k)
+        cap = 0
+        if cfg.layout == "padded":  # capacity = max observed count, read once, untimed
+            probe = moe.moe_dispatch_layout(idx, E, R, workspace=ws)
+            cap = int(probe["expert_counts"].max().item())
+            del probe
+        rows = T * k if cap == 0 else E * cap
+        lay = moe.moe_dispatch_layout(idx, E, R, capacity=cap, rows=rows, workspace=ws)
+        if cfg.dispatch == "fp8":
+            recv_q, recv_scale = moe.moe_dispatch_fp8(x, lay["dispatch_pos"], rows)
+            y = experts.dequantise(recv_q, recv_scale)
+        else:
+            recv_x = moe.moe_dispatch_bf16(x, lay["dispatch_pos"], rows)
+            y = recv_x.clone() if cfg.expert == "identity" else experts.affine(
+                recv_x, inputs.make_expert_noise(cfg, rows))
+        out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+        kept = int((lay["dispatch_pos"] >= 0).sum().item())
+        flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    s.synchronize()
+
+    def step(ev=None):
+        """One pass of the path; with `ev`, events ev[1..3] mark the stage ends."""
+        moe.moe_route_topk(logits, k, topk_idx=idx, topk_w=w)
+        if ev is not None:
+            ev[1].record(s)
+        moe.moe_dispatch_layout(idx, E, R, capacity=cap, rows=rows, out=lay, workspace=ws)
+        if ev is not None:
+            ev[2].record(s)
+        if cfg.dispatch == "fp8":
+            moe.moe_dispatch_fp8(x, lay["dispatch_pos"], rows, recv_q=recv_q, recv_scale=recv_scale)
+        else:
+            moe.moe_dispatch_bf16(x, lay["dispatch_pos"], rows, recv_x=recv_x)
+        if ev is not None:
+            ev[3].record(s)
+        moe.moe_combine_bf16(y, lay["dispatch_pos"], w, out=out)
+
+    nb = algorithmic_bytes(cfg, rows, kept)
+    K, W = args.steps, args.warmup
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    with torch.cuda.stream(s):
+        for i in range(W):
+            flush.fill_(i)
+            step()
+        s.synchronize()
+        sampler = ClockSampler(local)
+        sampler.start()
+        barrier(world, dev)
+        torch.cuda.synchronize(dev)
+        sampler.mark_start()
+        for i in range(K):
+            flush.fill_(i)
+            evs[i][0].record(s)
+            step(evs[i])
+            evs[i][4].record(s)
+        s.synchronize()
+        torch.cuda.synchronize(dev)
+        barrier(world, dev)
+        sampler.mark_end()
+        clocks = sampler.stop()
+
+    stage_ms = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(4)] for e in evs])
+    step_ms = stage_ms.sum(1)
+    local_ms = [float(step_ms.mean()), *[float(v) for v in stage_ms.mean(0)]]
+    ms = max_over_ranks(local_ms, world, dev)
+    ms_step, ms_route, ms_layout, ms_dispatch, ms_combine = ms
+
+    # ---- CUDA graph of the same step (launch overhead removed) ----
+    graph_ms = None
+    if not args.no_graph:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            step()
+        gt = []
+        with torch.cuda.stream(s):
+            for i in range(max(W, 3)):
+                g.replay()
+            for i in range(min(K, 200)):
+                flush.fill_(i)
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(s)
+                g.replay()
+                b.record(s)
+                gt.append((a, b))
+            s.synchronize()
+        graph_ms = max_over_ranks([float(np.mean([a.elapsed_time(b) for a, b in gt]))], world, dev)[0]
+        del g
+
+    # ---- end to end through the public API, host buffers in and out ----
+    logits_pin = logits_h.pin_memory()
+    x_pin = x_h.pin_memory()
+    out_pin = torch.empty(T, H, dtype=torch.bfloat16).pin_memory()
+    e2e = []
+    with torch.cuda.stream(s):
+        for i in range(max(W, 3) + min(K, 100)):
+            flush.fill_(i)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(s)
+            logits.copy_(logits_pin, non_blocking=True)
+            x.copy_(x_pin, non_blocking=True)
+            step()
+            out_pin.copy_(out, non_blocking=True)
+            b.record(s)
+            if i >= max(W, 3):
+                e2e.append((a, b))
+        s.synchronize()
+    e2e_ms = max_over_ranks([float(np.mean([a.elapsed_time(b) for a, b in e2e]))], world, dev)[0]
+    h2d = logits_h.numel() * 4 + x_h.numel() * 2
+    d2h = out.numel() * 2
+
+    peak, peak_kind = load_peak()
+    n_gpus = world
+    value = n_gpus * nb["step"] / (ms_step * 1e-3) / 1e9
+    comb_gbs = nb["combine"] / (ms_combine * 1e-3) / 1e9
+    dc_ms = ms_layout + ms_dispatch + ms_combine
+    dc_bytes = nb["layout"] + nb["dispatch"] + nb["combine"]
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": n_gpus, "steps": K,
+            "warmup": W, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": cfg.describe(), "parallelism": f"replicas x{n_gpus}",
+                       "l2": "flushed before every step (512 MiB write outside the timed events)",
+                       "capacity": cap, "rows": rows, "timing": "CUDA events per stage, eager launches"},
+            "us_per_layer": ms_step * 1e3,
+            "stages_us": {"route": ms_route * 1e3, "layout": ms_layout * 1e3,
+                          "dispatch": ms_dispatch * 1e3, "combine": ms_combine * 1e3},
+            "dispatch_combine": {"us": dc_ms * 1e3, "bytes": dc_bytes,
+                                 "gbs": dc_bytes / (dc_ms * 1e-3) / 1e9,
+                                 "frac_of_8tbs": dc_bytes / (dc_ms * 1e-3) / 1e9 / SPEC_HBM_GBS,
+                                 "frac_of_measured": dc_bytes / (dc_ms * 1e-3) / 1e9 / peak},
+            "graph_us_per_layer": graph_ms * 1e3 if graph_ms else None,
+            "bytes_per_step": nb,
+            "roofline": {"bound": "hbm", "kernel": "k_combine_bf16", "achieved": comb_gbs,
+                         "peak": peak, "unit": "GB/s", "frac": comb_gbs / peak,
+                         "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+                         else "fallback 6650 GB/s",
+                         "traffic": combine_traffic(cfg.name),
+                         "algorithmic_bytes_per_launch": nb["combine"]},
+            "e2e": {"value": n_gpus * nb["step"] / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                    "us_per_step": e2e_ms * 1e3, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": KERNELS_PER_STEP * K,
+            "clocks": clocks,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(cfg)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        barrier(world, dev)
+        dist.destroy_process_group()
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", choices=sorted(inputs.CONFIGS), default="dsv3")
+    ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,230 @@
+"""combine_moe_route_08_b200 -- Mixture-of-Experts route, dispatch and combine
+on one B200 (sm_100a).
+
+A thin ctypes binding over ``libmoe_route.so`` (C ABI in
+``include/moe_route.h``): the functions here carry the C names, marshal
+torch CUDA tensors to device pointers and the current stream, allocate the
+outputs the caller did not pass (torch is used for device memory and
+streams only), and raise :class:`MoeError` on a non-OK status.  Every step of
+the path runs in the library's CUDA kernels; there is no CPU or torch
+fallback: importing this package fails if the library is missing.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "MoeError", "lib", "moe_status_string", "moe_route_topk", "moe_layout_workspace_bytes",
+    "moe_dispatch_layout", "moe_dispatch_bf16", "moe_dispatch_fp8", "moe_combine_bf16",
+    "moe_quantize_e4m3", "Workspace", "LIB_PATH",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_route.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m combine_moe_route_08_b200.build` "
+        "(nvcc, sm_100a). This package has no fallback path.")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+_P = ctypes.c_void_p
+_i32, _i64, _sz = ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+
+lib.moe_status_string.argtypes = [_i32]
+lib.moe_status_string.restype = ctypes.c_char_p
+lib.moe_route_topk.argtypes = [_P, _i32, _i32, _i32, _i32, _P, _P, _P]
+lib.moe_route_topk.restype = _i32
+lib.moe_layout_workspace_bytes.argtypes = [_i32, _i32, _i32, _i32]
+lib.moe_layout_workspace_bytes.restype = _sz
+lib.moe_dispatch_layout.argtypes = [_P, _i32, _i32, _i32, _i32, _i32, _i64, _P, _P, _P, _P, _P, _P,
+                                    _P, _sz, _P, _P]
+lib.moe_dispatch_layout.restype = _i32
+lib.moe_dispatch_bf16.argtypes = [_P, _i32, _i32, _i32, _P, _P, _i64, _P, _P]
+lib.moe_dispatch_bf16.restype = _i32
+lib.moe_dispatch_fp8.argtypes = [_P, _i32, _i32, _i32, _P, _P, _P, _i64, _P, _P]
+lib.moe_dispatch_fp8.restype = _i32
+lib.moe_combine_bf16.argtypes = [_P, _P, _P, _i32, _i32, _i32, _i64, _P, _P, _P]
+lib.moe_combine_bf16.restype = _i32
+lib.moe_quantize_e4m3.argtypes = [_P, _i64, _P, _P]
+lib.moe_quantize_e4m3.restype = _i32
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = 1
+MOE_ERR_UNSUPPORTED = 2
+MOE_ERR_CAPACITY = 3
+MOE_ERR_WORKSPACE = 4
+MOE_ERR_TIMEOUT = 5
+MOE_ERR_CUDA = 6
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {moe_status_string(status)}")
+
+
+def moe_status_string(status: int) -> str:
+    return lib.moe_status_string(status).decode()
+
+
+def _check(status: int, where: str):
+    if status != MOE_OK:
+        raise MoeError(status, where)
+
+
+def _ptr(t: torch.Tensor | None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return t.data_ptr() or None
+
+
+def _stream(stream) -> int | None:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream or None
+
+
+def _bits16(t: torch.Tensor) -> torch.Tensor:
+    if t.dtype not in (torch.bfloat16, torch.int16, torch.uint16):
+        raise ValueError(f"expected bf16 data, got {t.dtype}")
+    return t
+
+
+# ---------------------------------------------------------------------------
+# entry points
+# ---------------------------------------------------------------------------
+
+def moe_route_topk(logits: torch.Tensor, k: int, renormalize: bool = False,
+                   topk_idx: torch.Tensor | None = None, topk_w: torch.Tensor | None = None,
+                   stream=None):
+    """Router softmax + top-k.  logits fp32 [T][E] -> (topk_idx int32 [T][k],
+    topk_w fp32 [T][k])."""
+    assert logits.dtype == torch.float32 and logits.dim() == 2
+    T, E = logits.shape
+    dev = logits.device
+    if topk_idx is None:
+        topk_idx = torch.empty(T, k, dtype=torch.int32, device=dev)
+    if topk_w is None:
+        topk_w = torch.empty(T, k, dtype=torch.float32, device=dev)
+    _check(lib.moe_route_topk(_ptr(logits), T, E, k, int(renormalize), _ptr(topk_idx),
+                              _ptr(topk_w), _stream(stream)), "moe_route_topk")
+    return topk_idx, topk_w
+
+
+def moe_layout_workspace_bytes(T: int, k: int, E: int, R: int) -> int:
+    return int(lib.moe_layout_workspace_bytes(T, k, E, R))
+
+
+class Workspace:
+    """A zero-filled device workspace for moe_dispatch_layout, grown on demand."""
+
+    def __init__(self, device="cuda"):
+        self.device = torch.device(device)
+        self.buf = torch.zeros(0, dtype=torch.uint8, device=self.device)
+
+    def get(self, nbytes: int) -> torch.Tensor:
+        if self.buf.numel() < nbytes:
+            self.buf = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=self.device)
+        return self.buf
+
+
+_default_ws: dict[torch.device, Workspace] = {}
+
+
+def moe_dispatch_layout(topk_idx: torch.Tensor, E: int, R: int, capacity: int = 0,
+                        rows: int | None = None, out: dict | None = None,
+                        workspace: Workspace | None = None, dev_status: torch.Tensor | None = None,
+                        stream=None) -> dict:
+    """Counts, offsets and index maps.  Returns a dict with expert_counts [E],
+    expert_src_counts [E][R], rank_counts [R], expert_offsets [E+1],
+    dispatch_pos [T][k], recv_src [rows] (int32 CUDA tensors) and ``rows``."""
+    assert topk_idx.dtype == torch.int32 and topk_idx.dim() == 2
+    T, k = topk_idx.shape
+    dev = topk_idx.device
+    if rows is None:
+        rows = T * k if capacity == 0 else E * capacity
+    if out is None:
+        out = dict(
+            expert_counts=torch.empty(E, dtype=torch.int32, device=dev),
+            expert_src_counts=torch.empty(E, R, dtype=torch.int32, device=dev),
+            rank_counts=torch.empty(R, dtype=torch.int32, device=dev),
+            expert_offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
+            dispatch_pos=torch.empty(T, k, dtype=torch.int32, device=dev),
+            recv_src=torch.empty(max(rows, 1), dtype=torch.int32, device=dev),
+        )
+    if workspace is None:
+        workspace = _default_ws.setdefault(dev, Workspace(dev))
+    nbytes = moe_layout_workspace_bytes(T, k, E, R)
+    if nbytes == 0:
+        raise MoeError(MOE_ERR_INVALID_ARG, "moe_layout_workspace_bytes")
+    ws = workspace.get(nbytes)
+    _check(lib.moe_dispatch_layout(
+        _ptr(topk_idx), T, k, E, R, capacity, rows,
+        _ptr(out["expert_counts"]), _ptr(out["expert_src_counts"]), _ptr(out["rank_counts"]),
+        _ptr(out["expert_offsets"]), _ptr(out["dispatch_pos"]), _ptr(out["recv_src"]),
+        _ptr(ws), ws.numel(), _ptr(dev_status), _stream(stream)), "moe_dispatch_layout")
+    out["rows"] = rows
+    return out
+
+
+def moe_dispatch_bf16(x: torch.Tensor, dispatch_pos: torch.Tensor, rows: int,
+                      recv_x: torch.Tensor | None = None, dev_status: torch.Tensor | None = None,
+                      stream=None) -> torch.Tensor:
+    """recv_x[dispatch_pos[g, j]] = x[g]; x bf16 [T][H] -> recv_x bf16 [rows][H]."""
+    x = _bits16(x)
+    T, H = x.shape
+    k = dispatch_pos.shape[1]
+    if recv_x is None:
+        recv_x = torch.empty(rows, H, dtype=x.dtype, device=x.device)
+    _check(lib.moe_dispatch_bf16(_ptr(x), T, H, k, _ptr(dispatch_pos), _ptr(recv_x), rows,
+                                 _ptr(dev_status), _stream(stream)), "moe_dispatch_bf16")
+    return recv_x
+
+
+def moe_dispatch_fp8(x: torch.Tensor, dispatch_pos: torch.Tensor, rows: int,
+                     recv_q: torch.Tensor | None = None, recv_scale: torch.Tensor | None = None,
+                     dev_status: torch.Tensor | None = None, stream=None):
+    """FP8 e4m3 dispatch with 1x128 fp32 scales: x bf16 [T][H] ->
+    (recv_q uint8 [rows][H], recv_scale fp32 [rows][H/128])."""
+    x = _bits16(x)
+    T, H = x.shape
+    k = dispatch_pos.shape[1]
+    if recv_q is None:
+        recv_q = torch.empty(rows, H, dtype=torch.uint8, device=x.device)
+    if recv_scale is None:
+        recv_scale = torch.empty(rows, max(H // 128, 1), dtype=torch.float32, device=x.device)
+    _check(lib.moe_dispatch_fp8(_ptr(x), T, H, k, _ptr(dispatch_pos), _ptr(recv_q),
+                                _ptr(recv_scale), rows, _ptr(dev_status), _stream(stream)),
+           "moe_dispatch_fp8")
+    return recv_q, recv_scale
+
+
+def moe_combine_bf16(y: torch.Tensor, dispatch_pos: torch.Tensor, topk_w: torch.Tensor,
+                     out: torch.Tensor | None = None, dev_status: torch.Tensor | None = None,
+                     stream=None) -> torch.Tensor:
+    """out[g] = bf16(sum_j w[g, j] * y[dispatch_pos[g, j]]) in fp32, ascending j."""
+    y = _bits16(y)
+    rows, H = y.shape
+    T, k = dispatch_pos.shape
+    assert topk_w.dtype == torch.float32 and tuple(topk_w.shape) == (T, k)
+    if out is None:
+        out = torch.empty(T, H, dtype=y.dtype, device=y.device)
+    _check(lib.moe_combine_bf16(_ptr(y), _ptr(dispatch_pos), _ptr(topk_w), T, H, k, rows,
+                                _ptr(out), _ptr(dev_status), _stream(stream)), "moe_combine_bf16")
+    return out
+
+
+def moe_quantize_e4m3(v: torch.Tensor, q: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """q = e4m3(v) elementwise with the dispatch kernel's converter."""
+    assert v.dtype == torch.float32
+    if q is None:
+        q = torch.empty(v.shape, dtype=torch.uint8, device=v.device)
+    _check(lib.moe_quantize_e4m3(_ptr(v), v.numel(), _ptr(q), _stream(stream)), "moe_quantize_e4m3")
+    return q

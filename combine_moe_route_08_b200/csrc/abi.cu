@@ -1,0 +1,172 @@
+// abi.cu -- the extern "C" entry points of libmoe_route.so (declared, with
+// their sources and contracts, in include/moe_route.h).  Every argument is
+// checked here, on the host, before anything is enqueued; the kernels then
+// only see in-range sizes and aligned pointers.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kernels.cuh"
+#include "moe_route.h"
+
+namespace {
+
+constexpr int kMaxE = 1024;
+constexpr int kMaxK = 32;
+constexpr int64_t kMaxIndex = INT32_MAX;
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool valid_tk(int T, int k) { return T >= 0 && k >= 1 && k <= kMaxK && static_cast<int64_t>(T) * k < kMaxIndex; }
+
+int launched(cudaError_t err) { return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+cudaStream_t as_stream(void *s) { return static_cast<cudaStream_t>(s); }
+
+// Dispatch/combine: shared checks of the per-slot arguments.
+int check_rows_args(int T, int H, int k, const void *dispatch_pos, int64_t rows)
+{
+    if (!valid_tk(T, k) || H < 8 || H % 8 != 0 || rows < 0 || rows >= kMaxIndex)
+        return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (dispatch_pos == nullptr || !aligned(dispatch_pos, 4)))
+        return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *moe_status_string(int status)
+{
+    switch (status) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+    case MOE_ERR_CAPACITY: return "MOE_ERR_CAPACITY";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+    case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    default: return "MOE_ERR_UNKNOWN";
+    }
+}
+
+int moe_route_topk(const float *logits, int T, int E, int k, int renormalize, int32_t *topk_idx,
+                   float *topk_w, void *stream)
+{
+    if (!valid_tk(T, k) || E < 1 || E > kMaxE || k > E)
+        return MOE_ERR_INVALID_ARG;
+    if (T == 0)
+        return MOE_OK;
+    if (!logits || !topk_idx || !topk_w || !aligned(logits, 4) || !aligned(topk_idx, 4) ||
+        !aligned(topk_w, 4))
+        return MOE_ERR_INVALID_ARG;
+    return launched(moe::route_topk(logits, T, E, k, renormalize != 0, topk_idx, topk_w,
+                                    as_stream(stream)));
+}
+
+static bool valid_layout_sizes(int T, int k, int E, int R)
+{
+    return valid_tk(T, k) && E >= 1 && E <= kMaxE && k <= E && R >= 1 && R <= E && E % R == 0 &&
+           T % R == 0;
+}
+
+size_t moe_layout_workspace_bytes(int T, int k, int E, int R)
+{
+    if (!valid_layout_sizes(T, k, E, R))
+        return 0;
+    return moe::layout_workspace_bytes(moe::layout_geom(T, k, E, R));
+}
+
+int moe_dispatch_layout(const int32_t *topk_idx, int T, int k, int E, int R, int capacity,
+                        int64_t rows, int32_t *expert_counts, int32_t *expert_src_counts,
+                        int32_t *rank_counts, int32_t *expert_offsets, int32_t *dispatch_pos,
+                        int32_t *recv_src, void *workspace, size_t ws_bytes, int32_t *dev_status,
+                        void *stream)
+{
+    if (!valid_layout_sizes(T, k, E, R) || capacity < 0 || rows < 0 || rows >= kMaxIndex)
+        return MOE_ERR_INVALID_ARG;
+    const int64_t needed = (capacity == 0) ? static_cast<int64_t>(T) * k
+                                           : static_cast<int64_t>(E) * capacity;
+    if (rows < needed)
+        return MOE_ERR_INVALID_ARG;
+    const void *arrays[] = {expert_counts, expert_src_counts, rank_counts, expert_offsets};
+    for (const void *p : arrays)
+        if (!p || !aligned(p, 4))
+            return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!topk_idx || !dispatch_pos || !aligned(topk_idx, 4) || !aligned(dispatch_pos, 4)))
+        return MOE_ERR_INVALID_ARG;
+    if (rows > 0 && (!recv_src || !aligned(recv_src, 4)))
+        return MOE_ERR_INVALID_ARG;
+    if (dev_status && !aligned(dev_status, 4))
+        return MOE_ERR_INVALID_ARG;
+    const moe::LayoutGeom g = moe::layout_geom(T, k, E, R);
+    if (!workspace || !aligned(workspace, 256) || ws_bytes < moe::layout_workspace_bytes(g))
+        return MOE_ERR_WORKSPACE;
+    return launched(moe::dispatch_layout(topk_idx, g, capacity, rows, expert_counts,
+                                         expert_src_counts, rank_counts, expert_offsets,
+                                         dispatch_pos, recv_src, workspace, dev_status,
+                                         as_stream(stream)));
+}
+
+int moe_dispatch_bf16(const uint16_t *x, int T, int H, int k, const int32_t *dispatch_pos,
+                      uint16_t *recv_x, int64_t rows, int32_t *dev_status, void *stream)
+{
+    const int st = check_rows_args(T, H, k, dispatch_pos, rows);
+    if (st != MOE_OK)
+        return st;
+    if (T == 0)
+        return MOE_OK;
+    if (!x || !recv_x || !aligned(x, 16) || !aligned(recv_x, 16) ||
+        (dev_status && !aligned(dev_status, 4)))
+        return MOE_ERR_INVALID_ARG;
+    return launched(moe::dispatch_bf16(x, T, H, k, dispatch_pos, recv_x, rows, dev_status,
+                                       as_stream(stream)));
+}
+
+int moe_dispatch_fp8(const uint16_t *x, int T, int H, int k, const int32_t *dispatch_pos,
+                     uint8_t *recv_q, float *recv_scale, int64_t rows, int32_t *dev_status,
+                     void *stream)
+{
+    const int st = check_rows_args(T, H, k, dispatch_pos, rows);
+    if (st != MOE_OK)
+        return st;
+    if (H % 128 != 0)
+        return MOE_ERR_UNSUPPORTED;
+    if (T == 0)
+        return MOE_OK;
+    if (!x || !recv_q || !recv_scale || !aligned(x, 16) || !aligned(recv_q, 16) ||
+        !aligned(recv_scale, 4) || (dev_status && !aligned(dev_status, 4)))
+        return MOE_ERR_INVALID_ARG;
+    return launched(moe::dispatch_fp8(x, T, H, k, dispatch_pos, recv_q, recv_scale, rows,
+                                      dev_status, as_stream(stream)));
+}
+
+int moe_combine_bf16(const uint16_t *y, const int32_t *dispatch_pos, const float *topk_w, int T,
+                     int H, int k, int64_t rows, uint16_t *out, int32_t *dev_status, void *stream)
+{
+    const int st = check_rows_args(T, H, k, dispatch_pos, rows);
+    if (st != MOE_OK)
+        return st;
+    if (T == 0)
+        return MOE_OK;
+    if (!out || !topk_w || !aligned(out, 16) || !aligned(topk_w, 4) ||
+        (dev_status && !aligned(dev_status, 4)))
+        return MOE_ERR_INVALID_ARG;
+    if (rows > 0 && (!y || !aligned(y, 16)))
+        return MOE_ERR_INVALID_ARG;
+    return launched(moe::combine_bf16(y, dispatch_pos, topk_w, T, H, k, rows, out, dev_status,
+                                      as_stream(stream)));
+}
+
+int moe_quantize_e4m3(const float *v, int64_t n, uint8_t *q, void *stream)
+{
+    if (n < 0)
+        return MOE_ERR_INVALID_ARG;
+    if (n == 0)
+        return MOE_OK;
+    if (!v || !q || !aligned(v, 4))
+        return MOE_ERR_INVALID_ARG;
+    return launched(moe::quantize_e4m3(v, n, q, as_stream(stream)));
+}
+
+}  // extern "C"

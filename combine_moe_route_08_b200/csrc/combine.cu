@@ -1,0 +1,99 @@
+// combine.cu -- gather each token's k expert rows and form the router-
+// weighted sum in fp32, stored as bf16.
+//
+// "Efficient and portable mixture-of-experts communication", "Combinação":
+// the receiver reads the routing table to know which buffer to read and which
+// weight each expert contribution gets, and computes their weighted sum;
+// "Enabling trillion-parameter models on AWS EFA", "Dağıtım/Birleştirme
+// Gecikmesi": bf16 combine, accumulation only at the receiver.
+//
+// One CTA per token; a thread owns 8 consecutive channels (16 bytes of each
+// row).  All of a batch of up to 8 rows are loaded before any is used (8
+// independent 16-byte loads in flight per thread), then the sum runs in
+// ascending j with a separate binary32 multiply and add per term
+// (__fmul_rn / __fadd_rn are never contracted into an FMA), so the output
+// is bit-reproducible.
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kMaxK = 32;
+constexpr int kMaxThreads = 512;
+constexpr int kBatch = 8;
+
+__global__ void __launch_bounds__(kMaxThreads)
+    k_combine_bf16(const uint4 *__restrict__ y, const int32_t *__restrict__ dispatch_pos,
+                   const float *__restrict__ topk_w, int nvec, int k, int64_t rows,
+                   uint4 *__restrict__ out, int32_t *__restrict__ dev_status)
+{
+    __shared__ int32_t srow[kMaxK];
+    __shared__ float sw[kMaxK];
+    const int g = blockIdx.x;
+    if (threadIdx.x < k) {
+        int r = dispatch_pos[static_cast<size_t>(g) * k + threadIdx.x];
+        if (r < -1 || r >= rows) {
+            report(dev_status, MOE_ERR_INVALID_ARG);
+            r = -1;
+        }
+        srow[threadIdx.x] = r;
+        sw[threadIdx.x] = topk_w[static_cast<size_t>(g) * k + threadIdx.x];
+    }
+    __syncthreads();
+
+    for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
+        float acc[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+            acc[c] = 0.0f;
+        for (int j0 = 0; j0 < k; j0 += kBatch) {
+            uint4 d[kBatch];
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+                const int j = j0 + u;
+                const int r = (j < k) ? srow[j] : -1;
+                d[u] = (r >= 0) ? ld_stream_v4(y + static_cast<size_t>(r) * nvec + v)
+                                : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+                const int j = j0 + u;
+                if (j < k && srow[j] >= 0) {
+                    const float wj = sw[j];
+                    const uint32_t wds[4] = {d[u].x, d[u].y, d[u].z, d[u].w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        acc[2 * i] = __fadd_rn(acc[2 * i], __fmul_rn(wj, bf16_lo(wds[i])));
+                        acc[2 * i + 1] = __fadd_rn(acc[2 * i + 1], __fmul_rn(wj, bf16_hi(wds[i])));
+                    }
+                }
+            }
+        }
+        const uint4 o = make_uint4(bf16x2_rn(acc[0], acc[1]), bf16x2_rn(acc[2], acc[3]),
+                                   bf16x2_rn(acc[4], acc[5]), bf16x2_rn(acc[6], acc[7]));
+        st_stream_v4(out + static_cast<size_t>(g) * nvec + v, o);
+    }
+}
+
+int threads_for(int units)
+{
+    const int passes = ceil_div(units, kMaxThreads);
+    return round_up(ceil_div(units, passes), 32);
+}
+
+}  // namespace
+
+cudaError_t combine_bf16(const uint16_t *y, const int32_t *dispatch_pos, const float *topk_w,
+                         int T, int H, int k, int64_t rows, uint16_t *out, int32_t *dev_status,
+                         cudaStream_t s)
+{
+    const int nvec = H / 8;
+    k_combine_bf16<<<T, threads_for(nvec), 0, s>>>(reinterpret_cast<const uint4 *>(y), dispatch_pos,
+                                                   topk_w, nvec, k, rows,
+                                                   reinterpret_cast<uint4 *>(out), dev_status);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

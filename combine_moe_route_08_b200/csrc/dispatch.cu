@@ -1,0 +1,174 @@
+// dispatch.cu -- row scatter of each token into its k expert rows, as bf16 or
+// as OCP E4M3 with 1x128 fp32 block scales.
+//
+// "Enabling trillion-parameter models on AWS EFA", "Dağıtım ve Birleştirme":
+// tokens are packed into contiguous per-expert buffers at the offsets the
+// counts gave; "Dağıtım/Birleştirme Gecikmesi": block-scaled fp8 dispatch.
+// DeepSeek-V3 fragments: activations scaled per token per 128 channels, and
+// the wish to fuse the fp8 cast into the load from global memory -- here the
+// cast happens in registers between the single read of x and the k writes.
+//
+// One CTA per token: the row of x is read once (16-byte loads that skip L1),
+// quantised once, and written k times with 16-byte streaming stores, each
+// destination row by the whole CTA in one coalesced sweep.
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kMaxK = 32;
+constexpr int kMaxThreads = 512;
+
+// Load the token's k destination rows into shared memory; rows outside
+// [0, rows) other than -1 are reported and skipped.
+__device__ __forceinline__ void load_rows(const int32_t *__restrict__ dispatch_pos, int g, int k,
+                                          int64_t rows, int32_t *srow, int32_t *dev_status)
+{
+    if (threadIdx.x < k) {
+        int r = dispatch_pos[static_cast<size_t>(g) * k + threadIdx.x];
+        if (r < -1 || r >= rows) {
+            report(dev_status, MOE_ERR_INVALID_ARG);
+            r = -1;
+        }
+        srow[threadIdx.x] = r;
+    }
+    __syncthreads();
+}
+
+__global__ void __launch_bounds__(kMaxThreads)
+    k_dispatch_bf16(const uint4 *__restrict__ x, int nvec, int k,
+                    const int32_t *__restrict__ dispatch_pos, uint4 *__restrict__ recv_x,
+                    int64_t rows, int32_t *__restrict__ dev_status)
+{
+    __shared__ int32_t srow[kMaxK];
+    const int g = blockIdx.x;
+    load_rows(dispatch_pos, g, k, rows, srow, dev_status);
+    const uint4 *xr = x + static_cast<size_t>(g) * nvec;
+    for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
+        const uint4 d = ld_stream_v4(xr + v);
+        for (int j = 0; j < k; ++j) {
+            const int r = srow[j];
+            if (r >= 0)
+                st_stream_v4(recv_x + static_cast<size_t>(r) * nvec + v, d);
+        }
+    }
+}
+
+// Thread t of the token owns channels [16t, 16t + 16); the 8 threads of one
+// 128-channel block are 8 consecutive lanes, so the block's amax is a 3-step
+// xor shuffle.  s = amax / 448 and every x / s are IEEE binary32 divisions
+// (__fdiv_rn), then the hardware converts to e4m3 with RNE + saturation.
+__global__ void __launch_bounds__(kMaxThreads)
+    k_dispatch_fp8(const uint4 *__restrict__ x, int H, int k,
+                   const int32_t *__restrict__ dispatch_pos, uint8_t *__restrict__ recv_q,
+                   float *__restrict__ recv_scale, int64_t rows, int32_t *__restrict__ dev_status)
+{
+    __shared__ int32_t srow[kMaxK];
+    const int g = blockIdx.x;
+    load_rows(dispatch_pos, g, k, rows, srow, dev_status);
+    const int ngrp = H / 16;
+    const int S = H / 128;
+    const uint4 *xr = x + static_cast<size_t>(g) * (H / 8);
+
+    for (int t0 = 0; t0 < ngrp; t0 += blockDim.x) {  // CTA-uniform trips (shuffles)
+        const int t = t0 + threadIdx.x;
+        const bool act = t < ngrp;
+        uint4 a = make_uint4(0, 0, 0, 0), b = make_uint4(0, 0, 0, 0);
+        if (act) {
+            a = ld_stream_v4(xr + 2 * t);
+            b = ld_stream_v4(xr + 2 * t + 1);
+        }
+        const uint32_t wds[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+        float f[16];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            f[2 * i] = bf16_lo(wds[i]);
+            f[2 * i + 1] = bf16_hi(wds[i]);
+        }
+        float amax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            amax = fmaxf(amax, fabsf(f[i]));
+        amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 2));
+        amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 4));
+        const float s = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 448.0f);
+
+        uint32_t c[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t lo = e4m3x2(__fdiv_rn(f[4 * i], s), __fdiv_rn(f[4 * i + 1], s));
+            const uint32_t hi = e4m3x2(__fdiv_rn(f[4 * i + 2], s), __fdiv_rn(f[4 * i + 3], s));
+            c[i] = lo | (hi << 16);
+        }
+        const uint4 q = make_uint4(c[0], c[1], c[2], c[3]);
+        if (act) {
+            for (int j = 0; j < k; ++j) {
+                const int r = srow[j];
+                if (r < 0)
+                    continue;
+                st_stream_v4(recv_q + static_cast<size_t>(r) * H + 16 * t, q);
+                if ((t & 7) == 0)
+                    __stcs(recv_scale + static_cast<size_t>(r) * S + (t >> 3), s);
+            }
+        }
+    }
+}
+
+__global__ void k_quantize_e4m3(const float *__restrict__ v, int64_t n, uint8_t *__restrict__ q)
+{
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t p = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; 2 * p < n; p += stride) {
+        const int64_t i = 2 * p;
+        if (i + 1 < n) {
+            const uint32_t c = e4m3x2(v[i], v[i + 1]);
+            q[i] = static_cast<uint8_t>(c & 0xff);
+            q[i + 1] = static_cast<uint8_t>(c >> 8);
+        } else {
+            q[i] = static_cast<uint8_t>(e4m3x2(v[i], 0.0f) & 0xff);
+        }
+    }
+}
+
+int threads_for(int units)
+{
+    // fewest passes of at most kMaxThreads threads, then as few threads as
+    // cover the units in that many passes (a multiple of the warp size)
+    const int passes = ceil_div(units, kMaxThreads);
+    return round_up(ceil_div(units, passes), 32);
+}
+
+}  // namespace
+
+cudaError_t dispatch_bf16(const uint16_t *x, int T, int H, int k, const int32_t *dispatch_pos,
+                          uint16_t *recv_x, int64_t rows, int32_t *dev_status, cudaStream_t s)
+{
+    const int nvec = H / 8;
+    k_dispatch_bf16<<<T, threads_for(nvec), 0, s>>>(reinterpret_cast<const uint4 *>(x), nvec, k,
+                                                    dispatch_pos, reinterpret_cast<uint4 *>(recv_x),
+                                                    rows, dev_status);
+    return cudaGetLastError();
+}
+
+cudaError_t dispatch_fp8(const uint16_t *x, int T, int H, int k, const int32_t *dispatch_pos,
+                         uint8_t *recv_q, float *recv_scale, int64_t rows, int32_t *dev_status,
+                         cudaStream_t s)
+{
+    k_dispatch_fp8<<<T, threads_for(H / 16), 0, s>>>(reinterpret_cast<const uint4 *>(x), H, k,
+                                                     dispatch_pos, recv_q, recv_scale, rows,
+                                                     dev_status);
+    return cudaGetLastError();
+}
+
+cudaError_t quantize_e4m3(const float *v, int64_t n, uint8_t *q, cudaStream_t s)
+{
+    const int64_t pairs = (n + 1) / 2;
+    const int64_t blocks = (pairs + 255) / 256;
+    const int grid = static_cast<int>(blocks < 148 * 32 ? blocks : 148 * 32);
+    k_quantize_e4m3<<<grid, 256, 0, s>>>(v, n, q);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

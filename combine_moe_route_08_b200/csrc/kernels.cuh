@@ -1,0 +1,47 @@
+// kernels.cuh -- launchers of the libmoe_route kernels (internal to the
+// library; the public surface is include/moe_route.h).  Arguments arrive here
+// already validated by the C ABI layer.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace moe {
+
+// Layout geometry: tokens are cut into chunks that never straddle two logical
+// source ranks; one CTA counts, and later places, the slots of one chunk.
+struct LayoutGeom {
+    int T, k, E, R;
+    int Tr;       // tokens per logical source rank
+    int CT;       // tokens per chunk
+    int cpr;      // chunks per rank
+    int nchunks;  // R * cpr
+};
+
+LayoutGeom layout_geom(int T, int k, int E, int R);
+size_t layout_workspace_bytes(const LayoutGeom &g);
+
+cudaError_t route_topk(const float *logits, int T, int E, int k, int renormalize,
+                       int32_t *topk_idx, float *topk_w, cudaStream_t s);
+
+cudaError_t dispatch_layout(const int32_t *topk_idx, const LayoutGeom &g, int capacity,
+                            int64_t rows, int32_t *expert_counts, int32_t *expert_src_counts,
+                            int32_t *rank_counts, int32_t *expert_offsets,
+                            int32_t *dispatch_pos, int32_t *recv_src, void *workspace,
+                            int32_t *dev_status, cudaStream_t s);
+
+cudaError_t dispatch_bf16(const uint16_t *x, int T, int H, int k, const int32_t *dispatch_pos,
+                          uint16_t *recv_x, int64_t rows, int32_t *dev_status, cudaStream_t s);
+
+cudaError_t dispatch_fp8(const uint16_t *x, int T, int H, int k, const int32_t *dispatch_pos,
+                         uint8_t *recv_q, float *recv_scale, int64_t rows, int32_t *dev_status,
+                         cudaStream_t s);
+
+cudaError_t combine_bf16(const uint16_t *y, const int32_t *dispatch_pos, const float *topk_w,
+                         int T, int H, int k, int64_t rows, uint16_t *out, int32_t *dev_status,
+                         cudaStream_t s);
+
+cudaError_t quantize_e4m3(const float *v, int64_t n, uint8_t *q, cudaStream_t s);
+
+}  // namespace moe

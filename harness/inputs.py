@@ -116,6 +116,17 @@ def make_random_rows(rows: int, H: int, seed: int) -> torch.Tensor:
     return y.to(torch.bfloat16)
 
 
+def make_row_bank(H: int, seed: int, n: int = 4096) -> torch.Tensor:
+    """A bank of n random bf16 rows N(0, 1); large synthetic row sets (expert
+    outputs of the prefill workload) are drawn from it by bank_rows_map."""
+    return make_random_rows(n, H, seed)
+
+
+def bank_rows_map(rows: int, n: int = 4096) -> torch.Tensor:
+    """Row r of a bank-drawn set is bank row (r * 7919) mod n (int64)."""
+    return (torch.arange(rows, dtype=torch.int64) * 7919) % n
+
+
 def make_random_case(T: int, H: int, E: int, k: int, seed: int, tie_levels: int = 0):
     """A small random case: (logits fp32 [T][E], x bf16 [T][H]).  With
     ``tie_levels`` > 0 the logits are integers in [0, tie_levels) so that ties

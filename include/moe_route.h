@@ -1,0 +1,224 @@
+/*
+ * moe_route.h -- C ABI of libmoe_route.so: Mixture-of-Experts routing,
+ * dispatch and combine on one GPU (sm_100a).
+ *
+ * The path: router logits -> softmax + top-k (moe_route_topk) -> per-expert
+ * counts, offsets and index maps (moe_dispatch_layout) -> row scatter of each
+ * token into per-expert receive buffers, as bf16 or as e4m3 with 1x128 block
+ * scales (moe_dispatch_bf16 / moe_dispatch_fp8) -> [expert computation, not
+ * part of this library] -> gather of the expert outputs and the router-
+ * weighted sum per token (moe_combine_bf16).  Expert-parallel ranks are
+ * logical: R partitions of this one device's memory.  Nothing here talks to
+ * another GPU.
+ *
+ * Sources (page title, section):
+ *   "Efficient and portable mixture-of-experts communication" (Perplexity,
+ *     2025-04-02): "Introdução", "Despacho", "Combinação".
+ *   "Enabling trillion-parameter models on AWS EFA" (Perplexity, 2025-11-04):
+ *     "Gönderme ve Alma Arabellekleri", "Dağıtım ve Birleştirme",
+ *     "Dağıtım/Birleştirme Gecikmesi".
+ *   DeepSeek-V3 report fragments quoted on the other pages: 1x128 activation
+ *     tiles (per token per 128 channels), gating kept in original precision,
+ *     combine kept in BF16.
+ *
+ * Conventions shared by every entry point
+ *   - Every array pointer is a DEVICE pointer owned by the caller.  The
+ *     library allocates nothing, keeps no pointer after the call returns and
+ *     never synchronises the device.
+ *   - bf16 data are passed as their 16-bit patterns (uint16_t).
+ *   - `stream` is a cudaStream_t (CUstream) passed as void*; NULL is the
+ *     legacy default stream.  All device work is enqueued on it and runs
+ *     asynchronously.
+ *   - Argument errors are detected on the host before anything is enqueued
+ *     and returned synchronously (MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED).
+ *     A failed launch returns MOE_ERR_CUDA.
+ *   - Errors found by the kernels themselves (an expert id or row outside its
+ *     range, a capacity overflow) are written to *dev_status, an int32 in
+ *     device memory that the caller zeroes beforehand and reads after the
+ *     stream has been synchronised: the first error code written wins.  A
+ *     kernel that finds such an error skips the offending element; it never
+ *     traps and never touches memory outside the documented ranges.
+ *     dev_status may be NULL (errors are then skipped silently).
+ *   - Row data pointers (x, recv_x, recv_q, y, out) must be 16-byte aligned;
+ *     recv_scale, logits and the index arrays 4-byte aligned.
+ *   - Sizes: 0 <= T, 1 <= k <= min(E, 32), 1 <= E <= 1024, 1 <= R <= E,
+ *     E % R == 0, T % R == 0 (T/R tokens per logical source rank), H % 8 == 0
+ *     (bf16 paths), H % 128 == 0 (fp8 path), T*k < 2^31, rows < 2^31.
+ *
+ * Token g = r*(T/R) + t belongs to logical source rank r; expert e lives on
+ * logical destination rank e / (E/R).  Slot i = g*k + j is token g's j-th
+ * expert choice.
+ */
+#ifndef MOE_ROUTE_H
+#define MOE_ROUTE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum moe_status {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1, /* bad size, NULL or misaligned pointer, bad id/row */
+    MOE_ERR_UNSUPPORTED = 2, /* valid request this build does not support (fp8 with H % 128 != 0) */
+    MOE_ERR_CAPACITY = 3,    /* padded layout: a slot beyond its expert's capacity was dropped */
+    MOE_ERR_WORKSPACE = 4,   /* workspace too small or misaligned */
+    MOE_ERR_TIMEOUT = 5,     /* a bounded wait inside a kernel gave up */
+    MOE_ERR_CUDA = 6         /* a CUDA launch or runtime call failed */
+} moe_status_t;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *moe_status_string(int status);
+
+/*
+ * moe_route_topk -- router softmax and top-k selection.
+ * Follows "Efficient and portable mixture-of-experts communication",
+ * "Introdução": the router's small linear layer yields a probability
+ * distribution over experts; the top-K experts are chosen and each expert
+ * output is weighted by a weight derived from that distribution.  Gating stays
+ * in its original precision (DeepSeek-V3 fragments): fp32 in, fp32 out.
+ *
+ *   logits    [T][E] fp32, row-major (E contiguous).
+ *   topk_idx  [T][k] int32 out: the k experts first in the order (logit
+ *             descending, expert index ascending); -0.0 and +0.0 are equal.
+ *   topk_w    [T][k] fp32 out: p_e = exp(l_e - m) / sum_e' exp(l_e' - m),
+ *             m = max logit, evaluated in binary64 and rounded once to fp32;
+ *             with renormalize != 0 the sum runs over the k chosen experts
+ *             only (softmax restricted to the top-k).
+ * Logits must be finite.  T == 0 enqueues nothing.
+ */
+int moe_route_topk(const float *logits, int T, int E, int k, int renormalize,
+                   int32_t *topk_idx, float *topk_w, void *stream);
+
+/*
+ * Bytes of device workspace moe_dispatch_layout needs for (T, k, E, R);
+ * 0 on invalid sizes.  The workspace must be 256-byte aligned and
+ * ZERO-FILLED BEFORE ITS FIRST USE (cudaMemset); every call leaves it
+ * reusable.  One workspace must not serve two layout calls that may run at
+ * the same time.
+ */
+size_t moe_layout_workspace_bytes(int T, int k, int E, int R);
+
+/*
+ * moe_dispatch_layout -- counts, offsets and index maps for dispatch/combine.
+ * Follows "Enabling trillion-parameter models on AWS EFA", "Gönderme ve Alma
+ * Arabellekleri" (per-expert token counts first; then every sender knows
+ * where its writes go; receive buffers are contiguous) and "Dağıtım ve
+ * Birleştirme" (counts per expert, cumulative sums -> offsets that pack tokens
+ * into contiguous per-expert buffers); "Efficient and portable mixture-of-
+ * experts communication", "Despacho" (source rank, expert index and token
+ * index kept for combine; tokens grouped per expert).
+ *
+ *   topk_idx          [T][k] int32: expert of each slot.  -1 marks an empty
+ *                     slot (skipped, not counted); any other id outside
+ *                     [0, E) is skipped and reported as MOE_ERR_INVALID_ARG
+ *                     through dev_status.
+ *   capacity          0: packed.  Expert e owns rows [off_e, off_e + n_e),
+ *                     off = exclusive prefix sum of the counts in expert
+ *                     order, so logical rank r's region is the contiguous
+ *                     run of its experts [r*E/R, (r+1)*E/R).
+ *                     > 0: padded.  Expert e owns rows [e*cap, (e+1)*cap); a
+ *                     slot at position >= cap inside its expert is dropped
+ *                     (dispatch_pos = -1) and MOE_ERR_CAPACITY is reported
+ *                     through dev_status.
+ *   rows              length of recv_src; at least T*k (packed) or E*cap
+ *                     (padded).
+ *   Slots of one expert take consecutive rows in ascending slot index
+ *   i = g*k + j (ascending source rank, then token): the layout is
+ *   deterministic.
+ *   expert_counts     [E]    out: slots routed to e (dropped ones included).
+ *   expert_src_counts [E][R] out: slots routed to e from source rank r.
+ *   rank_counts       [R]    out: slots routed to rank r's experts.
+ *   expert_offsets    [E+1]  out: first row of expert e; [E] = packed total
+ *                     or E*cap.
+ *   dispatch_pos      [T][k] out: row of slot (g, j), or -1.
+ *   recv_src          [rows] out: the slot i = g*k + j a row holds, or -1
+ *                     for every row no slot fills.
+ *   workspace         see moe_layout_workspace_bytes; MOE_ERR_WORKSPACE if
+ *                     ws_bytes is too small or the pointer misaligned.
+ */
+int moe_dispatch_layout(const int32_t *topk_idx, int T, int k, int E, int R,
+                        int capacity, int64_t rows, int32_t *expert_counts,
+                        int32_t *expert_src_counts, int32_t *rank_counts,
+                        int32_t *expert_offsets, int32_t *dispatch_pos,
+                        int32_t *recv_src, void *workspace, size_t ws_bytes,
+                        int32_t *dev_status, void *stream);
+
+/*
+ * moe_dispatch_bf16 -- row scatter: recv_x[dispatch_pos[g][j]] = x[g].
+ * Follows "Enabling trillion-parameter models on AWS EFA", "Dağıtım ve
+ * Birleştirme" (tokens packed into contiguous per-expert buffers) and
+ * "Efficient and portable mixture-of-experts communication", "Despacho".
+ *
+ *   x             [T][H] bf16 bits, row-major.
+ *   dispatch_pos  [T][k] int32 rows from moe_dispatch_layout; -1 skipped; a
+ *                 row outside [0, rows) is skipped and reported
+ *                 (MOE_ERR_INVALID_ARG via dev_status).
+ *   recv_x        [rows][H] bf16 bits out; rows no slot targets are not
+ *                 written.
+ * T == 0 enqueues nothing.
+ */
+int moe_dispatch_bf16(const uint16_t *x, int T, int H, int k,
+                      const int32_t *dispatch_pos, uint16_t *recv_x,
+                      int64_t rows, int32_t *dev_status, void *stream);
+
+/*
+ * moe_dispatch_fp8 -- quantise each token once on 1x128 blocks and scatter
+ * the codes and scales to its k rows.
+ * Follows "Enabling trillion-parameter models on AWS EFA", "Dağıtım/
+ * Birleştirme Gecikmesi" (block-scaled fp8 dispatch) and the DeepSeek-V3
+ * fragments (activations scaled per token per 128 channels); the format is
+ * OCP E4M3 (max finite 448).
+ *
+ *   For each token g and block b of 128 channels:
+ *     amax = max |x|, s = amax / 448 (IEEE binary32 division; s = 1 when
+ *     amax == 0), q = e4m3(x / s) (binary32 division, round to nearest even,
+ *     saturating at +-448).
+ *   recv_q      [rows][H] uint8 e4m3 codes out.
+ *   recv_scale  [rows][H/128] fp32 scales out (dequantised value = e4m3(q)*s).
+ *   dispatch_pos, rows, dev_status: as for moe_dispatch_bf16.
+ * H % 128 != 0 returns MOE_ERR_UNSUPPORTED.  T == 0 enqueues nothing.
+ */
+int moe_dispatch_fp8(const uint16_t *x, int T, int H, int k,
+                     const int32_t *dispatch_pos, uint8_t *recv_q,
+                     float *recv_scale, int64_t rows, int32_t *dev_status,
+                     void *stream);
+
+/*
+ * moe_combine_bf16 -- gather each token's k expert outputs and form the
+ * router-weighted sum.
+ * Follows "Efficient and portable mixture-of-experts communication",
+ * "Combinação" (the receiver reads the routing table for which row to read
+ * and which weight to give it, and computes the weighted sum of the expert
+ * contributions) and "Enabling trillion-parameter models on AWS EFA",
+ * "Dağıtım/Birleştirme Gecikmesi" (bf16 combine; accumulation only at the
+ * receiver).
+ *
+ *   out[g][h] = bf16_rne( acc ), acc = 0; for j = 0..k-1 ascending, slots
+ *   with dispatch_pos == -1 skipped: acc = acc + (topk_w[g][j] *
+ *   y[dispatch_pos[g][j]][h]), one binary32 multiply and one binary32 add
+ *   per term (no fused multiply-add), so the result is bit-reproducible.
+ *   y       [rows][H] bf16 bits (expert outputs, rows as laid out).
+ *   topk_w  [T][k] fp32.
+ *   out     [T][H] bf16 bits out.
+ * T == 0 enqueues nothing.
+ */
+int moe_combine_bf16(const uint16_t *y, const int32_t *dispatch_pos,
+                     const float *topk_w, int T, int H, int k, int64_t rows,
+                     uint16_t *out, int32_t *dev_status, void *stream);
+
+/*
+ * moe_quantize_e4m3 -- q[i] = e4m3(v[i]) with the converter moe_dispatch_fp8
+ * uses (round to nearest even, saturating at +-448, NaN -> 0x7F).  Exposed
+ * so the converter can be checked on every binary32 bit pattern.
+ *   v  [n] fp32 (4-byte aligned);  q  [n] uint8 out.
+ */
+int moe_quantize_e4m3(const float *v, int64_t n, uint8_t *q, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_ROUTE_H */

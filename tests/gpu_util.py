@@ -1,0 +1,77 @@
+"""Helpers shared by the GPU tests: cached seeded inputs and oracle results
+per workload, tolerance checks.  Everything the oracle sees comes from the
+harness generators (CPU), never from the CUDA path."""
+from __future__ import annotations
+
+import functools
+
+import numpy as np
+import torch
+
+import oracle
+from harness import experts, inputs
+
+U = 2.0 ** -24
+
+
+def to_dev(a, dtype=None):
+    t = torch.from_numpy(np.ascontiguousarray(a)) if isinstance(a, np.ndarray) else a
+    if dtype is not None:
+        t = t.to(dtype)
+    return t.cuda()
+
+
+def ulp_bf16(a: np.ndarray) -> np.ndarray:
+    """Spacing of bf16 at |a|: 2^(max(floor(log2|a|), -126) - 7)."""
+    a = np.abs(a.astype(np.float64))
+    e = np.floor(np.log2(np.maximum(a, 2.0 ** -126)))
+    return 2.0 ** (np.maximum(e, -126) - 7)
+
+
+def ulp_f32(a: np.ndarray) -> np.ndarray:
+    return np.spacing(np.abs(a.astype(np.float32))).astype(np.float64)
+
+
+def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
+    return inputs.bits_to_bf16(bits).float().numpy().astype(np.float64)
+
+
+def gpu_bits(t: torch.Tensor) -> np.ndarray:
+    """bf16 CUDA tensor -> numpy uint16 bit patterns."""
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+@functools.lru_cache(maxsize=5)
+def workload(name: str):
+    """Seeded inputs of a workload and the oracle's route and layout on them."""
+    cfg = inputs.CONFIGS[name]
+    logits = inputs.make_logits(cfg)
+    x = inputs.make_x(cfg)
+    idx, w = oracle.route(logits.numpy(), cfg.k)
+    packed = oracle.layout(idx, cfg.E, cfg.R)
+    cap = int(packed["expert_counts"].max()) if cfg.layout == "padded" else 0
+    lay = oracle.layout(idx, cfg.E, cfg.R, cap) if cap else packed
+    return dict(cfg=cfg, logits=logits, x=x, x_bits=inputs.bf16_bits(x), idx=idx, w=w,
+                layout=lay, cap=cap, rows=int(lay["recv_src"].shape[0]))
+
+
+def stand_in_y_cpu(wl, recv_bits=None, recv_q=None, recv_scale=None):
+    """The workload's stand-in expert applied on the CPU to oracle outputs."""
+    cfg = wl["cfg"]
+    if cfg.expert == "identity":
+        return recv_bits
+    if cfg.expert == "affine":
+        noise = inputs.make_expert_noise(cfg, recv_bits.shape[0])
+        return inputs.bf16_bits(experts.affine(inputs.bits_to_bf16(recv_bits), noise))
+    y = experts.dequantise(torch.from_numpy(recv_q), torch.from_numpy(recv_scale))
+    return inputs.bf16_bits(y)
+
+
+def check_combine(out_bits: np.ndarray, acc: np.ndarray, oracle_out_bits: np.ndarray, where: str):
+    """The contract: |out - acc| <= 1 bf16 ulp of the oracle's fp32 sum.
+    Returns the fraction of outputs bit-identical to the oracle's bf16."""
+    out = bf16_to_f64(out_bits)
+    err = np.abs(out - acc.astype(np.float64))
+    bad = err > ulp_bf16(acc)
+    assert not bad.any(), f"{where}: {int(bad.sum())} outputs beyond 1 bf16 ulp, max err {err.max()}"
+    return float(np.mean(out_bits == oracle_out_bits))

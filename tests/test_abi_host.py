@@ -1,0 +1,124 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every entry point include/moe_route.h declares, and rejects bad arguments
+synchronously, before anything touches the CUDA runtime."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "moe_route.h")
+
+# fake device addresses: never dereferenced, because every call below must
+# fail validation (or be a no-op) before a kernel could be launched
+A16 = 0x10000
+A4 = 0x10004
+
+
+@pytest.fixture(scope="module")
+def moe():
+    from combine_moe_route_08_b200 import build
+    build.build()
+    import combine_moe_route_08_b200 as m
+    return m
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_path():
+    names = declared_functions()
+    for want in ["moe_route_topk", "moe_layout_workspace_bytes", "moe_dispatch_layout",
+                 "moe_dispatch_bf16", "moe_dispatch_fp8", "moe_combine_bf16",
+                 "moe_status_string", "moe_quantize_e4m3"]:
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(moe):
+    for name in declared_functions():
+        assert hasattr(moe.lib, name), name
+        assert callable(getattr(moe.lib, name))
+
+
+def test_python_binding_has_the_c_names(moe):
+    for name in declared_functions():
+        assert callable(getattr(moe, name)), name
+
+
+def test_status_strings(moe):
+    assert moe.moe_status_string(0) == "MOE_OK"
+    assert moe.moe_status_string(3) == "MOE_ERR_CAPACITY"
+    assert moe.moe_status_string(99) == "MOE_ERR_UNKNOWN"
+
+
+def test_workspace_bytes(moe):
+    # dsv3-like decode: 32 ranks of 128 tokens, one chunk per rank
+    assert moe.moe_layout_workspace_bytes(4096, 8, 256, 32) == 256 + 32 * 256 * 4
+    # prefill-like: 4096 tokens per rank cut into chunks of 256 tokens
+    assert moe.moe_layout_workspace_bytes(32768, 8, 256, 8) == 256 + 128 * 256 * 4
+    assert moe.moe_layout_workspace_bytes(0, 2, 8, 2) == 256 + 256  # histogram rounded up to 256 B
+    for bad in [(-1, 2, 8, 2), (64, 0, 8, 2), (64, 33, 64, 2), (64, 2, 8, 3), (63, 2, 8, 2),
+                (64, 9, 8, 2), (64, 2, 2048, 2)]:
+        assert moe.moe_layout_workspace_bytes(*bad) == 0, bad
+
+
+def test_route_rejects_bad_arguments(moe):
+    f = moe.lib.moe_route_topk
+    assert f(A4, 4, 8, 0, 0, A4, A4, None) == moe.MOE_ERR_INVALID_ARG      # k = 0
+    assert f(A4, 4, 8, 9, 0, A4, A4, None) == moe.MOE_ERR_INVALID_ARG      # k > E
+    assert f(A4, 4, 2048, 8, 0, A4, A4, None) == moe.MOE_ERR_INVALID_ARG   # E > 1024
+    assert f(None, 4, 8, 2, 0, A4, A4, None) == moe.MOE_ERR_INVALID_ARG    # NULL
+    assert f(A4 + 1, 4, 8, 2, 0, A4, A4, None) == moe.MOE_ERR_INVALID_ARG  # misaligned
+    assert f(None, 0, 8, 2, 0, None, None, None) == moe.MOE_OK             # T = 0: no-op
+
+
+def test_layout_rejects_bad_arguments(moe):
+    f = moe.lib.moe_dispatch_layout
+    ws = moe.moe_layout_workspace_bytes(8, 2, 4, 2)
+    ok = dict(idx=A4, T=8, k=2, E=4, R=2, cap=0, rows=16, ws=A16 * 16, wsb=ws)
+
+    def call(**kw):
+        a = {**ok, **kw}
+        return f(a["idx"], a["T"], a["k"], a["E"], a["R"], a["cap"], a["rows"], A4, A4, A4, A4,
+                 A4, A4, a["ws"], a["wsb"], None, None)
+
+    assert call(R=3) == moe.MOE_ERR_INVALID_ARG            # E % R != 0
+    assert call(T=7) == moe.MOE_ERR_INVALID_ARG            # T % R != 0
+    assert call(rows=15) == moe.MOE_ERR_INVALID_ARG        # fewer rows than T*k
+    assert call(cap=5, rows=19) == moe.MOE_ERR_INVALID_ARG  # fewer rows than E*cap
+    assert call(cap=-1) == moe.MOE_ERR_INVALID_ARG
+    assert call(idx=None) == moe.MOE_ERR_INVALID_ARG
+    assert call(wsb=ws - 4) == moe.MOE_ERR_WORKSPACE
+    assert call(ws=A16 + 16) == moe.MOE_ERR_WORKSPACE      # not 256-byte aligned
+    assert call(ws=None) == moe.MOE_ERR_WORKSPACE
+
+
+def test_dispatch_and_combine_reject_bad_arguments(moe):
+    d16, d8, c16 = moe.lib.moe_dispatch_bf16, moe.lib.moe_dispatch_fp8, moe.lib.moe_combine_bf16
+    assert d16(A16, 4, 100, 2, A4, A16, 8, None, None) == moe.MOE_ERR_INVALID_ARG   # H % 8
+    assert d16(A16 + 8, 4, 256, 2, A4, A16, 8, None, None) == moe.MOE_ERR_INVALID_ARG  # x align
+    assert d16(A16, 4, 256, 0, A4, A16, 8, None, None) == moe.MOE_ERR_INVALID_ARG   # k = 0
+    assert d16(A16, 4, 256, 2, None, A16, 8, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert d16(None, 0, 256, 2, None, None, 0, None, None) == moe.MOE_OK            # T = 0
+    assert d8(A16, 4, 200, 2, A4, A16, A4, 8, None, None) == moe.MOE_ERR_UNSUPPORTED  # H % 128
+    assert d8(A16, 4, 256, 2, A4, A16 + 4, A4, 8, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert d8(A16, 4, 256, 2, A4, A16, A4 + 1, 8, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert c16(A16, A4, A4, 4, 256, 2, 8, A16 + 2, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert c16(A16, A4, None, 4, 256, 2, 8, A16, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert c16(A16, A4, A4, 4, 256, 2, -1, A16, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert c16(None, None, None, 0, 256, 2, 0, None, None, None) == moe.MOE_OK
+    assert moe.lib.moe_quantize_e4m3(A4, -1, A16, None) == moe.MOE_ERR_INVALID_ARG
+    assert moe.lib.moe_quantize_e4m3(None, 0, None, None) == moe.MOE_OK
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_valid_call_without_a_device_reports_cuda_error(moe):
+    # arguments pass validation; the launch fails (no device) and is reported
+    st = moe.lib.moe_route_topk(A4, 4, 8, 2, 0, A4, A4, None)
+    assert st == moe.MOE_ERR_CUDA

@@ -1,0 +1,79 @@
+"""Host-side pieces of bench.py, on the CPU: the algorithmic byte counts, the
+max-over-ranks reduction with two gloo ranks, and the reference arm's
+rank-0-only output under a two-rank launch."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+from conftest import ROOT
+
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+from harness import inputs  # noqa: E402
+
+
+def test_algorithmic_bytes_dsv3():
+    cfg = inputs.CONFIGS["dsv3"]
+    nb = bench.algorithmic_bytes(cfg, rows=cfg.T * cfg.k, kept=cfg.T * cfg.k)
+    T, H, k = 4096, 7168, 8
+    assert nb["dispatch"] == T * H * 2 + T * k * 4 + T * k * H + T * k * 56 * 4     # 301.07 MB
+    assert nb["combine"] == T * k * H * 2 + T * k * 8 + T * H * 2                   # 528.74 MB
+    assert nb["route"] == T * 256 * 4 + T * k * 8
+    assert abs(nb["dispatch"] / 1e6 - 301.07) < 0.01
+    assert abs(nb["combine"] / 1e6 - 528.74) < 0.01
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), WORLD_SIZE=str(world),
+                      RANK=str(rank), LOCAL_RANK=str(rank))
+    import torch.distributed as dist
+    bench.init_dist(world, "gloo")
+    got = bench.max_over_ranks([1.0 + rank, 10.0 - rank, 0.5 * rank], world, torch.device("cpu"))
+    bench.barrier(world)
+    q.put((rank, got))
+    dist.destroy_process_group()
+
+
+def test_max_over_ranks_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = dict(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert res[0] == res[1] == [2.0, 10.0, 0.5]
+
+
+@pytest.mark.parametrize("world", [1, 2])
+def test_reference_arm_prints_one_line_from_rank0(world, tmp_path):
+    outs = []
+    for rank in range(world):
+        env = dict(os.environ, WORLD_SIZE=str(world), RANK=str(rank), LOCAL_RANK=str(rank),
+                   MASTER_ADDR="127.0.0.1")
+        p = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                            "--config", "tiny", "--steps", "3", "--warmup", "3",
+                            "--gpus", str(world)],
+                           env=env, capture_output=True, text=True, timeout=300)
+        assert p.returncode == 0, p.stderr
+        outs.append(p.stdout.strip())
+    assert outs[0] and all(o == "" for o in outs[1:])
+    line = json.loads(outs[0])
+    assert line["impl"] == "reference" and line["unit"] == "GB/s" and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle"
+    assert line["e2e"]["h2d_bytes_per_step"] == 0

@@ -1,0 +1,240 @@
+"""Edge cases of the CUDA path against the oracle: empty and ragged inputs,
+maximum sizes (E = 1024, k = 32), masked and invalid expert ids, capacity
+overflow, out-of-range rows, extreme fp8 inputs, workspace reuse,
+determinism, and the e4m3 converter on every binary32 bit pattern."""
+import concurrent.futures as cf
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from harness import inputs
+from gpu_util import bf16_to_f64, check_combine, gpu_bits, to_dev, ulp_f32
+
+pytestmark = pytest.mark.gpu
+
+LAYOUT_KEYS = ["expert_counts", "expert_src_counts", "rank_counts", "expert_offsets",
+               "dispatch_pos", "recv_src"]
+
+
+@pytest.fixture(scope="module")
+def moe():
+    import combine_moe_route_08_b200 as m
+    return m
+
+
+def _status():
+    return torch.zeros(1, dtype=torch.int32, device="cuda")
+
+
+def _full_path_vs_oracle(moe, logits, x, E, k, R, cap=0, fp8=True, idx_override=None):
+    """Every stage on the GPU against the oracle on the same inputs."""
+    T, H = x.shape
+    idx_o, w_o = oracle.route(logits.numpy(), k)
+    if T:
+        idx, w = moe.moe_route_topk(to_dev(logits), k)
+        torch.cuda.synchronize()
+        assert np.array_equal(idx.cpu().numpy(), idx_o)
+        assert np.all(np.abs(w.cpu().numpy().astype(np.float64) - w_o) <= ulp_f32(w_o))
+    if idx_override is not None:
+        idx_o = idx_override
+    lay_o = oracle.layout(idx_o, E, R, cap)
+    rows = lay_o["recv_src"].shape[0]
+    st = _status()
+    lay = moe.moe_dispatch_layout(to_dev(idx_o.reshape(T, k)), E, R, capacity=cap, rows=rows,
+                                  dev_status=st)
+    torch.cuda.synchronize()
+    for key in LAYOUT_KEYS:
+        assert np.array_equal(lay[key].cpu().numpy(), lay_o[key].reshape(lay[key].shape)), key
+    want_status = {oracle.OK: 0, oracle.ERR_CAPACITY: moe.MOE_ERR_CAPACITY,
+                   oracle.ERR_INVALID: moe.MOE_ERR_INVALID_ARG}[lay_o["status"]]
+    assert st.item() == want_status
+    pos_o = lay_o["dispatch_pos"]
+    filled = lay_o["recv_src"] >= 0
+    xb = inputs.bf16_bits(x)
+    if fp8:
+        q, s = moe.moe_dispatch_fp8(to_dev(x), lay["dispatch_pos"], rows)
+        qo, so = oracle.dispatch_fp8(xb, pos_o, rows)
+        torch.cuda.synchronize()
+        assert np.array_equal(q.cpu().numpy()[filled], qo[filled])
+        assert np.array_equal(s.cpu().numpy()[filled].view(np.uint32), so[filled].view(np.uint32))
+    else:
+        r = moe.moe_dispatch_bf16(to_dev(x), lay["dispatch_pos"], rows)
+        ro = oracle.dispatch_bf16(xb, pos_o, rows)
+        torch.cuda.synchronize()
+        assert np.array_equal(gpu_bits(r)[filled], ro[filled])
+    y = inputs.make_random_rows(rows, H, seed=T * 31 + E)
+    acc, out_o = oracle.combine(inputs.bf16_bits(y), pos_o, w_o)
+    out = moe.moe_combine_bf16(to_dev(y), lay["dispatch_pos"], to_dev(w_o))
+    torch.cuda.synchronize()
+    if T:
+        assert check_combine(gpu_bits(out), acc, out_o, "edge") == 1.0
+
+
+@pytest.mark.parametrize("T,E,k,R,H,cap", [
+    (1, 4, 1, 1, 128, 0),
+    (7, 8, 2, 1, 256, 0),
+    (33, 64, 8, 1, 384, 0),
+    (257, 384, 8, 1, 7168, 0),       # ragged against the 256-token chunk
+    (300, 16, 16, 2, 128, 0),        # k = E
+    (300, 16, 16, 2, 128, 300),      # k = E, padded, cap = T
+    (520, 1024, 32, 8, 128, 0),      # maximum E and k
+    (4096 + 44, 32, 4, 4, 256, 0),   # several chunks per rank, ragged
+    (1200, 24, 6, 3, 512, 120),      # padded with drops
+])
+def test_random_shapes_all_stages(moe, T, E, k, R, H, cap):
+    logits, x = inputs.make_random_case(T, H, E, k, seed=T + E + k + H)
+    _full_path_vs_oracle(moe, logits, x, E, k, R, cap=cap, fp8=(H % 128 == 0))
+    _full_path_vs_oracle(moe, logits, x, E, k, R, cap=cap, fp8=False)
+
+
+def test_ties_in_logits(moe):
+    logits, x = inputs.make_random_case(200, 256, 64, 8, seed=3, tie_levels=3)
+    _full_path_vs_oracle(moe, logits, x, 64, 8, 4)
+
+
+def test_masked_and_invalid_ids(moe):
+    T, E, k, R, H = 96, 16, 4, 4, 256
+    logits, x = inputs.make_random_case(T, H, E, k, seed=21)
+    idx, _ = oracle.route(logits.numpy(), k)
+    rng = np.random.default_rng(4)
+    idx[rng.random(idx.shape) < 0.2] = -1
+    _full_path_vs_oracle(moe, logits, x, E, k, R, idx_override=idx.copy())
+    idx[3, 1] = E + 5
+    idx[7, 0] = -9
+    _full_path_vs_oracle(moe, logits, x, E, k, R, idx_override=idx.copy())
+
+
+def test_empty_token_set(moe):
+    E, k, R, H = 8, 2, 2, 256
+    for cap in [0, 3]:
+        rows = 0 if cap == 0 else E * cap + 2
+        idx = torch.empty(0, k, dtype=torch.int32, device="cuda")
+        lay = moe.moe_dispatch_layout(idx, E, R, capacity=cap, rows=rows)
+        torch.cuda.synchronize()
+        assert lay["expert_counts"].sum().item() == 0
+        assert lay["expert_src_counts"].sum().item() == 0
+        assert lay["rank_counts"].sum().item() == 0
+        assert lay["expert_offsets"].cpu().tolist() == [e * cap for e in range(E + 1)]
+        if rows:
+            assert torch.all(lay["recv_src"][:rows] == -1)
+    x = torch.empty(0, H, dtype=torch.bfloat16, device="cuda")
+    pos = torch.empty(0, k, dtype=torch.int32, device="cuda")
+    moe.moe_dispatch_bf16(x, pos, 0, recv_x=torch.empty(1, H, dtype=torch.bfloat16, device="cuda"))
+    moe.moe_dispatch_fp8(x, pos, 0, recv_q=torch.empty(1, H, dtype=torch.uint8, device="cuda"),
+                         recv_scale=torch.empty(1, 2, device="cuda"))
+    moe.moe_combine_bf16(torch.empty(1, H, dtype=torch.bfloat16, device="cuda"), pos,
+                         torch.empty(0, k, device="cuda"))
+    moe.moe_route_topk(torch.empty(0, E, device="cuda"), k)
+    torch.cuda.synchronize()
+
+
+def test_out_of_range_rows_are_skipped_and_reported(moe):
+    T, H, k, rows = 16, 256, 2, 32
+    x = inputs.make_random_rows(T, H, seed=5)
+    pos = np.arange(T * k, dtype=np.int32).reshape(T, k)
+    pos[2, 1] = rows          # one past the end
+    pos[5, 0] = -3            # below -1
+    pos[9, 1] = 1 << 30       # far away
+    guard = 4
+    buf = torch.zeros(rows + guard, H, dtype=torch.bfloat16, device="cuda")
+    st = _status()
+    moe.moe_dispatch_bf16(to_dev(x), to_dev(pos), rows, recv_x=buf[:rows], dev_status=st)
+    torch.cuda.synchronize()
+    assert st.item() == moe.MOE_ERR_INVALID_ARG
+    assert torch.all(buf[rows:] == 0)
+    clean = pos.copy()
+    clean[clean >= rows] = -1
+    clean[clean < -1] = -1
+    want = oracle.dispatch_bf16(inputs.bf16_bits(x), clean, rows)
+    got = gpu_bits(buf[:rows])
+    rows_ok = sorted(set(clean[clean >= 0].tolist()))
+    assert np.array_equal(got[rows_ok], want[rows_ok])
+    for fn in ("fp8", "combine"):
+        st = _status()
+        if fn == "fp8":
+            qb = torch.zeros(rows + guard, H, dtype=torch.uint8, device="cuda")
+            moe.moe_dispatch_fp8(to_dev(x), to_dev(pos), rows, recv_q=qb[:rows],
+                                 recv_scale=torch.zeros(rows, H // 128, device="cuda"), dev_status=st)
+            torch.cuda.synchronize()
+            assert torch.all(qb[rows:] == 0)
+        else:
+            w = np.ones((T, k), np.float32)
+            out = moe.moe_combine_bf16(buf[:rows], to_dev(pos), to_dev(w), dev_status=st)
+            y = gpu_bits(buf[:rows])
+            acc, out_o = oracle.combine(y, clean, w)
+            torch.cuda.synchronize()
+            check_combine(gpu_bits(out), acc, out_o, "bad rows")
+        assert st.item() == moe.MOE_ERR_INVALID_ARG
+
+
+def test_fp8_extreme_values(moe):
+    """All-zero blocks, signed zeros, bf16 subnormals, the largest bf16
+    magnitudes and single spikes, quantised exactly like the oracle."""
+    H, T = 1024, 12
+    x = torch.zeros(T, H, dtype=torch.float32)
+    x[1] = -0.0
+    x[2] = torch.linspace(-1e-38, 1e-38, H)                 # bf16 subnormals
+    x[3] = 3.0e38
+    x[3, ::3] = -3.3e38
+    x[4, 5] = 1.0                                            # one spike per row
+    x[5] = torch.randn(H) * 1e-30
+    x[6] = torch.randn(H) * 1e30
+    x[7, :128] = 448.0
+    x[8] = torch.arange(H, dtype=torch.float32) - 500
+    x[9:] = torch.randn(T - 9, H)
+    xb = x.to(torch.bfloat16)
+    pos = np.arange(T * 2, dtype=np.int32).reshape(T, 2)
+    q, s = moe.moe_dispatch_fp8(to_dev(xb), to_dev(pos), T * 2)
+    qo, so = oracle.dispatch_fp8(inputs.bf16_bits(xb), pos, T * 2)
+    torch.cuda.synchronize()
+    assert np.array_equal(q.cpu().numpy(), qo)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), so.view(np.uint32))
+
+
+def test_workspace_reuse_and_determinism(moe):
+    ws = moe.Workspace("cuda")
+    cfgs = [(4096, 256, 8, 32), (64, 8, 2, 2), (32768, 256, 8, 8), (4096, 256, 8, 32)]
+    first = {}
+    for T, E, k, R in cfgs:
+        logits, _ = inputs.make_random_case(T, 8, E, k, seed=T + E)
+        idx_o, _ = oracle.route(logits.numpy(), k)
+        want = oracle.layout(idx_o, E, R)
+        idx = to_dev(idx_o)
+        for rep in range(2):
+            lay = moe.moe_dispatch_layout(idx, E, R, workspace=ws)
+            torch.cuda.synchronize()
+            for key in LAYOUT_KEYS:
+                assert np.array_equal(lay[key].cpu().numpy(), want[key].reshape(lay[key].shape))
+        first.setdefault((T, E), lay["dispatch_pos"].clone())
+    # the workspace's ticket is back at zero after every call
+    assert int(ws.buf[:4].view(torch.int32).item()) == 0
+
+
+def _mismatch_range(args):
+    first_bits, codes = args
+    return oracle.e4m3_count_mismatch(first_bits, codes)
+
+
+def test_e4m3_converter_every_binary32_pattern(moe):
+    """The dispatch kernel's converter on all 2^32 bit patterns against the
+    oracle's encoder (written from the OCP OFP8 definition)."""
+    oracle.build()
+    chunk = 1 << 28
+    workers = max(1, min(16, os.cpu_count() or 1))
+    bad_total = 0
+    with cf.ThreadPoolExecutor(workers) as pool:   # ctypes calls release the GIL
+        for start in range(0, 1 << 32, chunk):
+            bits = torch.arange(start, start + chunk, dtype=torch.int64, device="cuda")
+            v = bits.to(torch.int32).view(torch.float32) if start < (1 << 31) else \
+                (bits - (1 << 32)).to(torch.int32).view(torch.float32)
+            codes = moe.moe_quantize_e4m3(v).cpu().numpy()
+            del bits, v
+            part = chunk // workers
+            jobs = [(start + i * part, codes[i * part:(i + 1) * part if i < workers - 1 else chunk])
+                    for i in range(workers)]
+            for n_bad, first_bad in pool.map(_mismatch_range, jobs):
+                bad_total += n_bad
+    assert bad_total == 0

@@ -1,0 +1,266 @@
+"""Parity of the CUDA path (through the C ABI) with the oracle, on the five
+seeded workloads at their full sizes, launched exactly as bench.py launches
+them.  Bit-exact: top-k indices, every layout output, bf16 rows, e4m3 codes
+and fp32 scales.  Combine: within one bf16 ulp of the oracle's fp32 sum (and
+in practice bit-identical, since both do the same binary32 operations in the
+same order).  Router weights: within one fp32 ulp (both round one binary64
+quotient to fp32; the binary64 values differ only by summation order and
+libm-vs-CUDA exp, far below 2^-25 relative)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from harness import experts, inputs
+from gpu_util import (bf16_to_f64, check_combine, gpu_bits, stand_in_y_cpu, to_dev, ulp_bf16,
+                      ulp_f32, workload)
+
+pytestmark = pytest.mark.gpu
+
+ALL = ["tiny", "mixtral", "dsv3", "kimi", "prefill"]
+LAYOUT_KEYS = ["expert_counts", "expert_src_counts", "rank_counts", "expert_offsets",
+               "dispatch_pos", "recv_src"]
+
+
+@pytest.fixture(scope="module")
+def moe():
+    import combine_moe_route_08_b200 as m
+    assert torch.cuda.is_available()
+    return m
+
+
+def _status():
+    return torch.zeros(1, dtype=torch.int32, device="cuda")
+
+
+# ------------------------------------------------------------------ route
+
+@pytest.mark.parametrize("name", ALL)
+@pytest.mark.parametrize("renormalize", [False, True])
+def test_route_parity(moe, name, renormalize):
+    wl = workload(name)
+    cfg = wl["cfg"]
+    idx_o, w_o = (wl["idx"], wl["w"]) if not renormalize else oracle.route(
+        wl["logits"].numpy(), cfg.k, renormalize=True)
+    idx, w = moe.moe_route_topk(to_dev(wl["logits"]), cfg.k, renormalize=renormalize)
+    torch.cuda.synchronize()
+    assert np.array_equal(idx.cpu().numpy(), idx_o)
+    w = w.cpu().numpy()
+    assert np.all(np.abs(w.astype(np.float64) - w_o) <= ulp_f32(w_o))
+
+
+# ----------------------------------------------------------------- layout
+
+def _gpu_layout(moe, idx_np, E, R, cap, rows, status=None):
+    out = moe.moe_dispatch_layout(to_dev(idx_np), E, R, capacity=cap, rows=rows, dev_status=status)
+    torch.cuda.synchronize()
+    return {k: out[k].cpu().numpy() for k in LAYOUT_KEYS}
+
+
+def _assert_layout_equal(got, want, where):
+    for key in LAYOUT_KEYS:
+        assert np.array_equal(got[key], want[key].reshape(got[key].shape)), f"{where}: {key}"
+
+
+@pytest.mark.parametrize("name", ALL)
+def test_layout_parity(moe, name):
+    wl = workload(name)
+    cfg = wl["cfg"]
+    st = _status()
+    got = _gpu_layout(moe, wl["idx"], cfg.E, cfg.R, wl["cap"], wl["rows"], st)
+    _assert_layout_equal(got, wl["layout"], name)
+    assert st.item() == 0
+
+
+@pytest.mark.parametrize("name", ["dsv3", "kimi", "prefill"])
+def test_layout_other_mode_parity(moe, name):
+    """Packed workloads also in padded form (cap = max count) and the padded
+    one also packed."""
+    wl = workload(name)
+    cfg = wl["cfg"]
+    if wl["cap"]:
+        cap, rows = 0, cfg.T * cfg.k
+    else:
+        cap = int(wl["layout"]["expert_counts"].max())
+        rows = cfg.E * cap
+    want = oracle.layout(wl["idx"], cfg.E, cfg.R, cap, rows)
+    got = _gpu_layout(moe, wl["idx"], cfg.E, cfg.R, cap, rows)
+    _assert_layout_equal(got, want, name)
+
+
+def test_layout_capacity_overflow_drops_and_reports(moe):
+    wl = workload("kimi")   # skewed: expert 0 is far above the mean
+    cfg = wl["cfg"]
+    cap = int(np.median(wl["layout"]["expert_counts"]))
+    rows = cfg.E * cap + 37                                   # 37 spare rows -> -1
+    want = oracle.layout(wl["idx"], cfg.E, cfg.R, cap, rows)
+    assert want["status"] == oracle.ERR_CAPACITY
+    st = _status()
+    got = _gpu_layout(moe, wl["idx"], cfg.E, cfg.R, cap, rows, st)
+    _assert_layout_equal(got, want, "overflow")
+    assert st.item() == moe.MOE_ERR_CAPACITY
+
+
+# --------------------------------------------------------------- dispatch
+
+@pytest.mark.parametrize("name", ["tiny", "mixtral"])
+def test_dispatch_bf16_parity_with_guard_rows(moe, name):
+    wl = workload(name)
+    cfg = wl["cfg"]
+    rows = wl["rows"]
+    want = oracle.dispatch_bf16(wl["x_bits"], wl["layout"]["dispatch_pos"], rows)
+    guard = 5
+    buf = torch.full((rows + 2 * guard, cfg.H), -7.0, dtype=torch.bfloat16, device="cuda")
+    recv = buf[guard:guard + rows]
+    st = _status()
+    moe.moe_dispatch_bf16(to_dev(wl["x"]), to_dev(wl["layout"]["dispatch_pos"]), rows,
+                          recv_x=recv, dev_status=st)
+    torch.cuda.synchronize()
+    got = gpu_bits(recv)
+    filled = wl["layout"]["recv_src"] >= 0
+    assert np.array_equal(got[filled], want[filled])
+    canary = gpu_bits(buf[:guard]), gpu_bits(buf[guard + rows:])
+    fill = inputs.bf16_bits(torch.tensor([-7.0], dtype=torch.bfloat16))[0]
+    assert np.all(canary[0] == fill) and np.all(canary[1] == fill)
+    assert st.item() == 0
+
+
+def _gpu_fp8(moe, wl, guard=3):
+    cfg = wl["cfg"]
+    rows = wl["rows"]
+    S = cfg.H // 128
+    qbuf = torch.full((rows + 2 * guard, cfg.H), 0xA5, dtype=torch.uint8, device="cuda")
+    sbuf = torch.full((rows + 2 * guard, S), -1.0, dtype=torch.float32, device="cuda")
+    st = _status()
+    moe.moe_dispatch_fp8(to_dev(wl["x"]), to_dev(wl["layout"]["dispatch_pos"]), rows,
+                         recv_q=qbuf[guard:guard + rows], recv_scale=sbuf[guard:guard + rows],
+                         dev_status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    assert torch.all(qbuf[:guard] == 0xA5) and torch.all(qbuf[guard + rows:] == 0xA5)
+    assert torch.all(sbuf[:guard] == -1.0) and torch.all(sbuf[guard + rows:] == -1.0)
+    return qbuf[guard:guard + rows], sbuf[guard:guard + rows]
+
+
+@pytest.mark.parametrize("name", ["dsv3", "kimi"])
+def test_dispatch_fp8_parity_full(moe, name):
+    wl = workload(name)
+    q, s = _gpu_fp8(moe, wl)
+    want_q, want_s = oracle.dispatch_fp8(wl["x_bits"], wl["layout"]["dispatch_pos"], wl["rows"])
+    filled = wl["layout"]["recv_src"] >= 0
+    assert np.array_equal(q.cpu().numpy()[filled], want_q[filled])
+    assert np.array_equal(s.cpu().numpy()[filled].view(np.uint32), want_s[filled].view(np.uint32))
+
+
+def test_dispatch_fp8_parity_prefill_sampled(moe):
+    """Prefill at full size (padded layout): the oracle quantises a sample of
+    tokens one by one; each must appear, bit-exact, in all k of its rows.
+    Padding rows of the padded layout stay untouched."""
+    wl = workload("prefill")
+    cfg = wl["cfg"]
+    q, s = _gpu_fp8(moe, wl)
+    rng = np.random.default_rng(0)
+    tokens = np.unique(np.concatenate([[0, 1, cfg.T - 1, cfg.T_r - 1, cfg.T_r],
+                                       rng.choice(cfg.T, 500, replace=False)])).astype(np.int32)
+    qt, st_ = oracle.quantize_tokens(wl["x_bits"], tokens)
+    pos = wl["layout"]["dispatch_pos"][tokens]                # [n][k]
+    rows_t = torch.from_numpy(pos.ravel().astype(np.int64)).cuda()
+    gq = q.index_select(0, rows_t).cpu().numpy().reshape(len(tokens), cfg.k, cfg.H)
+    gs = s.index_select(0, rows_t).cpu().numpy().reshape(len(tokens), cfg.k, -1)
+    assert np.array_equal(gq, np.repeat(qt[:, None], cfg.k, 1))
+    assert np.array_equal(gs.view(np.uint32), np.repeat(st_[:, None], cfg.k, 1).view(np.uint32))
+    pad = torch.from_numpy(np.nonzero(wl["layout"]["recv_src"] < 0)[0]).cuda()
+    assert pad.numel() > 0
+    assert torch.all(q.index_select(0, pad) == 0xA5)
+
+
+# ---------------------------------------------------------------- combine
+
+@pytest.mark.parametrize("name", ["tiny", "mixtral", "dsv3", "kimi"])
+def test_combine_parity_full(moe, name):
+    """y = the workload's stand-in expert applied (on the CPU) to the oracle's
+    dispatch output; the same y and the oracle's weights go to both sides."""
+    wl = workload(name)
+    cfg = wl["cfg"]
+    pos = wl["layout"]["dispatch_pos"]
+    if cfg.dispatch == "bf16":
+        y = stand_in_y_cpu(wl, recv_bits=oracle.dispatch_bf16(wl["x_bits"], pos, wl["rows"]))
+    else:
+        rq, rs = oracle.dispatch_fp8(wl["x_bits"], pos, wl["rows"])
+        y = stand_in_y_cpu(wl, recv_q=rq, recv_scale=rs)
+    acc, out_o = oracle.combine(y, pos, wl["w"])
+    st = _status()
+    out = moe.moe_combine_bf16(to_dev(inputs.bits_to_bf16(y)), to_dev(pos), to_dev(wl["w"]),
+                               dev_status=st)
+    torch.cuda.synchronize()
+    exact = check_combine(gpu_bits(out), acc, out_o, name)
+    assert exact == 1.0, f"{name}: {exact:.6f} bit-identical"
+    assert st.item() == 0
+
+
+def test_combine_parity_prefill_sampled(moe):
+    wl = workload("prefill")
+    cfg = wl["cfg"]
+    bank = inputs.make_row_bank(cfg.H, seed=cfg.seed * 10 + 2)
+    rmap = inputs.bank_rows_map(wl["rows"])
+    y_dev = bank.cuda().index_select(0, rmap.cuda())
+    out = moe.moe_combine_bf16(y_dev, to_dev(wl["layout"]["dispatch_pos"]), to_dev(wl["w"]))
+    torch.cuda.synchronize()
+    del y_dev
+    rng = np.random.default_rng(1)
+    tokens = np.unique(np.concatenate([[0, cfg.T - 1], rng.choice(cfg.T, 400, replace=False)]))
+    tokens = tokens.astype(np.int32)
+    pos = wl["layout"]["dispatch_pos"]
+    # compact y for the sampled tokens: rows renumbered 0..n*k-1
+    used = pos[tokens].ravel()
+    y_small = inputs.bf16_bits(bank[rmap[torch.from_numpy(used.astype(np.int64))]])
+    pos_small = np.arange(len(used), dtype=np.int32).reshape(len(tokens), cfg.k)
+    acc, out_o = oracle.combine(y_small, pos_small, wl["w"][tokens])
+    got = gpu_bits(out)[tokens]
+    assert check_combine(got, acc, out_o, "prefill") == 1.0
+
+
+# --------------------------------------------------------- whole path
+
+@pytest.mark.parametrize("name", ALL)
+def test_whole_path_on_gpu_vs_oracle(moe, name):
+    """route -> layout -> dispatch -> stand-in expert -> combine, each side on
+    its own data.  Weights may differ by one fp32 ulp, which moves each
+    product by at most 2^-23 |w y|: the combine bound widens by that much."""
+    wl = workload(name)
+    cfg = wl["cfg"]
+    x = to_dev(wl["x"])
+    idx, w = moe.moe_route_topk(to_dev(wl["logits"]), cfg.k)
+    lay = moe.moe_dispatch_layout(idx, cfg.E, cfg.R, capacity=wl["cap"], rows=wl["rows"])
+    pos_o = wl["layout"]["dispatch_pos"]
+    if cfg.dispatch == "bf16":
+        recv = moe.moe_dispatch_bf16(x, lay["dispatch_pos"], wl["rows"])
+        y = recv if cfg.expert == "identity" else experts.affine(
+            recv, inputs.make_expert_noise(cfg, wl["rows"]))
+    else:
+        rq, rs = moe.moe_dispatch_fp8(x, lay["dispatch_pos"], wl["rows"])
+        y = experts.dequantise(rq, rs)
+    out = moe.moe_combine_bf16(y, lay["dispatch_pos"], w)
+    torch.cuda.synchronize()
+    assert np.array_equal(idx.cpu().numpy(), wl["idx"])
+    assert np.array_equal(lay["dispatch_pos"].cpu().numpy(), pos_o)
+    # oracle side (sampled tokens for the large workloads)
+    rng = np.random.default_rng(2)
+    tokens = np.arange(cfg.T, dtype=np.int32) if cfg.T <= 512 else \
+        np.unique(rng.choice(cfg.T, 256, replace=False)).astype(np.int32)
+    if cfg.dispatch == "bf16":
+        y_o = stand_in_y_cpu(wl, recv_bits=oracle.dispatch_bf16(wl["x_bits"], pos_o, wl["rows"]))
+        acc, _ = oracle.combine(y_o, pos_o, wl["w"], tokens=tokens)
+        yf = bf16_to_f64(y_o)
+        terms = np.abs(wl["w"][tokens].astype(np.float64))[:, :, None] * yf[pos_o[tokens]]
+    else:
+        qt, st_ = oracle.quantize_tokens(wl["x_bits"], tokens)
+        y_tok = stand_in_y_cpu(wl, recv_q=qt, recv_scale=st_)          # [n][H]
+        y_small = np.repeat(y_tok, cfg.k, 0)                             # row = i*k + j
+        pos_small = np.arange(len(tokens) * cfg.k, dtype=np.int32).reshape(len(tokens), cfg.k)
+        acc, _ = oracle.combine(y_small, pos_small, wl["w"][tokens])
+        yf = bf16_to_f64(y_small).reshape(len(tokens), cfg.k, cfg.H)
+        terms = np.abs(wl["w"][tokens].astype(np.float64))[:, :, None] * np.abs(yf)
+    got = bf16_to_f64(gpu_bits(out)[tokens])
+    tol = ulp_bf16(acc) + 2.0 ** -22 * terms.sum(1)
+    assert np.all(np.abs(got - acc) <= tol)
