@@ -12,19 +12,25 @@
 // The pages' receiver fills its buffers in a nondeterministic order; here the
 // slots of an expert take consecutive rows in ascending slot index g*k + j, so
 // the layout is bit-reproducible.  Atomics only ever build histograms (an
-// order-free result); every position comes from prefix sums:
+// order-free result); every position comes from prefix sums.
 //
-//   k_layout_count  (one CTA per chunk of tokens inside one logical rank)
-//       shared-memory histogram of the chunk (warp-aggregated with
-//       __match_any_sync), stored to the workspace; the last CTA to finish
-//       (atomic ticket, no waiting) turns the chunk histograms into per-chunk
-//       exclusive prefixes per expert, the per-(expert, source rank) counts,
-//       the expert totals, their exclusive scan (offsets) and rank totals.
-//   k_layout_assign (one CTA per chunk again)
-//       each warp owns a contiguous run of the chunk's slots; per-warp
-//       histograms -> exclusive prefix over the warps -> in-warp rank of each
-//       slot among equal experts (__match_any_sync + popc of the lower lanes)
-//       gives the slot's row; recv_src is the inverse map, -1 elsewhere.
+// Tokens are cut into chunks that never straddle two logical source ranks
+// (at most 8192 slots each); one 1024-thread CTA owns a chunk and each of its
+// 32 warps a contiguous run of at most 8 x 32 slots, which every lane keeps in
+// registers (one load round trip per kernel).
+//
+//   k_layout_hist    chunk histogram (per-warp __match_any_sync aggregation,
+//                    shared-memory atomics) -> workspace hist[chunk][E].
+//   k_layout_assign  every CTA sums the histogram columns it needs (the base
+//                    of its chunk inside each expert, the expert totals) --
+//                    redundant but parallel, no serial tail -- scans the
+//                    totals into offsets, builds per-warp histograms of its
+//                    own slots, scans them over the warps, and ranks each
+//                    slot among the equal experts of its warp step
+//                    (__match_any_sync + popc of the lower lanes) to get its
+//                    row.  CTA 0 also writes counts, offsets and rank sums.
+// The kernel boundary between the two is the only grid-wide ordering; nothing
+// waits on another CTA.
 #include <algorithm>
 
 #include "common.cuh"
@@ -34,9 +40,11 @@ namespace moe {
 
 namespace {
 
-constexpr int kLayoutThreads = 256;
-constexpr int kLayoutWarps = kLayoutThreads / 32;
-constexpr size_t kTicketBytes = 256;
+constexpr int kThreads = 1024;
+constexpr int kWarps = kThreads / 32;
+constexpr int kMaxSteps = 8;                       // 32-slot steps per warp
+constexpr int kChunkSlots = kThreads * kMaxSteps;  // 8192
+constexpr int kColBatch = 16;                      // histogram loads in flight per thread
 
 __device__ __forceinline__ void chunk_tokens(const LayoutGeom &G, int c, int &t0, int &t1)
 {
@@ -47,6 +55,18 @@ __device__ __forceinline__ void chunk_tokens(const LayoutGeom &G, int c, int &t0
     t1 = min(t0 + G.CT, rank_end);
 }
 
+// This warp's run of slots [w0, w1) inside chunk c, in 32-slot steps.
+__device__ __forceinline__ void warp_run(const LayoutGeom &G, int c, int64_t &w0, int64_t &w1)
+{
+    int t0, t1;
+    chunk_tokens(G, c, t0, t1);
+    const int64_t i0 = static_cast<int64_t>(t0) * G.k, i1 = static_cast<int64_t>(t1) * G.k;
+    const int64_t seg = static_cast<int64_t>(ceil_div(static_cast<int>(i1 - i0), kWarps * 32)) * 32;
+    const int w = threadIdx.x >> 5;
+    w0 = min(i0 + w * seg, i1);
+    w1 = min(w0 + seg, i1);
+}
+
 __device__ __forceinline__ unsigned lanemask_lt()
 {
     unsigned m;
@@ -54,21 +74,65 @@ __device__ __forceinline__ unsigned lanemask_lt()
     return m;
 }
 
-// In-place exclusive scan of a[0..n) by 256 threads (n <= 1024); a[n] gets
-// the total.  `tot` is 9 ints of scratch shared memory.
+// The lane's slots of its warp run, loaded in one go (-1 past the end).
+__device__ __forceinline__ void load_run(const int32_t *__restrict__ topk_idx, int64_t w0,
+                                         int64_t w1, int (&e)[kMaxSteps])
+{
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int s = 0; s < kMaxSteps; ++s) {
+        const int64_t i = w0 + 32 * s + lane;
+        e[s] = (i < w1) ? __ldg(topk_idx + i) : -1;
+    }
+}
+
+// Key for __match_any_sync: the expert, or a value no expert and no other
+// lane uses for slots that are empty, masked or invalid.
+__device__ __forceinline__ int match_key(int e, int E, int lane)
+{
+    return (static_cast<unsigned>(e) < static_cast<unsigned>(E)) ? e : (0x40000000 | lane);
+}
+
+__global__ void __launch_bounds__(kThreads)
+    k_layout_hist(const int32_t *__restrict__ topk_idx, LayoutGeom G,
+                  int32_t *__restrict__ ws_hist, int32_t *__restrict__ dev_status)
+{
+    extern __shared__ int32_t h[];  // [E]
+    const int E = G.E, lane = threadIdx.x & 31;
+    const int c = blockIdx.x;
+    int64_t w0, w1;
+    warp_run(G, c, w0, w1);
+    int e[kMaxSteps];
+    load_run(topk_idx, w0, w1, e);
+    for (int x = threadIdx.x; x < E; x += kThreads)
+        h[x] = 0;
+    __syncthreads();
+
+    bool bad = false;
+#pragma unroll
+    for (int s = 0; s < kMaxSteps; ++s) {
+        if (w0 + 32 * s >= w1)
+            break;  // warp-uniform
+        const bool valid = static_cast<unsigned>(e[s]) < static_cast<unsigned>(E);
+        bad |= !valid && e[s] != -1 && (w0 + 32 * s + lane < w1);
+        const unsigned mask = __match_any_sync(kFullMask, match_key(e[s], E, lane));
+        if (valid && lane == __ffs(mask) - 1)
+            atomicAdd(&h[e[s]], __popc(mask));
+    }
+    if (bad)
+        report(dev_status, MOE_ERR_INVALID_ARG);
+    __syncthreads();
+    for (int x = threadIdx.x; x < E; x += kThreads)
+        ws_hist[static_cast<size_t>(c) * E + x] = h[x];
+}
+
+// In-place exclusive scan of a[0..n) (n <= kThreads) by the whole CTA; a[n]
+// receives the total.  `tot` is kWarps + 1 ints of shared scratch.
 __device__ void block_exclusive_scan(int32_t *a, int n, int32_t *tot)
 {
-    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-    const int per = ceil_div(n, kLayoutThreads);  // <= 4
-    const int b = tid * per;
-    int loc[4];
-    int sum = 0;
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-        loc[u] = (u < per && b + u < n) ? a[b + u] : 0;
-        sum += loc[u];
-    }
-    int incl = sum;
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    const int v = (tid < n) ? a[tid] : 0;
+    int incl = v;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
         const int t = __shfl_up_sync(kFullMask, incl, off);
@@ -76,215 +140,174 @@ __device__ void block_exclusive_scan(int32_t *a, int n, int32_t *tot)
             incl += t;
     }
     if (lane == 31)
-        tot[wid] = incl;
+        tot[w] = incl;
     __syncthreads();
-    if (tid == 0) {
-        int run = 0;
-        for (int w = 0; w < kLayoutWarps; ++w) {
-            const int t = tot[w];
-            tot[w] = run;
-            run += t;
-        }
-        tot[kLayoutWarps] = run;
-    }
-    __syncthreads();
-    int run = tot[wid] + incl - sum;
+    if (w == 0) {
+        const int t = tot[lane];
+        int x = t;
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-        if (u < per && b + u < n) {
-            a[b + u] = run;
-            run += loc[u];
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(kFullMask, x, off);
+            if (lane >= off)
+                x += y;
         }
+        tot[lane] = x - t;  // exclusive over warps
+        if (lane == 31)
+            tot[kWarps] = x;
     }
+    __syncthreads();
+    if (tid < n)
+        a[tid] = tot[w] + incl - v;
     if (tid == 0)
-        a[n] = tot[kLayoutWarps];
+        a[n] = tot[kWarps];
     __syncthreads();
 }
 
-__global__ void __launch_bounds__(kLayoutThreads)
-    k_layout_count(const int32_t *__restrict__ topk_idx, LayoutGeom G, int capacity,
-                   int32_t *__restrict__ ws_hist, unsigned *__restrict__ ws_ticket,
-                   int32_t *__restrict__ expert_counts, int32_t *__restrict__ expert_src_counts,
-                   int32_t *__restrict__ rank_counts, int32_t *__restrict__ expert_offsets,
-                   int32_t *__restrict__ dev_status)
+__global__ void __launch_bounds__(kThreads)
+    k_layout_assign(const int32_t *__restrict__ topk_idx, LayoutGeom G, int capacity, int64_t rows,
+                    const int32_t *__restrict__ ws_hist, int32_t *__restrict__ expert_counts,
+                    int32_t *__restrict__ expert_src_counts, int32_t *__restrict__ rank_counts,
+                    int32_t *__restrict__ expert_offsets, int32_t *__restrict__ dispatch_pos,
+                    int32_t *__restrict__ recv_src, int32_t *__restrict__ dev_status)
 {
-    extern __shared__ int32_t sm[];  // [E + 1] histogram, later the scan
-    __shared__ int32_t scan_tot[kLayoutWarps + 1];
-    __shared__ bool is_last;
-    const int E = G.E;
-    const int tid = threadIdx.x, lane = tid & 31;
+    extern __shared__ int32_t sm[];
+    const int E = G.E, lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    int32_t *wh = sm;                   // [kWarps][E] per-warp counts, then bases
+    int32_t *off = wh + kWarps * E;     // [E + 1] expert totals, then their scan
+    int32_t *chb = off + E + 1;         // [E] slots of e in earlier chunks
+    int32_t *tot = chb + E;             // [kWarps + 1]
     const int c = blockIdx.x;
 
-    for (int e = tid; e <= E; e += kLayoutThreads)
-        sm[e] = 0;
-    __syncthreads();
+    int64_t w0, w1;
+    warp_run(G, c, w0, w1);
+    int e[kMaxSteps];
+    load_run(topk_idx, w0, w1, e);  // in flight while the columns are summed
 
-    int t0, t1;
-    chunk_tokens(G, c, t0, t1);
-    const int64_t i0 = static_cast<int64_t>(t0) * G.k, i1 = static_cast<int64_t>(t1) * G.k;
-    bool bad = false;
-    for (int64_t base = i0; base < i1; base += kLayoutThreads) {  // CTA-uniform trips
-        const int64_t i = base + tid;
-        const int e = (i < i1) ? __ldg(topk_idx + i) : -1;
-        const bool valid = static_cast<unsigned>(e) < static_cast<unsigned>(E);
-        bad |= (i < i1) && !valid && e != -1;
-        const unsigned mask = __match_any_sync(kFullMask, valid ? e : (0x40000000 | lane));
-        if (valid && lane == __ffs(mask) - 1)
-            atomicAdd(&sm[e], __popc(mask));
-    }
-    if (bad)
-        report(dev_status, MOE_ERR_INVALID_ARG);
-    __syncthreads();
+    for (int x = threadIdx.x; x < kWarps * E; x += kThreads)
+        wh[x] = 0;
 
-    int32_t *mine = ws_hist + static_cast<size_t>(c) * E;
-    for (int e = tid; e < E; e += kLayoutThreads)
-        mine[e] = sm[e];
-    __threadfence();
-    __syncthreads();
-    if (tid == 0)
-        is_last = (atomicAdd(ws_ticket, 1u) == gridDim.x - 1);
-    __syncthreads();
-    if (!is_last)
-        return;
-    __threadfence();
-
-    // ---- last CTA: per expert, walk the chunks in order ----
+    // histogram columns: base of this chunk inside each expert, expert totals,
+    // and (CTA 0) the per-source-rank counts
     const int n = G.nchunks;
-    for (int e = tid; e < E; e += kLayoutThreads) {
-        int run = 0, src = 0;
-        for (int c0 = 0; c0 < n; c0 += 8) {
-            int v[8];
+    for (int x = threadIdx.x; x < E; x += kThreads) {
+        int before = 0, total = 0, rank_sum = 0, next_rank_end = G.cpr;
+        for (int c0 = 0; c0 < n; c0 += kColBatch) {
+            int v[kColBatch];
 #pragma unroll
-            for (int u = 0; u < 8; ++u)
-                v[u] = (c0 + u < n) ? __ldcg(ws_hist + static_cast<size_t>(c0 + u) * E + e) : 0;
+            for (int u = 0; u < kColBatch; ++u)
+                v[u] = (c0 + u < n) ? __ldg(ws_hist + static_cast<size_t>(c0 + u) * E + x) : 0;
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
+            for (int u = 0; u < kColBatch; ++u) {
                 const int cc = c0 + u;
-                if (cc < n) {
-                    ws_hist[static_cast<size_t>(cc) * E + e] = run;  // chunk's base in e
-                    run += v[u];
-                    src += v[u];
-                    if (cc % G.cpr == G.cpr - 1) {
-                        expert_src_counts[static_cast<size_t>(e) * G.R + cc / G.cpr] = src;
-                        src = 0;
+                if (cc < c)
+                    before += v[u];
+                total += v[u];
+                if (c == 0 && cc < n) {
+                    rank_sum += v[u];
+                    if (cc + 1 == next_rank_end) {
+                        expert_src_counts[static_cast<size_t>(x) * G.R + cc / G.cpr] = rank_sum;
+                        rank_sum = 0;
+                        next_rank_end += G.cpr;
                     }
                 }
             }
         }
-        expert_counts[e] = run;
-        sm[e] = run;
+        off[x] = total;
+        chb[x] = before;
+        if (c == 0)
+            expert_counts[x] = total;
     }
     __syncthreads();
-    block_exclusive_scan(sm, E, scan_tot);  // sm[e] = slots of experts < e, sm[E] = total
-    for (int e = tid; e <= E; e += kLayoutThreads)
-        expert_offsets[e] = (capacity == 0) ? sm[e] : e * capacity;
-    const int L = E / G.R;
-    for (int r = tid; r < G.R; r += kLayoutThreads)
-        rank_counts[r] = sm[(r + 1) * L] - sm[r * L];
-    if (tid == 0)
-        *ws_ticket = 0u;  // leave the workspace reusable
-}
 
-__global__ void __launch_bounds__(kLayoutThreads)
-    k_layout_assign(const int32_t *__restrict__ topk_idx, LayoutGeom G, int capacity, int64_t rows,
-                    const int32_t *__restrict__ ws_hist, const int32_t *__restrict__ expert_counts,
-                    const int32_t *__restrict__ expert_offsets, int32_t *__restrict__ dispatch_pos,
-                    int32_t *__restrict__ recv_src, int32_t *__restrict__ dev_status)
-{
-    extern __shared__ int32_t sm[];
-    const int E = G.E;
-    int32_t *wh = sm;                      // [8][E] per-warp running base
-    int32_t *ob = sm + kLayoutWarps * E;   // [E + 1] expert row base
-    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-    const int c = blockIdx.x;
-
-    for (int x = tid; x < kLayoutWarps * E; x += kLayoutThreads)
-        wh[x] = 0;
-    for (int e = tid; e <= E; e += kLayoutThreads)
-        ob[e] = expert_offsets[e];
-    __syncthreads();
-
-    int t0, t1;
-    chunk_tokens(G, c, t0, t1);
-    const int64_t i0 = static_cast<int64_t>(t0) * G.k, i1 = static_cast<int64_t>(t1) * G.k;
-    const int64_t seg = static_cast<int64_t>(ceil_div(static_cast<int>(i1 - i0), kLayoutWarps * 32)) * 32;
-    const int64_t w0 = min(i0 + w * seg, i1), w1 = min(w0 + seg, i1);
+    // per-warp histogram of this CTA's slots (warp-private rows: no atomics)
     int32_t *mywh = wh + w * E;
-
-    // pass A: per-warp histogram of its run of slots
-    for (int64_t base = w0; base < w1; base += 32) {  // warp-uniform trips
-        const int64_t i = base + lane;
-        const int e = (i < w1) ? __ldg(topk_idx + i) : -1;
-        const bool valid = static_cast<unsigned>(e) < static_cast<unsigned>(E);
-        const unsigned mask = __match_any_sync(kFullMask, valid ? e : (0x40000000 | lane));
+#pragma unroll
+    for (int s = 0; s < kMaxSteps; ++s) {
+        if (w0 + 32 * s >= w1)
+            break;
+        const bool valid = static_cast<unsigned>(e[s]) < static_cast<unsigned>(E);
+        const unsigned mask = __match_any_sync(kFullMask, match_key(e[s], E, lane));
         if (valid && lane == __ffs(mask) - 1)
-            mywh[e] += __popc(mask);
+            mywh[e[s]] += __popc(mask);
         __syncwarp();
     }
-    __syncthreads();
+    block_exclusive_scan(off, E, tot);  // off[e] = slots of experts < e; off[E] = total
 
-    // pass B: base of each warp = chunk base in e + slots of e in earlier warps
-    for (int e = tid; e < E; e += kLayoutThreads) {
-        int run = ws_hist[static_cast<size_t>(c) * E + e];
-#pragma unroll
-        for (int ww = 0; ww < kLayoutWarps; ++ww) {
-            const int t = wh[ww * E + e];
-            wh[ww * E + e] = run;
+    if (c == 0) {
+        for (int x = threadIdx.x; x <= E; x += kThreads)
+            expert_offsets[x] = (capacity == 0) ? off[x] : x * capacity;
+        const int L = E / G.R;
+        for (int r = threadIdx.x; r < G.R; r += kThreads)
+            rank_counts[r] = off[(r + 1) * L] - off[r * L];
+    }
+    // per-warp base of each expert's positions: earlier chunks + earlier warps
+    for (int x = threadIdx.x; x < E; x += kThreads) {
+        int run = chb[x];
+#pragma unroll 8
+        for (int ww = 0; ww < kWarps; ++ww) {
+            const int t = wh[ww * E + x];
+            wh[ww * E + x] = run;
             run += t;
         }
     }
     __syncthreads();
 
-    // pass C: rank inside the warp among equal experts -> row
-    bool dropped = false;
-    for (int64_t base = w0; base < w1; base += 32) {
-        const int64_t i = base + lane;
-        const int e = (i < w1) ? __ldg(topk_idx + i) : -1;
-        const bool valid = static_cast<unsigned>(e) < static_cast<unsigned>(E);
-        const unsigned mask = __match_any_sync(kFullMask, valid ? e : (0x40000000 | lane));
-        const int p = valid ? mywh[e] + __popc(mask & lanemask_lt()) : 0;
+    // rank every slot among equal experts, in slot order
+    bool dropped = false, bad_row = false;
+#pragma unroll
+    for (int s = 0; s < kMaxSteps; ++s) {
+        if (w0 + 32 * s >= w1)
+            break;
+        const int64_t i = w0 + 32 * s + lane;
+        const bool valid = static_cast<unsigned>(e[s]) < static_cast<unsigned>(E);
+        const unsigned mask = __match_any_sync(kFullMask, match_key(e[s], E, lane));
+        const int p = valid ? mywh[e[s]] + __popc(mask & lanemask_lt()) : 0;
         __syncwarp();
         if (valid && lane == __ffs(mask) - 1)
-            mywh[e] += __popc(mask);
+            mywh[e[s]] += __popc(mask);
         __syncwarp();
         if (i < w1) {
-            int row = -1;
+            int64_t row = -1;
             if (valid) {
                 if (capacity == 0)
-                    row = ob[e] + p;
+                    row = off[e[s]] + p;
                 else if (p < capacity)
-                    row = e * capacity + p;
+                    row = static_cast<int64_t>(e[s]) * capacity + p;
                 else
                     dropped = true;
             }
             if (row >= rows) {  // cannot happen for a consistent layout; never write past rows
-                report(dev_status, MOE_ERR_INVALID_ARG);
+                bad_row = true;
                 row = -1;
             }
-            dispatch_pos[i] = row;
+            dispatch_pos[i] = static_cast<int32_t>(row);
             if (row >= 0)
                 recv_src[row] = static_cast<int32_t>(i);
         }
     }
     if (dropped)
         report(dev_status, MOE_ERR_CAPACITY);
+    if (bad_row)
+        report(dev_status, MOE_ERR_INVALID_ARG);
 
     // rows that no slot fills -> -1
-    const int64_t stride = static_cast<int64_t>(gridDim.x) * kLayoutThreads;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * kThreads;
+    const int64_t first = static_cast<int64_t>(c) * kThreads + threadIdx.x;
     if (capacity == 0) {
-        for (int64_t r = ob[E] + static_cast<int64_t>(c) * kLayoutThreads + tid; r < rows; r += stride)
+        for (int64_t r = off[E] + first; r < rows; r += stride)
             recv_src[r] = -1;
     } else {
-        for (int e = c; e < E; e += gridDim.x) {
-            const int filled = min(expert_counts[e], capacity);
-            for (int p = filled + tid; p < capacity; p += kLayoutThreads)
-                recv_src[static_cast<int64_t>(e) * capacity + p] = -1;
+        for (int x = c; x < E; x += gridDim.x) {
+            const int filled = min(off[x + 1] - off[x], capacity);
+            for (int p = filled + threadIdx.x; p < capacity; p += kThreads)
+                recv_src[static_cast<int64_t>(x) * capacity + p] = -1;
         }
-        for (int64_t r = static_cast<int64_t>(E) * capacity + static_cast<int64_t>(c) * kLayoutThreads + tid;
-             r < rows; r += stride)
+        for (int64_t r = static_cast<int64_t>(E) * capacity + first; r < rows; r += stride)
             recv_src[r] = -1;
     }
 }
+
+size_t assign_smem_bytes(int E) { return (static_cast<size_t>(kWarps + 2) * E + 1 + kWarps + 1) * sizeof(int32_t); }
 
 }  // namespace
 
@@ -296,7 +319,7 @@ LayoutGeom layout_geom(int T, int k, int E, int R)
     g.E = E;
     g.R = R;
     g.Tr = T / R;
-    g.CT = std::max(1, 2048 / k);  // about 2048 slots per chunk
+    g.CT = std::max(1, kChunkSlots / k);  // at most 8192 slots per chunk
     g.cpr = std::max(1, ceil_div(g.Tr, g.CT));
     g.nchunks = R * g.cpr;
     return g;
@@ -305,7 +328,7 @@ LayoutGeom layout_geom(int T, int k, int E, int R)
 size_t layout_workspace_bytes(const LayoutGeom &g)
 {
     const size_t hist = static_cast<size_t>(g.nchunks) * g.E * sizeof(int32_t);
-    return kTicketBytes + (hist + 255) / 256 * 256;
+    return std::max<size_t>(256, (hist + 255) / 256 * 256);
 }
 
 cudaError_t dispatch_layout(const int32_t *topk_idx, const LayoutGeom &g, int capacity, int64_t rows,
@@ -314,19 +337,22 @@ cudaError_t dispatch_layout(const int32_t *topk_idx, const LayoutGeom &g, int ca
                             int32_t *recv_src, void *workspace, int32_t *dev_status,
                             cudaStream_t s)
 {
-    unsigned *ticket = static_cast<unsigned *>(workspace);
-    int32_t *hist = reinterpret_cast<int32_t *>(static_cast<char *>(workspace) + kTicketBytes);
-    const size_t smem1 = (g.E + 1) * sizeof(int32_t);
-    k_layout_count<<<g.nchunks, kLayoutThreads, smem1, s>>>(topk_idx, g, capacity, hist, ticket,
-                                                            expert_counts, expert_src_counts,
-                                                            rank_counts, expert_offsets, dev_status);
+    int32_t *hist = static_cast<int32_t *>(workspace);
+    k_layout_hist<<<g.nchunks, kThreads, g.E * sizeof(int32_t), s>>>(topk_idx, g, hist, dev_status);
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess)
         return err;
-    const size_t smem2 = (static_cast<size_t>(kLayoutWarps) * g.E + g.E + 1) * sizeof(int32_t);
-    k_layout_assign<<<g.nchunks, kLayoutThreads, smem2, s>>>(topk_idx, g, capacity, rows, hist,
-                                                             expert_counts, expert_offsets,
-                                                             dispatch_pos, recv_src, dev_status);
+    const size_t smem = assign_smem_bytes(g.E);
+    if (smem > 48 * 1024) {
+        err = cudaFuncSetAttribute(k_layout_assign, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   static_cast<int>(smem));
+        if (err != cudaSuccess)
+            return err;
+    }
+    k_layout_assign<<<g.nchunks, kThreads, smem, s>>>(topk_idx, g, capacity, rows, hist,
+                                                      expert_counts, expert_src_counts, rank_counts,
+                                                      expert_offsets, dispatch_pos, recv_src,
+                                                      dev_status);
     return cudaGetLastError();
 }
 

@@ -8,10 +8,16 @@
 // Each lane holds the logits e = i*32 + lane (a warp-wide load per i is one
 // coalesced 128-byte line).  k rounds of warp arg-max under the order (logit
 // descending, index ascending) pick the experts; a per-lane bit mask removes
-// the winners.  The softmax denominator is summed in binary64 over all E
-// experts and every weight is one binary64 quotient rounded once to fp32, so
-// the result differs from any other correct binary64 evaluation by at most
-// one fp32 ulp.
+// the winners.
+//
+// The softmax is evaluated in fp32 with its error bounded (u = 2^-24):
+//   d = l - m is split exactly into d_hi + d_lo (Knuth's TwoSum), so the
+//   exponent sees no rounding of the difference; t = expf(d_hi) * (1 + d_lo)
+//   has relative error <= 5u (expf is within 2 ulp = 4u, plus one rounding);
+//   the denominator is a compensated (Neumaier) sum of the positive t, within
+//   2u of their exact sum; w = t_j / S is one IEEE division (u).  Hence
+//   |w - p| <= 13u * p (+ O(u^2)) for the exact probability p, i.e. within 16
+//   fp32 ulps of the correctly rounded value; in practice 1-2 ulps.
 #include <cfloat>
 #include <climits>
 
@@ -36,6 +42,38 @@ __device__ __forceinline__ bool better(const Cand &a, const Cand &b)
     if (b.e == INT_MAX)
         return true;
     return a.v > b.v || (a.v == b.v && a.e < b.e);
+}
+
+// a + b == s + err exactly (Knuth's TwoSum; explicit _rn ops are never
+// contracted or reassociated)
+__device__ __forceinline__ void two_sum(float a, float b, float &s, float &err)
+{
+    s = __fadd_rn(a, b);
+    const float bb = __fsub_rn(s, a);
+    err = __fadd_rn(__fsub_rn(a, __fsub_rn(s, bb)), __fsub_rn(b, bb));
+}
+
+// Neumaier's compensated summation step: (sum + comp) absorbs t.
+__device__ __forceinline__ void neumaier_add(float &sum, float &comp, float t)
+{
+    float s, err;
+    two_sum(sum, t, s, err);
+    sum = s;
+    comp = __fadd_rn(comp, err);
+}
+
+// exp(l - m) for fp32 l <= m: the difference split exactly into hi + lo, the
+// exponential of hi by expf, the first-order factor (1 + lo) applied with one
+// fused multiply-add (|lo| <= 2^-24 |hi|, so the dropped lo^2/2 is far below
+// the rounding of the result).
+__device__ __forceinline__ float exp_diff(float l, float m)
+{
+    float hi, lo;
+    two_sum(l, -m, hi, lo);
+    if (hi < -104.0f)  // expf underflows to 0 (and keeps an overflowed hi from making NaN)
+        return 0.0f;
+    const float t = expf(hi);
+    return __fmaf_rn(t, lo, t);
 }
 
 template <int NPL>
@@ -92,27 +130,36 @@ __global__ void __launch_bounds__(kRouteWarps * 32)
             vmax = best.v;
     }
 
-    const double m = static_cast<double>(vmax);
-    double denom = 0.0;
+    // softmax over all E logits, in fp32 with compensated summation
+    float sum = 0.0f, comp = 0.0f;
 #pragma unroll
     for (int i = 0; i < NPL; ++i)
         if (i * 32 + lane < E)
-            denom += exp(static_cast<double>(v[i]) - m);
+            neumaier_add(sum, comp, exp_diff(v[i], vmax));
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1)
-        denom += __shfl_xor_sync(kFullMask, denom, off);
+    for (int off = 16; off > 0; off >>= 1) {
+        const float os = __shfl_xor_sync(kFullMask, sum, off);
+        const float oc = __shfl_xor_sync(kFullMask, comp, off);
+        comp = __fadd_rn(comp, oc);
+        neumaier_add(sum, comp, os);
+    }
+    float denom = __fadd_rn(sum, comp);
 
-    const double num = (lane < k) ? exp(static_cast<double>(my_v) - m) : 0.0;
+    const float num = (lane < k) ? exp_diff(my_v, vmax) : 0.0f;
     if (renormalize) {
-        double s = num;
+        float ks = num, kc = 0.0f;
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1)
-            s += __shfl_xor_sync(kFullMask, s, off);
-        denom = s;
+        for (int off = 16; off > 0; off >>= 1) {
+            const float os = __shfl_xor_sync(kFullMask, ks, off);
+            const float oc = __shfl_xor_sync(kFullMask, kc, off);
+            kc = __fadd_rn(kc, oc);
+            neumaier_add(ks, kc, os);
+        }
+        denom = __fadd_rn(ks, kc);
     }
     if (lane < k) {
         topk_idx[static_cast<size_t>(g) * k + lane] = my_e;
-        topk_w[static_cast<size_t>(g) * k + lane] = __double2float_rn(num / denom);
+        topk_w[static_cast<size_t>(g) * k + lane] = __fdiv_rn(num, denom);
     }
 }
 

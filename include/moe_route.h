@@ -84,9 +84,10 @@ const char *moe_status_string(int status);
  *   topk_idx  [T][k] int32 out: the k experts first in the order (logit
  *             descending, expert index ascending); -0.0 and +0.0 are equal.
  *   topk_w    [T][k] fp32 out: p_e = exp(l_e - m) / sum_e' exp(l_e' - m),
- *             m = max logit, evaluated in binary64 and rounded once to fp32;
- *             with renormalize != 0 the sum runs over the k chosen experts
- *             only (softmax restricted to the top-k).
+ *             m = max logit; with renormalize != 0 the sum runs over the k
+ *             chosen experts only (softmax restricted to the top-k).  Computed
+ *             in fp32 (exact split of l - m, expf, compensated sum, one IEEE
+ *             division): |topk_w - p| <= 14 * 2^-24 * p.
  * Logits must be finite.  T == 0 enqueues nothing.
  */
 int moe_route_topk(const float *logits, int T, int E, int k, int renormalize,
@@ -94,10 +95,9 @@ int moe_route_topk(const float *logits, int T, int E, int k, int renormalize,
 
 /*
  * Bytes of device workspace moe_dispatch_layout needs for (T, k, E, R);
- * 0 on invalid sizes.  The workspace must be 256-byte aligned and
- * ZERO-FILLED BEFORE ITS FIRST USE (cudaMemset); every call leaves it
- * reusable.  One workspace must not serve two layout calls that may run at
- * the same time.
+ * 0 on invalid sizes.  The workspace must be 256-byte aligned; its contents
+ * need no initialisation and are scratch (per-chunk histograms).  One
+ * workspace must not serve two layout calls that may run at the same time.
  */
 size_t moe_layout_workspace_bytes(int T, int k, int E, int R);
 

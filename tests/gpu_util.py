@@ -32,6 +32,16 @@ def ulp_f32(a: np.ndarray) -> np.ndarray:
     return np.spacing(np.abs(a.astype(np.float32))).astype(np.float64)
 
 
+def route_w_tol(w_oracle: np.ndarray) -> np.ndarray:
+    """Bound on |w_gpu - w_oracle| for the router weights.  The kernel's fp32
+    softmax is within 13u of the exact probability p (u = 2^-24: an exact
+    split of l - m, expf within 2 ulp = 4u plus one rounding for each term and
+    for the numerator, a compensated sum within 2u, one IEEE division); the
+    oracle rounds a binary64 value once (within u).  Hence 14u * p, plus the
+    spacing of fp32 subnormals."""
+    return 14 * 2.0 ** -24 * np.abs(w_oracle.astype(np.float64)) * (1 + 2.0 ** -20) + 2.0 ** -149
+
+
 def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
     return inputs.bits_to_bf16(bits).float().numpy().astype(np.float64)
 

@@ -3,9 +3,8 @@ seeded workloads at their full sizes, launched exactly as bench.py launches
 them.  Bit-exact: top-k indices, every layout output, bf16 rows, e4m3 codes
 and fp32 scales.  Combine: within one bf16 ulp of the oracle's fp32 sum (and
 in practice bit-identical, since both do the same binary32 operations in the
-same order).  Router weights: within one fp32 ulp (both round one binary64
-quotient to fp32; the binary64 values differ only by summation order and
-libm-vs-CUDA exp, far below 2^-25 relative)."""
+same order).  Router weights: within 14 * 2^-24 relative of the oracle's
+(the kernel's fp32 softmax error bound, derived in gpu_util.route_w_tol)."""
 import numpy as np
 import pytest
 import torch
@@ -13,7 +12,7 @@ import torch
 import oracle
 from harness import experts, inputs
 from gpu_util import (bf16_to_f64, check_combine, gpu_bits, stand_in_y_cpu, to_dev, ulp_bf16,
-                      ulp_f32, workload)
+                      route_w_tol, ulp_f32, workload)
 
 pytestmark = pytest.mark.gpu
 
@@ -46,7 +45,9 @@ def test_route_parity(moe, name, renormalize):
     torch.cuda.synchronize()
     assert np.array_equal(idx.cpu().numpy(), idx_o)
     w = w.cpu().numpy()
-    assert np.all(np.abs(w.astype(np.float64) - w_o) <= ulp_f32(w_o))
+    err = np.abs(w.astype(np.float64) - w_o)
+    assert np.all(err <= route_w_tol(w_o))
+    print(f"{name}: max weight error {np.max(err / ulp_f32(w_o)):.2f} fp32 ulp")
 
 
 # ----------------------------------------------------------------- layout
@@ -91,7 +92,7 @@ def test_layout_other_mode_parity(moe, name):
 def test_layout_capacity_overflow_drops_and_reports(moe):
     wl = workload("kimi")   # skewed: expert 0 is far above the mean
     cfg = wl["cfg"]
-    cap = int(np.median(wl["layout"]["expert_counts"]))
+    cap = max(1, int(wl["layout"]["expert_counts"].max()) // 2)
     rows = cfg.E * cap + 37                                   # 37 spare rows -> -1
     want = oracle.layout(wl["idx"], cfg.E, cfg.R, cap, rows)
     assert want["status"] == oracle.ERR_CAPACITY
@@ -225,8 +226,9 @@ def test_combine_parity_prefill_sampled(moe):
 @pytest.mark.parametrize("name", ALL)
 def test_whole_path_on_gpu_vs_oracle(moe, name):
     """route -> layout -> dispatch -> stand-in expert -> combine, each side on
-    its own data.  Weights may differ by one fp32 ulp, which moves each
-    product by at most 2^-23 |w y|: the combine bound widens by that much."""
+    its own data.  Weights may differ by 14u relative (u = 2^-24), which moves
+    each product by at most 14u |w y|; with the two sums' own rounding
+    (gamma_k each, k = 8) the bound widens by less than 2^-19 sum |w y|."""
     wl = workload(name)
     cfg = wl["cfg"]
     x = to_dev(wl["x"])
@@ -262,5 +264,5 @@ def test_whole_path_on_gpu_vs_oracle(moe, name):
         yf = bf16_to_f64(y_small).reshape(len(tokens), cfg.k, cfg.H)
         terms = np.abs(wl["w"][tokens].astype(np.float64))[:, :, None] * np.abs(yf)
     got = bf16_to_f64(gpu_bits(out)[tokens])
-    tol = ulp_bf16(acc) + 2.0 ** -22 * terms.sum(1)
+    tol = ulp_bf16(acc) + 2.0 ** -19 * terms.sum(1)
     assert np.all(np.abs(got - acc) <= tol)
