@@ -19,14 +19,14 @@ import torch
 __all__ = [
     "MoeError", "lib", "moe_status_string", "moe_route_topk", "moe_layout_workspace_bytes",
     "moe_dispatch_layout", "moe_dispatch_bf16", "moe_dispatch_fp8", "moe_combine_bf16",
-    "moe_quantize_e4m3", "Workspace", "LIB_PATH",
+    "moe_quantize_e4m3", "moe_dispatch_layout_noalloc", "Workspace", "LIB_PATH",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_route.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m combine_moe_route_08_b200.build` "
+        f"{LIB_PATH} is missing: build it with `python combine_moe_route_08_b200/build.py` "
         "(nvcc, sm_100a). This package has no fallback path.")
 
 lib = ctypes.CDLL(LIB_PATH)
@@ -43,6 +43,9 @@ lib.moe_layout_workspace_bytes.restype = _sz
 lib.moe_dispatch_layout.argtypes = [_P, _i32, _i32, _i32, _i32, _i32, _i64, _P, _P, _P, _P, _P, _P,
                                     _P, _sz, _P, _P]
 lib.moe_dispatch_layout.restype = _i32
+lib.moe_dispatch_layout_noalloc.argtypes = [_P, _i32, _i32, _i32, _i32, _i32, _i64, _P, _P, _P,
+                                            _P, _P, _P, _P, _P]
+lib.moe_dispatch_layout_noalloc.restype = _i32
 lib.moe_dispatch_bf16.argtypes = [_P, _i32, _i32, _i32, _P, _P, _i64, _P, _P]
 lib.moe_dispatch_bf16.restype = _i32
 lib.moe_dispatch_fp8.argtypes = [_P, _i32, _i32, _i32, _P, _P, _P, _i64, _P, _P]
@@ -170,6 +173,36 @@ def moe_dispatch_layout(topk_idx: torch.Tensor, E: int, R: int, capacity: int = 
         _ptr(out["expert_counts"]), _ptr(out["expert_src_counts"]), _ptr(out["rank_counts"]),
         _ptr(out["expert_offsets"]), _ptr(out["dispatch_pos"]), _ptr(out["recv_src"]),
         _ptr(ws), ws.numel(), _ptr(dev_status), _stream(stream)), "moe_dispatch_layout")
+    out["rows"] = rows
+    return out
+
+
+def moe_dispatch_layout_noalloc(topk_idx: torch.Tensor, E: int, R: int, capacity: int = 0,
+                                rows: int | None = None, out: dict | None = None,
+                                dev_status: torch.Tensor | None = None, stream=None) -> dict:
+    """moe_dispatch_layout without a workspace, for callers that cannot
+    allocate device memory: the library's fixed 1 MiB device scratch is used
+    instead (see include/moe_route.h).  Calls that overlap on the GPU race on
+    that scratch."""
+    assert topk_idx.dtype == torch.int32 and topk_idx.dim() == 2
+    T, k = topk_idx.shape
+    dev = topk_idx.device
+    if rows is None:
+        rows = T * k if capacity == 0 else E * capacity
+    if out is None:
+        out = dict(
+            expert_counts=torch.empty(E, dtype=torch.int32, device=dev),
+            expert_src_counts=torch.empty(E, R, dtype=torch.int32, device=dev),
+            rank_counts=torch.empty(R, dtype=torch.int32, device=dev),
+            expert_offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
+            dispatch_pos=torch.empty(T, k, dtype=torch.int32, device=dev),
+            recv_src=torch.empty(max(rows, 1), dtype=torch.int32, device=dev),
+        )
+    _check(lib.moe_dispatch_layout_noalloc(
+        _ptr(topk_idx), T, k, E, R, capacity, rows,
+        _ptr(out["expert_counts"]), _ptr(out["expert_src_counts"]), _ptr(out["rank_counts"]),
+        _ptr(out["expert_offsets"]), _ptr(out["dispatch_pos"]), _ptr(out["recv_src"]),
+        _ptr(dev_status), _stream(stream)), "moe_dispatch_layout_noalloc")
     out["rows"] = rows
     return out
 

@@ -147,6 +147,43 @@ int moe_dispatch_layout(const int32_t *topk_idx, int T, int k, int E, int R,
                         int32_t *dev_status, void *stream);
 
 /*
+ * moe_dispatch_layout_noalloc -- moe_dispatch_layout for callers that cannot
+ * allocate device memory.  The pages have no counterpart: this is a
+ * deployment variant of the entry point above, not a step of the method.
+ *
+ * Some callers cannot hand the layout a workspace: a plugin or custom-op
+ * layer that receives only its input and output buffers and no allocator,
+ * a host callback or latency-critical loop where cudaMalloc would
+ * synchronise the device, a deployment whose device memory is budgeted up
+ * front.  This entry point takes the same arguments as moe_dispatch_layout
+ * minus the workspace, and allocates nothing (no cudaMalloc, no cudaFree,
+ * no allocating library call).  Its scratch is a file-scope __device__
+ * array of MOE_LAYOUT_NOALLOC_SCRATCH_BYTES (1 MiB) inside this library:
+ * every GPU that loads the library holds it until the process exits.
+ *
+ *   - Limit: (T, k, E, R) whose moe_layout_workspace_bytes exceeds
+ *     MOE_LAYOUT_NOALLOC_SCRATCH_BYTES are rejected with MOE_ERR_WORKSPACE
+ *     before anything is enqueued (e.g. E = 256 fits up to 1024 chunks of at
+ *     most 8192 slots each; every workload of the benchmark fits).
+ *   - Set-up: the first call on each device looks the array's device address
+ *     up (cudaGetSymbolAddress, with that device current) and keeps it; make
+ *     that first call before any stream capture on that device.
+ *   - Sharing: all calls share the one array and it keeps the last call's
+ *     contents.  Each call rewrites every scratch word it reads, so nothing
+ *     needs clearing, but two calls whose kernels overlap on the GPU (other
+ *     streams, other host threads) race on the array: serialise them.
+ *   - Arguments, outputs and errors are otherwise those of
+ *     moe_dispatch_layout.
+ */
+#define MOE_LAYOUT_NOALLOC_SCRATCH_BYTES ((size_t)1 << 20)
+
+int moe_dispatch_layout_noalloc(const int32_t *topk_idx, int T, int k, int E, int R,
+                                int capacity, int64_t rows, int32_t *expert_counts,
+                                int32_t *expert_src_counts, int32_t *rank_counts,
+                                int32_t *expert_offsets, int32_t *dispatch_pos,
+                                int32_t *recv_src, int32_t *dev_status, void *stream);
+
+/*
  * moe_dispatch_bf16 -- row scatter: recv_x[dispatch_pos[g][j]] = x[g].
  * Follows "Enabling trillion-parameter models on AWS EFA", "Dağıtım ve
  * Birleştirme" (tokens packed into contiguous per-expert buffers) and
