@@ -1,6 +1,9 @@
 """Build libmoe_route.so in-tree with nvcc for sm_100a.
 
-    python -m combine_moe_route_08_b200.build [--force]
+    python combine_moe_route_08_b200/build.py [--force] [--ptxas-v]
+
+(Run as a script or load it by path: importing the package itself requires
+the library to exist already.)
 
 Floating-point flags: no flush-to-zero, IEEE division and square root, and
 no FMA contraction, so the bit-exact paths (fp8 scales and codes, the fp32

@@ -8,7 +8,7 @@ import re
 import pytest
 import torch
 
-from conftest import ROOT
+from conftest import ROOT, build_cuda_lib
 
 HEADER = os.path.join(ROOT, "include", "moe_route.h")
 
@@ -20,8 +20,7 @@ A4 = 0x10004
 
 @pytest.fixture(scope="module")
 def moe():
-    from combine_moe_route_08_b200 import build
-    build.build()
+    build_cuda_lib()
     import combine_moe_route_08_b200 as m
     return m
 
