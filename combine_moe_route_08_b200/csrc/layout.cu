@@ -19,18 +19,25 @@
 // 32 warps a contiguous run of at most 8 x 32 slots, which every lane keeps in
 // registers (one load round trip per kernel).
 //
-//   k_layout_hist    chunk histogram (per-warp __match_any_sync aggregation,
+//   k_layout_hist    chunk histogram (per-warp aggregation of equal experts,
 //                    shared-memory atomics) -> workspace hist[chunk][E].
 //   k_layout_assign  every CTA sums the histogram columns it needs (the base
-//                    of its chunk inside each expert, the expert totals) --
-//                    redundant but parallel, no serial tail -- scans the
-//                    totals into offsets, builds per-warp histograms of its
-//                    own slots, scans them over the warps, and ranks each
-//                    slot among the equal experts of its warp step
-//                    (__match_any_sync + popc of the lower lanes) to get its
-//                    row.  CTA 0 also writes counts, offsets and rank sums.
+//                    of its chunk inside each expert, the expert totals, its
+//                    rank's source counts) with all its threads -- redundant
+//                    but parallel, no serial tail -- scans the totals into
+//                    offsets, builds per-warp histograms of its own slots,
+//                    scans them over the warps, and ranks each slot among the
+//                    equal experts of its warp step (equality mask + popc of
+//                    the lower lanes) to get its row.  CTA 0 also writes
+//                    counts, offsets and rank sums; the first chunk of each
+//                    rank writes that rank's source-count column.
 // The kernel boundary between the two is the only grid-wide ordering; nothing
 // waits on another CTA.
+//
+// The equality mask of a warp step ("which lanes hold my expert") is built
+// from one __ballot_sync per key bit; __match_any_sync would give the same
+// mask but costs about 2000 cycles per call on this part (measured with
+// clock64 stamps), which dominated the kernel.
 #include <algorithm>
 
 #include "common.cuh"
@@ -86,11 +93,30 @@ __device__ __forceinline__ void load_run(const int32_t *__restrict__ topk_idx, i
     }
 }
 
-// Key for __match_any_sync: the expert, or a value no expert and no other
-// lane uses for slots that are empty, masked or invalid.
-__device__ __forceinline__ int match_key(int e, int E, int lane)
+// Lanes of the warp holding the same key as this lane.  __match_any_sync is
+// slow on this part (thousands of cycles per call), so the equality mask is
+// built from one ballot per key bit: a lane matches where every bit agrees.
+__device__ __forceinline__ unsigned match_mask(int key, int nbits)
 {
-    return (static_cast<unsigned>(e) < static_cast<unsigned>(E)) ? e : (0x40000000 | lane);
+    unsigned mask = kFullMask;
+    for (int b = 0; b < nbits; ++b) {
+        const bool bit = (key >> b) & 1;
+        const unsigned bal = __ballot_sync(kFullMask, bit);
+        mask &= bit ? bal : ~bal;
+    }
+    return mask;
+}
+
+// Key bits: enough for max(E - 1, 31), plus one bit that marks a slot that
+// is empty, masked or invalid (key = lane | that bit, unique in the warp).
+__device__ __forceinline__ int key_bits(int E)
+{
+    return 32 - __clz(max(E - 1, 31)) + 1;
+}
+
+__device__ __forceinline__ int match_key(int e, int E, int lane, int nbits)
+{
+    return (static_cast<unsigned>(e) < static_cast<unsigned>(E)) ? e : (lane | (1 << (nbits - 1)));
 }
 
 __global__ void __launch_bounds__(kThreads)
@@ -100,6 +126,7 @@ __global__ void __launch_bounds__(kThreads)
     extern __shared__ int32_t h[];  // [E]
     const int E = G.E, lane = threadIdx.x & 31;
     const int c = blockIdx.x;
+    const int nb = key_bits(E);
     int64_t w0, w1;
     warp_run(G, c, w0, w1);
     int e[kMaxSteps];
@@ -115,7 +142,7 @@ __global__ void __launch_bounds__(kThreads)
             break;  // warp-uniform
         const bool valid = static_cast<unsigned>(e[s]) < static_cast<unsigned>(E);
         bad |= !valid && e[s] != -1 && (w0 + 32 * s + lane < w1);
-        const unsigned mask = __match_any_sync(kFullMask, match_key(e[s], E, lane));
+        const unsigned mask = match_mask(match_key(e[s], E, lane, nb), nb);
         if (valid && lane == __ffs(mask) - 1)
             atomicAdd(&h[e[s]], __popc(mask));
     }
@@ -172,6 +199,7 @@ __global__ void __launch_bounds__(kThreads)
 {
     extern __shared__ int32_t sm[];
     const int E = G.E, lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const int nb = key_bits(E);
     int32_t *wh = sm;                   // [kWarps][E] per-warp counts, then bases
     int32_t *off = wh + kWarps * E;     // [E + 1] expert totals, then their scan
     int32_t *chb = off + E + 1;         // [E] slots of e in earlier chunks
@@ -183,40 +211,60 @@ __global__ void __launch_bounds__(kThreads)
     int e[kMaxSteps];
     load_run(topk_idx, w0, w1, e);  // in flight while the columns are summed
 
-    for (int x = threadIdx.x; x < kWarps * E; x += kThreads)
+    for (int x = threadIdx.x + 3 * max(1, min(kThreads / E, kWarps / 3)) * E; x < kWarps * E;
+         x += kThreads)
         wh[x] = 0;
 
-    // histogram columns: base of this chunk inside each expert, expert totals,
-    // and (CTA 0) the per-source-rank counts
+    // histogram columns: base of this chunk inside each expert (earlier
+    // chunks), expert totals, and this chunk's rank column of the
+    // per-source-rank counts.  P threads per expert each sum a contiguous
+    // part of the chunks (coalesced over experts); the parts meet in shared
+    // memory (the per-warp rows, not yet used).
     const int n = G.nchunks;
-    for (int x = threadIdx.x; x < E; x += kThreads) {
-        int before = 0, total = 0, rank_sum = 0, next_rank_end = G.cpr;
-        for (int c0 = 0; c0 < n; c0 += kColBatch) {
-            int v[kColBatch];
+    const int P = max(1, min(kThreads / E, kWarps / 3));
+    const int r = c / G.cpr;
+    {
+        const int x = threadIdx.x % E, part = threadIdx.x / E;
+        if (part < P) {
+            const int per = ceil_div(n, P);
+            const int cb = part * per, ce = min(n, cb + per);
+            int before = 0, total = 0, mine = 0;
+            for (int c0 = cb; c0 < ce; c0 += kColBatch) {
+                int v[kColBatch];
 #pragma unroll
-            for (int u = 0; u < kColBatch; ++u)
-                v[u] = (c0 + u < n) ? __ldg(ws_hist + static_cast<size_t>(c0 + u) * E + x) : 0;
+                for (int u = 0; u < kColBatch; ++u)
+                    v[u] = (c0 + u < ce) ? __ldg(ws_hist + static_cast<size_t>(c0 + u) * E + x) : 0;
 #pragma unroll
-            for (int u = 0; u < kColBatch; ++u) {
-                const int cc = c0 + u;
-                if (cc < c)
-                    before += v[u];
-                total += v[u];
-                if (c == 0 && cc < n) {
-                    rank_sum += v[u];
-                    if (cc + 1 == next_rank_end) {
-                        expert_src_counts[static_cast<size_t>(x) * G.R + cc / G.cpr] = rank_sum;
-                        rank_sum = 0;
-                        next_rank_end += G.cpr;
-                    }
+                for (int u = 0; u < kColBatch; ++u) {
+                    const int cc = c0 + u;
+                    before += (cc < c) ? v[u] : 0;
+                    total += v[u];
+                    mine += (cc >= r * G.cpr && cc < (r + 1) * G.cpr) ? v[u] : 0;
                 }
             }
+            wh[(3 * part) * E + x] = before;
+            wh[(3 * part + 1) * E + x] = total;
+            wh[(3 * part + 2) * E + x] = mine;
+        }
+    }
+    __syncthreads();
+    for (int x = threadIdx.x; x < E; x += kThreads) {
+        int before = 0, total = 0, mine = 0;
+        for (int part = 0; part < P; ++part) {
+            before += wh[(3 * part) * E + x];
+            total += wh[(3 * part + 1) * E + x];
+            mine += wh[(3 * part + 2) * E + x];
         }
         off[x] = total;
         chb[x] = before;
         if (c == 0)
             expert_counts[x] = total;
+        if (c == r * G.cpr)  // first chunk of its rank writes the rank's column
+            expert_src_counts[static_cast<size_t>(x) * G.R + r] = mine;
     }
+    __syncthreads();
+    for (int x = threadIdx.x; x < 3 * P * E; x += kThreads)
+        wh[x] = 0;
     __syncthreads();
 
     // per-warp histogram of this CTA's slots (warp-private rows: no atomics)
@@ -226,7 +274,7 @@ __global__ void __launch_bounds__(kThreads)
         if (w0 + 32 * s >= w1)
             break;
         const bool valid = static_cast<unsigned>(e[s]) < static_cast<unsigned>(E);
-        const unsigned mask = __match_any_sync(kFullMask, match_key(e[s], E, lane));
+        const unsigned mask = match_mask(match_key(e[s], E, lane, nb), nb);
         if (valid && lane == __ffs(mask) - 1)
             mywh[e[s]] += __popc(mask);
         __syncwarp();
@@ -237,8 +285,8 @@ __global__ void __launch_bounds__(kThreads)
         for (int x = threadIdx.x; x <= E; x += kThreads)
             expert_offsets[x] = (capacity == 0) ? off[x] : x * capacity;
         const int L = E / G.R;
-        for (int r = threadIdx.x; r < G.R; r += kThreads)
-            rank_counts[r] = off[(r + 1) * L] - off[r * L];
+        for (int rr = threadIdx.x; rr < G.R; rr += kThreads)
+            rank_counts[rr] = off[(rr + 1) * L] - off[rr * L];
     }
     // per-warp base of each expert's positions: earlier chunks + earlier warps
     for (int x = threadIdx.x; x < E; x += kThreads) {
@@ -260,7 +308,7 @@ __global__ void __launch_bounds__(kThreads)
             break;
         const int64_t i = w0 + 32 * s + lane;
         const bool valid = static_cast<unsigned>(e[s]) < static_cast<unsigned>(E);
-        const unsigned mask = __match_any_sync(kFullMask, match_key(e[s], E, lane));
+        const unsigned mask = match_mask(match_key(e[s], E, lane, nb), nb);
         const int p = valid ? mywh[e[s]] + __popc(mask & lanemask_lt()) : 0;
         __syncwarp();
         if (valid && lane == __ffs(mask) - 1)

@@ -6,9 +6,11 @@
 // precision (DeepSeek-V3 fragments): fp32 logits in, fp32 weights out.
 //
 // Each lane holds the logits e = i*32 + lane (a warp-wide load per i is one
-// coalesced 128-byte line).  k rounds of warp arg-max under the order (logit
-// descending, index ascending) pick the experts; a per-lane bit mask removes
-// the winners.
+// coalesced 128-byte line), as order-preserving 32-bit keys.  k rounds of
+// warp arg-max under the order (logit descending, index ascending) pick the
+// experts: one warp-wide max of the lanes' best keys and one warp-wide min of
+// the indices holding it (redux.sync, a single instruction each), then the
+// winner's key is cleared.
 //
 // The softmax is evaluated in fp32 with its error bounded (u = 2^-24):
 //   d = l - m is split exactly into d_hi + d_lo (Knuth's TwoSum), so the
@@ -19,7 +21,6 @@
 //   |w - p| <= 13u * p (+ O(u^2)) for the exact probability p, i.e. within 16
 //   fp32 ulps of the correctly rounded value; in practice 1-2 ulps.
 #include <cfloat>
-#include <climits>
 
 #include "common.cuh"
 #include "kernels.cuh"
@@ -29,20 +30,6 @@ namespace moe {
 namespace {
 
 constexpr int kRouteWarps = 8;  // tokens per CTA
-
-struct Cand {
-    float v;
-    int e;  // INT_MAX: no candidate
-};
-
-__device__ __forceinline__ bool better(const Cand &a, const Cand &b)
-{
-    if (a.e == INT_MAX)
-        return false;
-    if (b.e == INT_MAX)
-        return true;
-    return a.v > b.v || (a.v == b.v && a.e < b.e);
-}
 
 // a + b == s + err exactly (Knuth's TwoSum; explicit _rn ops are never
 // contracted or reassociated)
@@ -100,34 +87,50 @@ __global__ void __launch_bounds__(kRouteWarps * 32)
         }
     }
 
+    // selection on order-preserving 32-bit keys: larger logit -> larger key,
+    // -0 and +0 the same key (x + 0.0f turns -0 into +0); key 0 = taken/absent
+    uint32_t key[NPL];
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
+        if ((gone >> i) & 1u) {
+            key[i] = 0u;
+        } else {
+            const uint32_t u = __float_as_uint(__fadd_rn(v[i], 0.0f));
+            key[i] = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+        }
+    }
     int my_e = 0;
     float my_v = 0.0f;
     float vmax = 0.0f;
     for (int j = 0; j < k; ++j) {
-        Cand best{-FLT_MAX, INT_MAX};
+        uint32_t best = 0u;
+#pragma unroll
+        for (int i = 0; i < NPL; ++i)
+            best = max(best, key[i]);
+        const uint32_t m = __reduce_max_sync(kFullMask, best);
+        uint32_t cand = 0xffffffffu;
+#pragma unroll
+        for (int i = NPL - 1; i >= 0; --i)
+            if (key[i] == m)
+                cand = static_cast<uint32_t>(i * 32 + lane);
+        const uint32_t e = __reduce_min_sync(kFullMask, cand);
+        const int ei = static_cast<int>(e >> 5);
+        float ve = 0.0f;
 #pragma unroll
         for (int i = 0; i < NPL; ++i) {
-            // e grows with i: a strict '>' keeps the lower index on ties
-            if (!((gone >> i) & 1u) && (best.e == INT_MAX || v[i] > best.v))
-                best = Cand{v[i], i * 32 + lane};
+            if (i == ei && (e & 31u) == static_cast<uint32_t>(lane)) {
+                key[i] = 0u;
+            }
+            if (i == ei)
+                ve = v[i];
         }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            Cand o;
-            o.v = __shfl_xor_sync(kFullMask, best.v, off);
-            o.e = __shfl_xor_sync(kFullMask, best.e, off);
-            if (better(o, best))
-                best = o;
-        }
-        // k <= E: every round has a winner
-        if ((best.e & 31) == lane)
-            gone |= 1u << (best.e >> 5);
+        ve = __shfl_sync(kFullMask, ve, static_cast<int>(e & 31u));
         if (lane == j) {
-            my_e = best.e;
-            my_v = best.v;
+            my_e = static_cast<int>(e);
+            my_v = ve;
         }
         if (j == 0)
-            vmax = best.v;
+            vmax = ve;
     }
 
     // softmax over all E logits, in fp32 with compensated summation
