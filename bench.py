@@ -382,11 +382,23 @@ def run_ours(args) -> None:
         if flush_needed:
             flush.buf.fill_(i)
     flush.buf = flush_buf
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+
+    # one step = one replay of a CUDA graph holding the four C ABI calls (the
+    # library launches its kernels with programmatic dependent launch)
+    with torch.cuda.stream(s):
+        for i in range(2):
+            step()
+    s.synchronize()
+    g_step = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_step, stream=s):
+        step()
+
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(K)]
     with torch.cuda.stream(s):
         for i in range(W):
             flush(i)
-            step()
+            g_step.replay()
         s.synchronize()
         sampler = ClockSampler(local)
         sampler.start()
@@ -396,40 +408,64 @@ def run_ours(args) -> None:
         for i in range(K):
             flush(i)
             evs[i][0].record(s)
-            step(evs[i])
-            evs[i][4].record(s)
+            g_step.replay()
+            evs[i][1].record(s)
         s.synchronize()
         torch.cuda.synchronize(dev)
         barrier(world, dev)
         sampler.mark_end()
         clocks = sampler.stop()
+    local_step = float(np.mean([a.elapsed_time(b) for a, b in evs]))
 
-    stage_ms = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(4)] for e in evs])
-    step_ms = stage_ms.sum(1)
-    local_ms = [float(step_ms.mean()), *[float(v) for v in stage_ms.mean(0)]]
-    ms = max_over_ranks(local_ms, world, dev)
-    ms_step, ms_route, ms_layout, ms_dispatch, ms_combine = ms
-
-    # ---- CUDA graph of the same step (launch overhead removed) ----
-    graph_ms = None
-    if not args.no_graph:
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=s):
-            step()
-        gt = []
+    # per-stage breakdown: the same step captured with timing events between
+    # the stages (event record nodes inside the graph), replayed and read back
+    # one step at a time
+    K2 = min(K, 200)
+    stage_ms = None
+    try:
+        xev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(5)]
+        g_st = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_st, stream=s):
+            xev[0].record(s)
+            step(xev)
+            xev[4].record(s)
+        rows_ms = []
         with torch.cuda.stream(s):
-            for i in range(max(W, 3)):
-                g.replay()
-            for i in range(min(K, 200)):
+            for i in range(K2 + 3):
                 flush(i)
-                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                a.record(s)
-                g.replay()
-                b.record(s)
-                gt.append((a, b))
+                g_st.replay()
+                s.synchronize()
+                if i >= 3:
+                    rows_ms.append([xev[j].elapsed_time(xev[j + 1]) for j in range(4)])
+        stage_ms = np.array(rows_ms).mean(0)
+        stage_how = "event record nodes between the stages inside the step graph"
+        del g_st
+    except (RuntimeError, TypeError):
+        stage_ms = None
+    if stage_ms is None:  # one graph per stage, events between replays
+        gs = []
+        for j, (fn, a) in enumerate(calls):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=s):
+                fn(*a)
+            gs.append(g)
+        rows_ms = []
+        with torch.cuda.stream(s):
+            for i in range(K2):
+                flush(i)
+                e = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+                e[0].record(s)
+                for j, g in enumerate(gs):
+                    g.replay()
+                    e[j + 1].record(s)
+                rows_ms.append(e)
             s.synchronize()
-        graph_ms = max_over_ranks([float(np.mean([a.elapsed_time(b) for a, b in gt]))], world, dev)[0]
-        del g
+        stage_ms = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(4)] for e in rows_ms]).mean(0)
+        stage_how = "one graph per stage, events between the replays"
+        del gs
+    ms = max_over_ranks([local_step, *[float(v) for v in stage_ms]], world, dev)
+    ms_step, ms_route, ms_layout, ms_dispatch, ms_combine = ms
+    del g_step
 
     # ---- end to end through the public API, host buffers in and out ----
     logits_pin = logits_h.pin_memory()
@@ -467,7 +503,7 @@ def run_ours(args) -> None:
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": cfg.describe(), "parallelism": f"replicas x{n_gpus}",
                        "l2": l2_mode,
-                       "capacity": cap, "rows": rows, "timing": "CUDA events per stage, eager launches"},
+                       "capacity": cap, "rows": rows, "timing": "CUDA events around each replay of the step's CUDA graph"},
             "us_per_layer": ms_step * 1e3,
             "stages_us": {"route": ms_route * 1e3, "layout": ms_layout * 1e3,
                           "dispatch": ms_dispatch * 1e3, "combine": ms_combine * 1e3},
@@ -475,7 +511,7 @@ def run_ours(args) -> None:
                                  "gbs": dc_bytes / (dc_ms * 1e-3) / 1e9,
                                  "frac_of_8tbs": dc_bytes / (dc_ms * 1e-3) / 1e9 / SPEC_HBM_GBS,
                                  "frac_of_measured": dc_bytes / (dc_ms * 1e-3) / 1e9 / peak},
-            "graph_us_per_layer": graph_ms * 1e3 if graph_ms else None,
+            "stage_timing": stage_how,
             "bytes_per_step": nb,
             "roofline": {"bound": "hbm", "kernel": "k_combine_bf16", "achieved": comb_gbs,
                          "peak": peak, "unit": "GB/s", "frac": comb_gbs / peak,
@@ -505,7 +541,6 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", choices=sorted(inputs.CONFIGS), default="dsv3")
-    ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3:

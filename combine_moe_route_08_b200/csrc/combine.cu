@@ -32,6 +32,7 @@ __global__ void __launch_bounds__(kMaxThreads)
     __shared__ int32_t srow[kMaxK];
     __shared__ float sw[kMaxK];
     const int g = blockIdx.x;
+    pdl_wait();
     if (threadIdx.x < k) {
         int r = dispatch_pos[static_cast<size_t>(g) * k + threadIdx.x];
         if (r < -1 || r >= rows) {
@@ -75,6 +76,7 @@ __global__ void __launch_bounds__(kMaxThreads)
                                    bf16x2_rn(acc[4], acc[5]), bf16x2_rn(acc[6], acc[7]));
         st_stream_v4(out + static_cast<size_t>(g) * nvec + v, o);
     }
+    pdl_trigger();
 }
 
 int threads_for(int units)
@@ -90,10 +92,9 @@ cudaError_t combine_bf16(const uint16_t *y, const int32_t *dispatch_pos, const f
                          cudaStream_t s)
 {
     const int nvec = H / 8;
-    k_combine_bf16<<<T, threads_for(nvec), 0, s>>>(reinterpret_cast<const uint4 *>(y), dispatch_pos,
-                                                   topk_w, nvec, k, rows,
-                                                   reinterpret_cast<uint4 *>(out), dev_status);
-    return cudaGetLastError();
+    return launch_pdl(k_combine_bf16, dim3(T), dim3(threads_for(nvec)), 0, s,
+                      reinterpret_cast<const uint4 *>(y), dispatch_pos, topk_w, nvec, k, rows,
+                      reinterpret_cast<uint4 *>(out), dev_status);
 }
 
 }  // namespace moe

@@ -26,6 +26,7 @@ constexpr int kMaxThreads = 512;
 __device__ __forceinline__ void load_rows(const int32_t *__restrict__ dispatch_pos, int g, int k,
                                           int64_t rows, int32_t *srow, int32_t *dev_status)
 {
+    pdl_wait();
     if (threadIdx.x < k) {
         int r = dispatch_pos[static_cast<size_t>(g) * k + threadIdx.x];
         if (r < -1 || r >= rows) {
@@ -54,6 +55,7 @@ __global__ void __launch_bounds__(kMaxThreads)
                 st_stream_v4(recv_x + static_cast<size_t>(r) * nvec + v, d);
         }
     }
+    pdl_trigger();
 }
 
 // Thread t of the token owns channels [16t, 16t + 16); the 8 threads of one
@@ -115,6 +117,7 @@ __global__ void __launch_bounds__(kMaxThreads)
             }
         }
     }
+    pdl_trigger();
 }
 
 __global__ void k_quantize_e4m3(const float *__restrict__ v, int64_t n, uint8_t *__restrict__ q)
@@ -146,20 +149,18 @@ cudaError_t dispatch_bf16(const uint16_t *x, int T, int H, int k, const int32_t 
                           uint16_t *recv_x, int64_t rows, int32_t *dev_status, cudaStream_t s)
 {
     const int nvec = H / 8;
-    k_dispatch_bf16<<<T, threads_for(nvec), 0, s>>>(reinterpret_cast<const uint4 *>(x), nvec, k,
-                                                    dispatch_pos, reinterpret_cast<uint4 *>(recv_x),
-                                                    rows, dev_status);
-    return cudaGetLastError();
+    return launch_pdl(k_dispatch_bf16, dim3(T), dim3(threads_for(nvec)), 0, s,
+                      reinterpret_cast<const uint4 *>(x), nvec, k, dispatch_pos,
+                      reinterpret_cast<uint4 *>(recv_x), rows, dev_status);
 }
 
 cudaError_t dispatch_fp8(const uint16_t *x, int T, int H, int k, const int32_t *dispatch_pos,
                          uint8_t *recv_q, float *recv_scale, int64_t rows, int32_t *dev_status,
                          cudaStream_t s)
 {
-    k_dispatch_fp8<<<T, threads_for(H / 16), 0, s>>>(reinterpret_cast<const uint4 *>(x), H, k,
-                                                     dispatch_pos, recv_q, recv_scale, rows,
-                                                     dev_status);
-    return cudaGetLastError();
+    return launch_pdl(k_dispatch_fp8, dim3(T), dim3(threads_for(H / 16)), 0, s,
+                      reinterpret_cast<const uint4 *>(x), H, k, dispatch_pos, recv_q, recv_scale,
+                      rows, dev_status);
 }
 
 cudaError_t quantize_e4m3(const float *v, int64_t n, uint8_t *q, cudaStream_t s)

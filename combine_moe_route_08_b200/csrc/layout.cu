@@ -129,10 +129,11 @@ __global__ void __launch_bounds__(kThreads)
     const int nb = key_bits(E);
     int64_t w0, w1;
     warp_run(G, c, w0, w1);
-    int e[kMaxSteps];
-    load_run(topk_idx, w0, w1, e);
     for (int x = threadIdx.x; x < E; x += kThreads)
         h[x] = 0;
+    pdl_wait();
+    int e[kMaxSteps];
+    load_run(topk_idx, w0, w1, e);
     __syncthreads();
 
     bool bad = false;
@@ -151,6 +152,7 @@ __global__ void __launch_bounds__(kThreads)
     __syncthreads();
     for (int x = threadIdx.x; x < E; x += kThreads)
         ws_hist[static_cast<size_t>(c) * E + x] = h[x];
+    pdl_trigger();
 }
 
 // In-place exclusive scan of a[0..n) (n <= kThreads) by the whole CTA; a[n]
@@ -208,6 +210,7 @@ __global__ void __launch_bounds__(kThreads)
 
     int64_t w0, w1;
     warp_run(G, c, w0, w1);
+    pdl_wait();
     int e[kMaxSteps];
     load_run(topk_idx, w0, w1, e);  // in flight while the columns are summed
 
@@ -353,6 +356,7 @@ __global__ void __launch_bounds__(kThreads)
         for (int64_t r = static_cast<int64_t>(E) * capacity + first; r < rows; r += stride)
             recv_src[r] = -1;
     }
+    pdl_trigger();
 }
 
 size_t assign_smem_bytes(int E) { return (static_cast<size_t>(kWarps + 2) * E + 1 + kWarps + 1) * sizeof(int32_t); }
@@ -386,8 +390,8 @@ cudaError_t dispatch_layout(const int32_t *topk_idx, const LayoutGeom &g, int ca
                             cudaStream_t s)
 {
     int32_t *hist = static_cast<int32_t *>(workspace);
-    k_layout_hist<<<g.nchunks, kThreads, g.E * sizeof(int32_t), s>>>(topk_idx, g, hist, dev_status);
-    cudaError_t err = cudaGetLastError();
+    cudaError_t err = launch_pdl(k_layout_hist, dim3(g.nchunks), dim3(kThreads), g.E * sizeof(int32_t),
+                                 s, topk_idx, g, hist, dev_status);
     if (err != cudaSuccess)
         return err;
     const size_t smem = assign_smem_bytes(g.E);
@@ -397,11 +401,9 @@ cudaError_t dispatch_layout(const int32_t *topk_idx, const LayoutGeom &g, int ca
         if (err != cudaSuccess)
             return err;
     }
-    k_layout_assign<<<g.nchunks, kThreads, smem, s>>>(topk_idx, g, capacity, rows, hist,
-                                                      expert_counts, expert_src_counts, rank_counts,
-                                                      expert_offsets, dispatch_pos, recv_src,
-                                                      dev_status);
-    return cudaGetLastError();
+    return launch_pdl(k_layout_assign, dim3(g.nchunks), dim3(kThreads), smem, s, topk_idx, g, capacity,
+                      rows, hist, expert_counts, expert_src_counts, rank_counts, expert_offsets,
+                      dispatch_pos, recv_src, dev_status);
 }
 
 }  // namespace moe

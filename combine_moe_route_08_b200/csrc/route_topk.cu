@@ -70,9 +70,13 @@ __global__ void __launch_bounds__(kRouteWarps * 32)
 {
     const int lane = threadIdx.x & 31;
     const int g = blockIdx.x * kRouteWarps + (threadIdx.x >> 5);
-    if (g >= T)
+    if (g >= T) {
+        pdl_wait();
+        pdl_trigger();
         return;  // warp-uniform
+    }
     const float *row = logits + static_cast<size_t>(g) * E;
+    pdl_wait();
 
     float v[NPL];
     uint32_t gone = 0;  // bit i: element i taken or past E
@@ -164,6 +168,7 @@ __global__ void __launch_bounds__(kRouteWarps * 32)
         topk_idx[static_cast<size_t>(g) * k + lane] = my_e;
         topk_w[static_cast<size_t>(g) * k + lane] = __fdiv_rn(num, denom);
     }
+    pdl_trigger();
 }
 
 template <int NPL>
@@ -171,8 +176,8 @@ cudaError_t launch(const float *logits, int T, int E, int k, int renormalize, in
                    float *w, cudaStream_t s)
 {
     const int grid = ceil_div(T, kRouteWarps);
-    k_route_topk<NPL><<<grid, kRouteWarps * 32, 0, s>>>(logits, T, E, k, renormalize, idx, w);
-    return cudaGetLastError();
+    return launch_pdl(k_route_topk<NPL>, dim3(grid), dim3(kRouteWarps * 32), 0, s, logits, T, E, k,
+                      renormalize, idx, w);
 }
 
 }  // namespace
