@@ -52,6 +52,7 @@ SPEC_HBM_GBS = 8000.0          # B200 HBM3e bandwidth the roofline target is quo
 FALLBACK_HBM_GBS = 6650.0      # earlier measured copy bandwidth on this machine
 L2_FLUSH_BYTES = 512 << 20
 KERNELS_PER_STEP = 5           # route, layout (2 kernels), dispatch, combine
+STEPS_PER_GRAPH = 10           # consecutive steps captured in one CUDA graph (no-flush workloads)
 
 
 # --------------------------------------------------------------------------
@@ -383,62 +384,93 @@ def run_ours(args) -> None:
             flush.buf.fill_(i)
     flush.buf = flush_buf
 
-    # one step = one replay of a CUDA graph holding the four C ABI calls (the
-    # library launches its kernels with programmatic dependent launch)
+    # Steps run as replays of CUDA graphs of the four C ABI calls (the library
+    # launches its kernels with programmatic dependent launch).  Workloads
+    # timed without an L2 flush put STEPS_PER_GRAPH consecutive steps in one
+    # graph, as a model forward puts many layers in one graph, so the graph
+    # launch latency is not paid per step; a 1-step graph runs the remainder.
+    # Flushed workloads replay one step per graph with the flush in between.
+    G = STEPS_PER_GRAPH if not flush_needed else 1
     with torch.cuda.stream(s):
         for i in range(2):
             step()
     s.synchronize()
-    g_step = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_step, stream=s):
-        step()
 
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(K)]
+    def capture(fn, n):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            for _ in range(n):
+                fn()
+        return g
+
+    def timed_replays(g_many, g_one, n_steps):
+        """n_steps steps as replays; returns per-step events (or region events)."""
+        if G == 1:
+            evs = []
+            for i in range(n_steps):
+                flush(i)
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(s)
+                g_one.replay()
+                b.record(s)
+                evs.append((a, b))
+            return evs
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(s)
+        for _ in range(n_steps // G):
+            g_many.replay()
+        for _ in range(n_steps % G):
+            g_one.replay()
+        b.record(s)
+        return [(a, b)]
+
+    def ms_per(evs, n_steps):
+        return float(sum(a.elapsed_time(b) for a, b in evs)) / n_steps
+
+    g_step1 = capture(step, 1)
+    g_stepG = capture(step, G) if G > 1 else g_step1
     with torch.cuda.stream(s):
-        for i in range(W):
-            flush(i)
-            g_step.replay()
+        timed_replays(g_stepG, g_step1, W)          # warm-up
         s.synchronize()
         sampler = ClockSampler(local)
         sampler.start()
         barrier(world, dev)
         torch.cuda.synchronize(dev)
         sampler.mark_start()
-        for i in range(K):
-            flush(i)
-            evs[i][0].record(s)
-            g_step.replay()
-            evs[i][1].record(s)
+        evs = timed_replays(g_stepG, g_step1, K)
         s.synchronize()
         torch.cuda.synchronize(dev)
         barrier(world, dev)
         sampler.mark_end()
         clocks = sampler.stop()
-    local_step = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    local_step = ms_per(evs, K)
 
-    # per-stage breakdown: the same step captured with timing events between
-    # the stages (event record nodes inside the graph), replayed and read back
-    # one step at a time
+    # per-stage breakdown: G consecutive steps captured with timing events
+    # between the stages (event record nodes inside the graph); each replay is
+    # read back before the next
     K2 = min(K, 200)
     stage_ms = None
     try:
-        xev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(5)]
+        xev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(5)]
+               for _ in range(G)]
         g_st = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g_st, stream=s):
-            xev[0].record(s)
-            step(xev)
-            xev[4].record(s)
+            for q in range(G):
+                xev[q][0].record(s)
+                step(xev[q])
+                xev[q][4].record(s)
         rows_ms = []
         with torch.cuda.stream(s):
-            for i in range(K2 + 3):
+            for i in range(max(1, K2 // G) + 2):
                 flush(i)
                 g_st.replay()
                 s.synchronize()
-                if i >= 3:
-                    rows_ms.append([xev[j].elapsed_time(xev[j + 1]) for j in range(4)])
+                if i >= 2:
+                    rows_ms += [[xev[q][j].elapsed_time(xev[q][j + 1]) for j in range(4)]
+                                for q in range(G)]
         stage_ms = np.array(rows_ms).mean(0)
-        stage_how = "event record nodes between the stages inside the step graph"
+        stage_how = (f"event record nodes between the stages of {G} consecutive step(s) "
+                     "inside one graph")
         del g_st
     except (RuntimeError, TypeError):
         stage_ms = None
@@ -464,29 +496,22 @@ def run_ours(args) -> None:
         stage_how = "one graph per stage, events between the replays"
         del gs
     # dispatch+combine as the pages count it (layout + dispatch + combine,
-    # route excluded): its own graph, K replays back to back
-    g_dc = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_dc, stream=s):
+    # route excluded): its own graphs, timed the same way
+    def dc_step():
         for fn, a in calls[1:]:
             rc = fn(*a)
             if rc != 0:
                 raise moe.MoeError(rc, fn.__name__)
-    dcev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-            for _ in range(K)]
+    g_dc1 = capture(dc_step, 1)
+    g_dcG = capture(dc_step, G) if G > 1 else g_dc1
     with torch.cuda.stream(s):
-        for i in range(W):
-            flush(i)
-            g_dc.replay()
-        for i in range(K):
-            flush(i)
-            dcev[i][0].record(s)
-            g_dc.replay()
-            dcev[i][1].record(s)
+        timed_replays(g_dcG, g_dc1, W)
+        dcev = timed_replays(g_dcG, g_dc1, K)
         s.synchronize()
-    local_dc = float(np.mean([a.elapsed_time(b) for a, b in dcev]))
+    local_dc = ms_per(dcev, K)
     ms = max_over_ranks([local_step, local_dc, *[float(v) for v in stage_ms]], world, dev)
     ms_step, ms_dc, ms_route, ms_layout, ms_dispatch, ms_combine = ms
-    del g_step, g_dc
+    del g_step1, g_stepG, g_dc1, g_dcG
 
     # ---- end to end through the public API, host buffers in and out ----
     logits_pin = logits_h.pin_memory()
@@ -524,12 +549,13 @@ def run_ours(args) -> None:
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": cfg.describe(), "parallelism": f"replicas x{n_gpus}",
                        "l2": l2_mode,
-                       "capacity": cap, "rows": rows, "timing": "CUDA events around each replay of the step's CUDA graph"},
+                       "capacity": cap, "rows": rows, "timing": (f"CUDA events around K steps run as replays of CUDA graphs of "
+                                  f"{G} consecutive step(s)")},
             "us_per_layer": ms_step * 1e3,
             "stages_us": {"route": ms_route * 1e3, "layout": ms_layout * 1e3,
                           "dispatch": ms_dispatch * 1e3, "combine": ms_combine * 1e3},
             "dispatch_combine": {"us": dc_ms * 1e3, "bytes": dc_bytes,
-                                 "how": "CUDA graph of layout + dispatch + combine, K replays back to back",
+                                 "how": "CUDA graphs of layout + dispatch + combine, K steps timed like the step",
                                  "gbs": dc_bytes / (dc_ms * 1e-3) / 1e9,
                                  "frac_of_8tbs": dc_bytes / (dc_ms * 1e-3) / 1e9 / SPEC_HBM_GBS,
                                  "frac_of_measured": dc_bytes / (dc_ms * 1e-3) / 1e9 / peak},
