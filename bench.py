@@ -62,10 +62,11 @@ STEPS_PER_GRAPH = 10           # consecutive steps captured in one CUDA graph (n
 def algorithmic_bytes(cfg: inputs.Config, rows: int, kept: int) -> dict:
     """Minimal bytes each stage must move.  kept = slots that have a row
     (T*k when nothing is dropped); rows = receive rows laid out."""
-    T, H, E, k, R = cfg.T, cfg.H, cfg.E, cfg.k, cfg.R
+    T, H, E, k, R = cfg.T, cfg.H, cfg.E, cfg.k_total, cfg.R
+    E_lay = cfg.E_phys if cfg.n_shared else E
     S = H // 128
     route = T * E * 4 + T * k * 8
-    layout = T * k * 4 + E * 4 * (2 + R) + 4 + R * 4 + T * k * 4 + rows * 4
+    layout = T * k * 4 + E_lay * 4 * (2 + R) + 4 + R * 4 + T * k * 4 + rows * 4
     if cfg.dispatch == "fp8":
         dispatch = T * H * 2 + T * k * 4 + kept * H + kept * S * 4
     else:
@@ -215,17 +216,22 @@ def oracle_step_on_sample(cfg: inputs.Config, wl: dict, tokens: int) -> tuple[fl
     import oracle
     sub = inputs.Config(cfg.name, cfg.index, tokens // cfg.R if tokens % cfg.R == 0 else tokens,
                         cfg.R if tokens % cfg.R == 0 else 1, cfg.H, cfg.E, cfg.k, cfg.dispatch,
-                        cfg.layout, cfg.expert, cfg.zipf)
+                        cfg.layout, cfg.expert, cfg.zipf, cfg.n_shared)
     T = sub.T
     logits = wl["logits_np"][:T]
     xb = wl["x_bits"][:T]
+    E_lay = cfg.E_phys if cfg.n_shared else cfg.E
     t0 = time.perf_counter()
-    idx, w = oracle.route(logits, cfg.k)
-    lay = oracle.layout(idx, cfg.E, sub.R)
+    if cfg.n_shared:
+        idx, w, _ = oracle.route_ex(logits, cfg.k, cfg.n_shared, 1.0, *wl["placement"],
+                                    cfg.E_phys, max(1, T // sub.R))
+    else:
+        idx, w = oracle.route(logits, cfg.k)
+    lay = oracle.layout(idx, E_lay, sub.R)
     cap = 0
     if cfg.layout == "padded":
         cap = int(lay["expert_counts"].max())
-        lay = oracle.layout(idx, cfg.E, sub.R, cap)
+        lay = oracle.layout(idx, E_lay, sub.R, cap)
     rows = lay["recv_src"].shape[0]
     pos = lay["dispatch_pos"]
     if cfg.dispatch == "fp8":
@@ -243,9 +249,10 @@ def oracle_step_on_sample(cfg: inputs.Config, wl: dict, tokens: int) -> tuple[fl
 def cpu_inputs(cfg: inputs.Config) -> dict:
     logits = inputs.make_logits(cfg)
     x = inputs.make_x(cfg)
-    bank = inputs.make_row_bank(cfg.H, seed=cfg.seed * 10 + 2, n=min(cfg.T * cfg.k, 32768))
+    bank = inputs.make_row_bank(cfg.H, seed=cfg.seed * 10 + 2, n=min(cfg.T * cfg.k_total, 32768))
     return dict(logits_np=logits.numpy(), x_bits=inputs.bf16_bits(x),
-                y_bank_bits=inputs.bf16_bits(bank))
+                y_bank_bits=inputs.bf16_bits(bank),
+                placement=inputs.expert_placement(cfg) if cfg.n_shared else None)
 
 
 def cpu_baseline(cfg: inputs.Config, budget_s: float = 12.0) -> dict:
@@ -311,7 +318,9 @@ def run_ours(args) -> None:
     import combine_moe_route_08_b200 as moe
 
     cfg = inputs.CONFIGS[args.config]
-    T, H, E, k, R = cfg.T, cfg.H, cfg.E, cfg.k, cfg.R
+    T, H, E, R = cfg.T, cfg.H, cfg.E, cfg.R
+    k = cfg.k_total                         # slots per token (routed + shared)
+    E_lay = cfg.E_phys if cfg.n_shared else E   # experts the layout sees
     logits_h = inputs.make_logits(cfg)
     x_h = inputs.make_x(cfg)
     logits = logits_h.to(dev)
@@ -319,15 +328,23 @@ def run_ours(args) -> None:
     s = torch.cuda.Stream(dev)
     ws = moe.Workspace(dev)
 
+    if cfg.n_shared:
+        offs_h, ids_h = inputs.expert_placement(cfg)
+        replica_offsets = torch.from_numpy(offs_h).to(dev)
+        replica_ids = torch.from_numpy(ids_h).to(dev)
     with torch.cuda.stream(s):
-        idx, w = moe.moe_route_topk(logits, k)
+        if cfg.n_shared:
+            idx, w = moe.moe_route_topk_ex(logits, cfg.k, cfg.n_shared, 1.0, replica_offsets,
+                                           replica_ids, cfg.E_phys, cfg.T_r)
+        else:
+            idx, w = moe.moe_route_topk(logits, k)
         cap = 0
         if cfg.layout == "padded":  # capacity = max observed count, read once, untimed
-            probe = moe.moe_dispatch_layout(idx, E, R, workspace=ws)
+            probe = moe.moe_dispatch_layout(idx, E_lay, R, workspace=ws)
             cap = int(probe["expert_counts"].max().item())
             del probe
-        rows = T * k if cap == 0 else E * cap
-        lay = moe.moe_dispatch_layout(idx, E, R, capacity=cap, rows=rows, workspace=ws)
+        rows = T * k if cap == 0 else E_lay * cap
+        lay = moe.moe_dispatch_layout(idx, E_lay, R, capacity=cap, rows=rows, workspace=ws)
         if cfg.dispatch == "fp8":
             recv_q, recv_scale = moe.moe_dispatch_fp8(x, lay["dispatch_pos"], rows)
             y = experts.dequantise(recv_q, recv_scale)
@@ -342,11 +359,18 @@ def run_ours(args) -> None:
 
     # the four C ABI calls of a step with their arguments marshalled once
     lib, sp = moe.lib, s.cuda_stream
-    ws_buf = ws.get(moe.moe_layout_workspace_bytes(T, k, E, R))
+    ws_buf = ws.get(moe.moe_layout_workspace_bytes(T, k, E_lay, R))
     pos = lay["dispatch_pos"]
+    route_call = (
+        (lib.moe_route_topk_ex, (logits.data_ptr(), T, E, cfg.k, 0, cfg.n_shared, 1.0,
+                                 replica_offsets.data_ptr(), replica_ids.data_ptr(),
+                                 replica_ids.numel(), cfg.E_phys, cfg.T_r, idx.data_ptr(),
+                                 w.data_ptr(), None, sp))
+        if cfg.n_shared else
+        (lib.moe_route_topk, (logits.data_ptr(), T, E, k, 0, idx.data_ptr(), w.data_ptr(), sp)))
     calls = [
-        (lib.moe_route_topk, (logits.data_ptr(), T, E, k, 0, idx.data_ptr(), w.data_ptr(), sp)),
-        (lib.moe_dispatch_layout, (idx.data_ptr(), T, k, E, R, cap, rows,
+        route_call,
+        (lib.moe_dispatch_layout, (idx.data_ptr(), T, k, E_lay, R, cap, rows,
                                    lay["expert_counts"].data_ptr(), lay["expert_src_counts"].data_ptr(),
                                    lay["rank_counts"].data_ptr(), lay["expert_offsets"].data_ptr(),
                                    pos.data_ptr(), lay["recv_src"].data_ptr(), ws_buf.data_ptr(),

@@ -17,7 +17,8 @@ import os
 import torch
 
 __all__ = [
-    "MoeError", "lib", "moe_status_string", "moe_route_topk", "moe_layout_workspace_bytes",
+    "MoeError", "lib", "moe_status_string", "moe_route_topk", "moe_route_topk_ex",
+    "moe_layout_workspace_bytes",
     "moe_dispatch_layout", "moe_dispatch_bf16", "moe_dispatch_fp8", "moe_combine_bf16",
     "moe_quantize_e4m3", "moe_dispatch_layout_noalloc", "Workspace", "LIB_PATH",
 ]
@@ -38,6 +39,9 @@ lib.moe_status_string.argtypes = [_i32]
 lib.moe_status_string.restype = ctypes.c_char_p
 lib.moe_route_topk.argtypes = [_P, _i32, _i32, _i32, _i32, _P, _P, _P]
 lib.moe_route_topk.restype = _i32
+lib.moe_route_topk_ex.argtypes = [_P, _i32, _i32, _i32, _i32, _i32, ctypes.c_float, _P, _P, _i32,
+                                  _i32, _i32, _P, _P, _P, _P]
+lib.moe_route_topk_ex.restype = _i32
 lib.moe_layout_workspace_bytes.argtypes = [_i32, _i32, _i32, _i32]
 lib.moe_layout_workspace_bytes.restype = _sz
 lib.moe_dispatch_layout.argtypes = [_P, _i32, _i32, _i32, _i32, _i32, _i64, _P, _P, _P, _P, _P, _P,
@@ -118,6 +122,34 @@ def moe_route_topk(logits: torch.Tensor, k: int, renormalize: bool = False,
         topk_w = torch.empty(T, k, dtype=torch.float32, device=dev)
     _check(lib.moe_route_topk(_ptr(logits), T, E, k, int(renormalize), _ptr(topk_idx),
                               _ptr(topk_w), _stream(stream)), "moe_route_topk")
+    return topk_idx, topk_w
+
+
+def moe_route_topk_ex(logits: torch.Tensor, k: int, n_shared: int = 0, shared_weight: float = 1.0,
+                      replica_offsets: torch.Tensor | None = None,
+                      replica_ids: torch.Tensor | None = None, E_phys: int | None = None,
+                      tokens_per_rank: int = 1, renormalize: bool = False,
+                      topk_idx: torch.Tensor | None = None, topk_w: torch.Tensor | None = None,
+                      dev_status: torch.Tensor | None = None, stream=None):
+    """Top-k over the routed logits plus n_shared always-selected shared
+    experts, each logical expert mapped to a physical replica by the token's
+    source rank.  Returns (topk_idx int32 [T][k+n_shared] physical ids,
+    topk_w fp32 [T][k+n_shared])."""
+    assert logits.dtype == torch.float32 and logits.dim() == 2
+    T, E = logits.shape
+    kk = k + n_shared
+    dev = logits.device
+    if E_phys is None:
+        E_phys = E + n_shared
+    if topk_idx is None:
+        topk_idx = torch.empty(T, kk, dtype=torch.int32, device=dev)
+    if topk_w is None:
+        topk_w = torch.empty(T, kk, dtype=torch.float32, device=dev)
+    n_ids = 0 if replica_ids is None else replica_ids.numel()
+    _check(lib.moe_route_topk_ex(_ptr(logits), T, E, k, int(renormalize), n_shared,
+                                 float(shared_weight), _ptr(replica_offsets), _ptr(replica_ids),
+                                 n_ids, E_phys, tokens_per_rank, _ptr(topk_idx), _ptr(topk_w),
+                                 _ptr(dev_status), _stream(stream)), "moe_route_topk_ex")
     return topk_idx, topk_w
 
 

@@ -60,7 +60,33 @@ int moe_route_topk(const float *logits, int T, int E, int k, int renormalize, in
     if (!logits || !topk_idx || !topk_w || !aligned(logits, 4) || !aligned(topk_idx, 4) ||
         !aligned(topk_w, 4))
         return MOE_ERR_INVALID_ARG;
-    return launched(moe::route_topk(logits, T, E, k, renormalize != 0, topk_idx, topk_w,
+    return launched(moe::route_topk(logits, T, E, k, renormalize != 0, topk_idx, topk_w, nullptr,
+                                    as_stream(stream)));
+}
+
+int moe_route_topk_ex(const float *logits, int T, int E, int k, int renormalize, int n_shared,
+                      float shared_weight, const int32_t *replica_offsets,
+                      const int32_t *replica_ids, int n_replica_ids, int E_phys,
+                      int tokens_per_rank, int32_t *topk_idx, float *topk_w, int32_t *dev_status,
+                      void *stream)
+{
+    if (n_shared < 0 || n_shared > kMaxK || !valid_tk(T, k + n_shared) || k < 1 || E < 1 ||
+        E > kMaxE || k > E || E_phys < 1 || tokens_per_rank < 1)
+        return MOE_ERR_INVALID_ARG;
+    if (replica_offsets != nullptr &&
+        (replica_ids == nullptr || n_replica_ids < 1 || !aligned(replica_offsets, 4) ||
+         !aligned(replica_ids, 4)))
+        return MOE_ERR_INVALID_ARG;
+    if (replica_offsets == nullptr && E_phys < E + n_shared)
+        return MOE_ERR_INVALID_ARG;
+    if (T == 0)
+        return MOE_OK;
+    if (!logits || !topk_idx || !topk_w || !aligned(logits, 4) || !aligned(topk_idx, 4) ||
+        !aligned(topk_w, 4) || (dev_status && !aligned(dev_status, 4)))
+        return MOE_ERR_INVALID_ARG;
+    const moe::RouteEx ex{n_shared, shared_weight, replica_offsets, replica_ids, n_replica_ids,
+                          E_phys, tokens_per_rank, dev_status};
+    return launched(moe::route_topk(logits, T, E, k, renormalize != 0, topk_idx, topk_w, &ex,
                                     as_stream(stream)));
 }
 

@@ -22,8 +22,22 @@ struct LayoutGeom {
 LayoutGeom layout_geom(int T, int k, int E, int R);
 size_t layout_workspace_bytes(const LayoutGeom &g);
 
+// Extension of the route: shared experts and expert replicas.
+struct RouteEx {
+    int n_shared;
+    float shared_weight;
+    const int32_t *replica_offsets;  // [E + n_shared + 1] or nullptr
+    const int32_t *replica_ids;      // [n_replica_ids]
+    int n_replica_ids;
+    int E_phys;
+    int tokens_per_rank;
+    int32_t *dev_status;
+};
+
+// ex == nullptr: the plain route (outputs [T][k]); otherwise outputs are
+// [T][k + ex->n_shared] physical expert ids.
 cudaError_t route_topk(const float *logits, int T, int E, int k, int renormalize,
-                       int32_t *topk_idx, float *topk_w, cudaStream_t s);
+                       int32_t *topk_idx, float *topk_w, const RouteEx *ex, cudaStream_t s);
 
 cudaError_t dispatch_layout(const int32_t *topk_idx, const LayoutGeom &g, int capacity,
                             int64_t rows, int32_t *expert_counts, int32_t *expert_src_counts,

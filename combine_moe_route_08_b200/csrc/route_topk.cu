@@ -12,6 +12,12 @@
 // the indices holding it (redux.sync, a single instruction each), then the
 // winner's key is cleared.
 //
+// The extended form (shared experts, expert replicas; DeepSeek-V3 fragments:
+// during decoding the shared expert is treated as a routed one that every
+// token selects, and redundant experts replicate heavily loaded ones)
+// appends the shared slots after the k routed ones and maps each logical
+// expert through the caller's replica table in the same epilogue.
+//
 // The softmax is evaluated in fp32 with its error bounded (u = 2^-24):
 //   d = l - m is split exactly into d_hi + d_lo (Knuth's TwoSum), so the
 //   exponent sees no rounding of the difference; t = expf(d_hi) * (1 + d_lo)
@@ -63,10 +69,10 @@ __device__ __forceinline__ float exp_diff(float l, float m)
     return __fmaf_rn(t, lo, t);
 }
 
-template <int NPL>
+template <int NPL, bool EX>
 __global__ void __launch_bounds__(kRouteWarps * 32)
     k_route_topk(const float *__restrict__ logits, int T, int E, int k, int renormalize,
-                 int32_t *__restrict__ topk_idx, float *__restrict__ topk_w)
+                 int32_t *__restrict__ topk_idx, float *__restrict__ topk_w, RouteEx ex)
 {
     const int lane = threadIdx.x & 31;
     const int g = blockIdx.x * kRouteWarps + (threadIdx.x >> 5);
@@ -164,36 +170,63 @@ __global__ void __launch_bounds__(kRouteWarps * 32)
         }
         denom = __fadd_rn(ks, kc);
     }
-    if (lane < k) {
-        topk_idx[static_cast<size_t>(g) * k + lane] = my_e;
-        topk_w[static_cast<size_t>(g) * k + lane] = __fdiv_rn(num, denom);
+    if (!EX) {
+        if (lane < k) {
+            topk_idx[static_cast<size_t>(g) * k + lane] = my_e;
+            topk_w[static_cast<size_t>(g) * k + lane] = __fdiv_rn(num, denom);
+        }
+    } else {
+        // shared experts E .. E + n_shared - 1 follow the routed ones; every
+        // logical expert maps to the replica chosen by the token's source rank
+        const int kk = k + ex.n_shared;
+        if (lane < kk) {
+            const int l = (lane < k) ? my_e : E + (lane - k);
+            const float wt = (lane < k) ? __fdiv_rn(num, denom) : ex.shared_weight;
+            int phys = l;
+            if (ex.replica_offsets != nullptr) {
+                const int a = ex.replica_offsets[l], b = ex.replica_offsets[l + 1];
+                if (a < 0 || b <= a || b > ex.n_replica_ids)
+                    phys = -1;
+                else
+                    phys = ex.replica_ids[a + (g / ex.tokens_per_rank) % (b - a)];
+            }
+            if (phys < 0 || phys >= ex.E_phys) {
+                report(ex.dev_status, MOE_ERR_INVALID_ARG);
+                phys = -1;
+            }
+            topk_idx[static_cast<size_t>(g) * kk + lane] = phys;
+            topk_w[static_cast<size_t>(g) * kk + lane] = wt;
+        }
     }
     pdl_trigger();
 }
 
 template <int NPL>
 cudaError_t launch(const float *logits, int T, int E, int k, int renormalize, int32_t *idx,
-                   float *w, cudaStream_t s)
+                   float *w, const RouteEx *ex, cudaStream_t s)
 {
     const int grid = ceil_div(T, kRouteWarps);
-    return launch_pdl(k_route_topk<NPL>, dim3(grid), dim3(kRouteWarps * 32), 0, s, logits, T, E, k,
-                      renormalize, idx, w);
+    if (ex == nullptr)
+        return launch_pdl(k_route_topk<NPL, false>, dim3(grid), dim3(kRouteWarps * 32), 0, s,
+                          logits, T, E, k, renormalize, idx, w, RouteEx{});
+    return launch_pdl(k_route_topk<NPL, true>, dim3(grid), dim3(kRouteWarps * 32), 0, s, logits,
+                      T, E, k, renormalize, idx, w, *ex);
 }
 
 }  // namespace
 
 cudaError_t route_topk(const float *logits, int T, int E, int k, int renormalize,
-                       int32_t *topk_idx, float *topk_w, cudaStream_t s)
+                       int32_t *topk_idx, float *topk_w, const RouteEx *ex, cudaStream_t s)
 {
     const int need = ceil_div(E, 32);
-    if (need <= 1) return launch<1>(logits, T, E, k, renormalize, topk_idx, topk_w, s);
-    if (need <= 2) return launch<2>(logits, T, E, k, renormalize, topk_idx, topk_w, s);
-    if (need <= 4) return launch<4>(logits, T, E, k, renormalize, topk_idx, topk_w, s);
-    if (need <= 8) return launch<8>(logits, T, E, k, renormalize, topk_idx, topk_w, s);
-    if (need <= 12) return launch<12>(logits, T, E, k, renormalize, topk_idx, topk_w, s);
-    if (need <= 16) return launch<16>(logits, T, E, k, renormalize, topk_idx, topk_w, s);
-    if (need <= 24) return launch<24>(logits, T, E, k, renormalize, topk_idx, topk_w, s);
-    return launch<32>(logits, T, E, k, renormalize, topk_idx, topk_w, s);
+    if (need <= 1) return launch<1>(logits, T, E, k, renormalize, topk_idx, topk_w, ex, s);
+    if (need <= 2) return launch<2>(logits, T, E, k, renormalize, topk_idx, topk_w, ex, s);
+    if (need <= 4) return launch<4>(logits, T, E, k, renormalize, topk_idx, topk_w, ex, s);
+    if (need <= 8) return launch<8>(logits, T, E, k, renormalize, topk_idx, topk_w, ex, s);
+    if (need <= 12) return launch<12>(logits, T, E, k, renormalize, topk_idx, topk_w, ex, s);
+    if (need <= 16) return launch<16>(logits, T, E, k, renormalize, topk_idx, topk_w, ex, s);
+    if (need <= 24) return launch<24>(logits, T, E, k, renormalize, topk_idx, topk_w, ex, s);
+    return launch<32>(logits, T, E, k, renormalize, topk_idx, topk_w, ex, s);
 }
 
 }  // namespace moe

@@ -49,6 +49,7 @@ class Config:
     layout: str         # "packed" or "padded"
     expert: str         # stand-in expert: "identity", "affine", "dequant"
     zipf: float = 0.0   # Zipf exponent of the per-expert logit bias (0: none)
+    n_shared: int = 0   # shared experts every token selects (one replica per rank)
 
     @property
     def T(self) -> int:
@@ -62,9 +63,22 @@ class Config:
     def seed(self) -> int:
         return 1000 + self.index
 
+    @property
+    def k_total(self) -> int:
+        """Experts each token selects: the k routed ones and the shared ones."""
+        return self.k + self.n_shared
+
+    @property
+    def E_phys(self) -> int:
+        """Physical experts: each rank hosts its E/R routed experts and one
+        replica of every shared expert."""
+        return self.E + self.n_shared * self.R
+
     def describe(self) -> str:
+        shared = (f" + {self.n_shared} shared (replicated per rank, {self.E_phys} physical experts)"
+                  if self.n_shared else "")
         return (f"{self.name}: T={self.T} ({self.T_r}x{self.R} ranks), H={self.H}, "
-                f"E={self.E}, k={self.k}, {self.dispatch} dispatch, {self.layout} layout")
+                f"E={self.E}, k={self.k}{shared}, {self.dispatch} dispatch, {self.layout} layout")
 
 
 CONFIGS = {
@@ -75,8 +89,30 @@ CONFIGS = {
         Config("dsv3", 2, 128, 32, 7168, 256, 8, "fp8", "packed", "dequant"),
         Config("kimi", 3, 128, 48, 7168, 384, 8, "fp8", "packed", "dequant", zipf=1.2),
         Config("prefill", 4, 4096, 8, 7168, 256, 8, "fp8", "padded", "dequant"),
+        # beyond the five: DeepSeek-V3-like decode where the shared expert is
+        # routed too (9 experts per token, 8 routed + 1 shared per rank)
+        Config("dsv3_shared", 5, 128, 32, 7168, 256, 8, "fp8", "packed", "dequant", n_shared=1),
     ]
 }
+
+
+def expert_placement(cfg: Config):
+    """Replica table of a config with shared experts: rank r hosts physical
+    experts [r*(L+S), (r+1)*(L+S)): its L = E/R routed experts, then one
+    replica of each of the S shared experts.  Returns (replica_offsets
+    [E+S+1], replica_ids) as int32 numpy arrays; routed expert e has one
+    replica, shared expert s has R (token of rank r uses the one on rank r)."""
+    import numpy as np
+    L, S, R = cfg.E // cfg.R, cfg.n_shared, cfg.R
+    per = L + S
+    ids, offs = [], [0]
+    for e in range(cfg.E):
+        ids.append((e // L) * per + e % L)
+        offs.append(len(ids))
+    for s_ in range(S):
+        ids += [r * per + L + s_ for r in range(R)]
+        offs.append(len(ids))
+    return np.array(offs, np.int32), np.array(ids, np.int32)
 
 
 def generator(seed: int, stream: int) -> torch.Generator:

@@ -94,6 +94,37 @@ int moe_route_topk(const float *logits, int T, int E, int k, int renormalize,
                    int32_t *topk_idx, float *topk_w, void *stream);
 
 /*
+ * moe_route_topk_ex -- moe_route_topk with shared experts and expert replicas.
+ * Follows the DeepSeek-V3 report fragments quoted on the third and fourth
+ * pages: during decoding the shared expert is treated as a routed one that
+ * every token always selects (so each token selects 9 experts), and each GPU
+ * also hosts redundant replicas of heavily loaded experts.
+ *
+ *   Routed part: exactly moe_route_topk over the E routed logits (k experts,
+ *   weights as there, renormalize over the k routed ones).  Shared part: the
+ *   n_shared logical experts E .. E + n_shared - 1 follow in slot order, each
+ *   with weight shared_weight.  Every chosen logical expert l is mapped to a
+ *   physical expert:
+ *     replica_offsets == NULL: physical id = l (needs E_phys >= E + n_shared);
+ *     otherwise l is served by replica_ids[replica_offsets[l] ..
+ *     replica_offsets[l + 1]) and the token g of source rank
+ *     r = g / tokens_per_rank uses replica r mod (number of replicas of l).
+ *   replica_offsets  [E + n_shared + 1] int32 (device), non-decreasing.
+ *   replica_ids      [n_replica_ids] int32 (device) physical ids in [0, E_phys).
+ *   topk_idx         [T][k + n_shared] int32 out: physical expert ids.
+ *   topk_w           [T][k + n_shared] fp32 out.
+ * A slot whose table entry is empty, out of [0, n_replica_ids) or gives an id
+ * outside [0, E_phys) gets -1 and MOE_ERR_INVALID_ARG through dev_status.
+ * Limits: 0 <= n_shared, 1 <= k, k + n_shared <= 32, tokens_per_rank >= 1.
+ * The output feeds moe_dispatch_layout with E_phys experts.
+ */
+int moe_route_topk_ex(const float *logits, int T, int E, int k, int renormalize, int n_shared,
+                      float shared_weight, const int32_t *replica_offsets,
+                      const int32_t *replica_ids, int n_replica_ids, int E_phys,
+                      int tokens_per_rank, int32_t *topk_idx, float *topk_w, int32_t *dev_status,
+                      void *stream);
+
+/*
  * Bytes of device workspace moe_dispatch_layout needs for (T, k, E, R);
  * 0 on invalid sizes.  The workspace must be 256-byte aligned; its contents
  * need no initialisation and are scratch (per-chunk histograms).  One

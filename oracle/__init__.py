@@ -50,6 +50,8 @@ def _load():
         i32, i64, u32 = ctypes.c_int, ctypes.c_int64, ctypes.c_uint32
         lib.oracle_route.argtypes = [P, i32, i32, i32, i32, P, P]
         lib.oracle_route.restype = i32
+        lib.oracle_route_ex.argtypes = [P, i32, i32, i32, i32, i32, ctypes.c_float, P, P, i32, i32, P, P]
+        lib.oracle_route_ex.restype = i32
         lib.oracle_layout.argtypes = [P, i32, i32, i32, i32, i32, i64, P, P, P, P, P, P]
         lib.oracle_layout.restype = i32
         lib.oracle_dispatch_bf16.argtypes = [P, i32, i32, i32, P, P, i64]
@@ -101,6 +103,28 @@ def route(logits: np.ndarray, k: int, renormalize: bool = False):
     if st != OK:
         raise ValueError(f"oracle_route status {st}")
     return idx, w
+
+
+def route_ex(logits: np.ndarray, k: int, n_shared: int = 0, shared_weight: float = 1.0,
+             replica_offsets=None, replica_ids=None, E_phys: int | None = None,
+             T_r: int = 1, renormalize: bool = False):
+    """Top-k over the routed logits, then n_shared always-selected shared
+    experts, every logical expert mapped to a physical replica chosen by the
+    token's source rank.  Returns (topk_idx [T][k+n_shared] physical ids,
+    topk_w [T][k+n_shared], status)."""
+    logits = _c(logits, np.float32)
+    T, E = logits.shape
+    kk = k + n_shared
+    if E_phys is None:
+        E_phys = E + n_shared
+    ro = None if replica_offsets is None else _c(replica_offsets, np.int32)
+    ri = None if replica_ids is None else _c(replica_ids, np.int32)
+    idx = np.empty((T, kk), np.int32)
+    w = np.empty((T, kk), np.float32)
+    st = _load().oracle_route_ex(_ptr(logits), T, E, k, int(renormalize), n_shared,
+                                 float(shared_weight), _ptr(ro), _ptr(ri), E_phys, T_r,
+                                 _ptr(idx), _ptr(w))
+    return idx, w, st
 
 
 # --------------------------------------------------------------------------

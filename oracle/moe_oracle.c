@@ -252,6 +252,69 @@ int oracle_route(const float *logits, int T, int E, int k, int renormalize,
     return ORACLE_OK;
 }
 
+/* Route with shared experts and expert replicas [DSV3: during decoding the
+ * shared expert is treated as a routed one that every token selects, so a
+ * token selects 9 experts; redundant experts replicate heavily loaded ones].
+ *
+ * Routed part: exactly oracle_route over the E routed logits (top-k and
+ * softmax weights, optionally renormalised over the chosen k).  Shared part:
+ * the n_shared logical experts E .. E + n_shared - 1 follow in slot order,
+ * each with weight shared_weight.  Every chosen logical expert l is then
+ * mapped to one of its physical replicas
+ *     replica_ids[replica_offsets[l] + (g / T_r) % n_rep(l)],
+ *     n_rep(l) = replica_offsets[l + 1] - replica_offsets[l],
+ * i.e. tokens of source rank r use replica r mod n_rep.  With no table
+ * (replica_offsets == NULL) the physical id is the logical one.  A replica
+ * id outside [0, E_phys) or an expert without replicas gives slot -1 and
+ * ORACLE_ERR_INVALID.  Outputs are [T][k + n_shared]. */
+int oracle_route_ex(const float *logits, int T, int E, int k, int renormalize,
+                    int n_shared, float shared_weight,
+                    const int32_t *replica_offsets, const int32_t *replica_ids,
+                    int E_phys, int T_r, int32_t *topk_idx, float *topk_w)
+{
+    if (n_shared < 0 || T_r < 1)
+        return ORACLE_ERR_INVALID;
+    const int kk = k + n_shared;
+    int32_t *idx = (int32_t *)malloc(sizeof(int32_t) * (size_t)(T > 0 ? T : 1) * k);
+    float *w = (float *)malloc(sizeof(float) * (size_t)(T > 0 ? T : 1) * k);
+    if (!idx || !w) {
+        free(idx);
+        free(w);
+        return ORACLE_ERR_INVALID;
+    }
+    int status = oracle_route(logits, T, E, k, renormalize, idx, w);
+    if (status != ORACLE_OK) {
+        free(idx);
+        free(w);
+        return status;
+    }
+    for (int g = 0; g < T; ++g) {
+        for (int j = 0; j < kk; ++j) {
+            int32_t l = (j < k) ? idx[(size_t)g * k + j] : E + (j - k);
+            float wt = (j < k) ? w[(size_t)g * k + j] : shared_weight;
+            int32_t phys = l;
+            if (replica_offsets) {
+                int32_t a = replica_offsets[l], b = replica_offsets[l + 1];
+                if (b <= a) {
+                    phys = -1;
+                } else {
+                    int32_t r = (g / T_r) % (b - a);
+                    phys = replica_ids[a + r];
+                }
+            }
+            if (phys < 0 || phys >= E_phys) {
+                phys = -1;
+                status = ORACLE_ERR_INVALID;
+            }
+            topk_idx[(size_t)g * kk + j] = phys;
+            topk_w[(size_t)g * kk + j] = wt;
+        }
+    }
+    free(idx);
+    free(w);
+    return status;
+}
+
 /* ------------------------------------------------------------------------ */
 /* Layout: counts -> offsets -> slots [EFA "Gönderme ve Alma Arabellekleri", */
 /* "Dağıtım ve Birleştirme"; EPMC "Despacho"]                                */

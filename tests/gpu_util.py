@@ -53,16 +53,38 @@ def gpu_bits(t: torch.Tensor) -> np.ndarray:
 
 @functools.lru_cache(maxsize=5)
 def workload(name: str):
-    """Seeded inputs of a workload and the oracle's route and layout on them."""
+    """Seeded inputs of a workload and the oracle's route and layout on them.
+    Workloads with shared experts route through the extended route (physical
+    expert ids over cfg.E_phys experts, cfg.k_total slots per token)."""
     cfg = inputs.CONFIGS[name]
     logits = inputs.make_logits(cfg)
     x = inputs.make_x(cfg)
-    idx, w = oracle.route(logits.numpy(), cfg.k)
-    packed = oracle.layout(idx, cfg.E, cfg.R)
+    placement = None
+    if cfg.n_shared:
+        placement = inputs.expert_placement(cfg)
+        idx, w, st = oracle.route_ex(logits.numpy(), cfg.k, cfg.n_shared, 1.0, *placement,
+                                     cfg.E_phys, cfg.T_r)
+        assert st == oracle.OK
+    else:
+        idx, w = oracle.route(logits.numpy(), cfg.k)
+    E_lay = cfg.E_phys if cfg.n_shared else cfg.E
+    packed = oracle.layout(idx, E_lay, cfg.R)
     cap = int(packed["expert_counts"].max()) if cfg.layout == "padded" else 0
-    lay = oracle.layout(idx, cfg.E, cfg.R, cap) if cap else packed
+    lay = oracle.layout(idx, E_lay, cfg.R, cap) if cap else packed
     return dict(cfg=cfg, logits=logits, x=x, x_bits=inputs.bf16_bits(x), idx=idx, w=w,
-                layout=lay, cap=cap, rows=int(lay["recv_src"].shape[0]))
+                layout=lay, cap=cap, rows=int(lay["recv_src"].shape[0]), E_lay=E_lay,
+                k=idx.shape[1], placement=placement)
+
+
+def gpu_route(moe, wl, renormalize=False):
+    """The GPU route of a workload (the extended one when it has shared experts)."""
+    cfg = wl["cfg"]
+    logits = to_dev(wl["logits"])
+    if not cfg.n_shared:
+        return moe.moe_route_topk(logits, cfg.k, renormalize=renormalize)
+    offs, ids = wl["placement"]
+    return moe.moe_route_topk_ex(logits, cfg.k, cfg.n_shared, 1.0, to_dev(offs), to_dev(ids),
+                                 cfg.E_phys, cfg.T_r, renormalize=renormalize)
 
 
 def stand_in_y_cpu(wl, recv_bits=None, recv_q=None, recv_scale=None):

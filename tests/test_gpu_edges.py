@@ -236,3 +236,85 @@ def test_e4m3_converter_every_binary32_pattern(moe):
             for n_bad, first_bad in pool.map(_mismatch_range, jobs):
                 bad_total += n_bad
     assert bad_total == 0
+
+
+def test_layout_large_token_count_many_chunks(moe):
+    """1M slots (131072 tokens x 8) over 8 logical ranks: 16 chunks per rank,
+    128 chunks in all; packed and padded layouts bit-exact."""
+    T, E, k, R = 131072, 256, 8, 8
+    rng = np.random.default_rng(17)
+    idx = np.argsort(rng.random((T, E), dtype=np.float32), axis=1)[:, :k].astype(np.int32)
+    want = oracle.layout(idx, E, R)
+    st = _status()
+    lay = moe.moe_dispatch_layout(to_dev(idx), E, R, dev_status=st)
+    torch.cuda.synchronize()
+    for key in LAYOUT_KEYS:
+        assert np.array_equal(lay[key].cpu().numpy(), want[key].reshape(lay[key].shape)), key
+    cap = int(want["expert_counts"].max()) - 7          # a few drops in the hottest experts
+    want_p = oracle.layout(idx, E, R, cap)
+    lay_p = moe.moe_dispatch_layout(to_dev(idx), E, R, capacity=cap, rows=E * cap, dev_status=st)
+    torch.cuda.synchronize()
+    for key in LAYOUT_KEYS:
+        assert np.array_equal(lay_p[key].cpu().numpy(), want_p[key].reshape(lay_p[key].shape)), key
+    assert st.item() == moe.MOE_ERR_CAPACITY
+
+
+def test_all_slots_masked(moe):
+    """Every slot empty (-1): nothing counted, nothing dispatched, combine
+    writes zeros."""
+    T, E, k, R, H = 64, 8, 2, 2, 256
+    idx = np.full((T, k), -1, np.int32)
+    st = _status()
+    lay = moe.moe_dispatch_layout(to_dev(idx), E, R, dev_status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    assert lay["expert_counts"].sum().item() == 0
+    assert torch.all(lay["dispatch_pos"] == -1) and torch.all(lay["recv_src"] == -1)
+    x = inputs.make_random_rows(T, H, seed=3)
+    recv = torch.full((T * k, H), 5.0, dtype=torch.bfloat16, device="cuda")
+    moe.moe_dispatch_bf16(to_dev(x), lay["dispatch_pos"], T * k, recv_x=recv)
+    out = moe.moe_combine_bf16(recv, lay["dispatch_pos"], torch.ones(T, k, device="cuda"))
+    torch.cuda.synchronize()
+    assert torch.all(recv == 5.0)
+    assert torch.all(out == 0)
+
+
+def test_route_ex_replicas_and_bad_table(moe):
+    """Extended route against the oracle: an expert with three replicas
+    chosen by source rank, two shared experts, renormalised routed weights,
+    then a table entry out of range (slot -1, reported)."""
+    T, E, k, Tr = 96, 16, 3, 8
+    logits, _ = inputs.make_random_case(T, 8, E, k, seed=41)
+    n_shared = 2
+    # logical 0..15 routed, 16..17 shared; physical ids 0..21
+    offs = [0]
+    ids = []
+    for l in range(E + n_shared):
+        reps = [l] if l != 5 else [5, 18, 19]
+        if l >= E:
+            reps = [l, l + 4]                      # shared: 16 -> {16, 20}, 17 -> {17, 21}
+        ids += reps
+        offs.append(len(ids))
+    offs = np.array(offs, np.int32)
+    ids = np.array(ids, np.int32)
+    for renorm in (False, True):
+        want_i, want_w, st_o = oracle.route_ex(logits.numpy(), k, n_shared, 0.75, offs, ids, 22, Tr,
+                                               renormalize=renorm)
+        assert st_o == oracle.OK
+        st = _status()
+        got_i, got_w = moe.moe_route_topk_ex(to_dev(logits), k, n_shared, 0.75, to_dev(offs),
+                                             to_dev(ids), 22, Tr, renormalize=renorm, dev_status=st)
+        torch.cuda.synchronize()
+        assert np.array_equal(got_i.cpu().numpy(), want_i)
+        gw = got_w.cpu().numpy().astype(np.float64)
+        assert np.all(np.abs(gw - want_w) <= route_w_tol(want_w))
+        assert st.item() == 0
+    bad = ids.copy()
+    bad[offs[7]] = 22                               # expert 7's replica: one past E_phys
+    want_i, _, st_o = oracle.route_ex(logits.numpy(), k, n_shared, 0.75, offs, bad, 22, Tr)
+    st = _status()
+    got_i, _ = moe.moe_route_topk_ex(to_dev(logits), k, n_shared, 0.75, to_dev(offs), to_dev(bad),
+                                     22, Tr, dev_status=st)
+    torch.cuda.synchronize()
+    assert st_o == oracle.ERR_INVALID and st.item() == moe.MOE_ERR_INVALID_ARG
+    assert np.array_equal(got_i.cpu().numpy(), want_i)

@@ -11,12 +11,12 @@ import torch
 
 import oracle
 from harness import experts, inputs
-from gpu_util import (bf16_to_f64, check_combine, gpu_bits, stand_in_y_cpu, to_dev, ulp_bf16,
-                      route_w_tol, ulp_f32, workload)
+from gpu_util import (bf16_to_f64, check_combine, gpu_bits, gpu_route, stand_in_y_cpu, to_dev,
+                      ulp_bf16, route_w_tol, ulp_f32, workload)
 
 pytestmark = pytest.mark.gpu
 
-ALL = ["tiny", "mixtral", "dsv3", "kimi", "prefill"]
+ALL = ["tiny", "mixtral", "dsv3", "kimi", "prefill", "dsv3_shared"]
 LAYOUT_KEYS = ["expert_counts", "expert_src_counts", "rank_counts", "expert_offsets",
                "dispatch_pos", "recv_src"]
 
@@ -39,9 +39,14 @@ def _status():
 def test_route_parity(moe, name, renormalize):
     wl = workload(name)
     cfg = wl["cfg"]
-    idx_o, w_o = (wl["idx"], wl["w"]) if not renormalize else oracle.route(
-        wl["logits"].numpy(), cfg.k, renormalize=True)
-    idx, w = moe.moe_route_topk(to_dev(wl["logits"]), cfg.k, renormalize=renormalize)
+    if not renormalize:
+        idx_o, w_o = wl["idx"], wl["w"]
+    elif cfg.n_shared:
+        idx_o, w_o, _ = oracle.route_ex(wl["logits"].numpy(), cfg.k, cfg.n_shared, 1.0,
+                                        *wl["placement"], cfg.E_phys, cfg.T_r, renormalize=True)
+    else:
+        idx_o, w_o = oracle.route(wl["logits"].numpy(), cfg.k, renormalize=True)
+    idx, w = gpu_route(moe, wl, renormalize)
     torch.cuda.synchronize()
     assert np.array_equal(idx.cpu().numpy(), idx_o)
     w = w.cpu().numpy()
@@ -68,7 +73,7 @@ def test_layout_parity(moe, name):
     wl = workload(name)
     cfg = wl["cfg"]
     st = _status()
-    got = _gpu_layout(moe, wl["idx"], cfg.E, cfg.R, wl["cap"], wl["rows"], st)
+    got = _gpu_layout(moe, wl["idx"], wl["E_lay"], cfg.R, wl["cap"], wl["rows"], st)
     _assert_layout_equal(got, wl["layout"], name)
     assert st.item() == 0
 
@@ -143,7 +148,7 @@ def _gpu_fp8(moe, wl, guard=3):
     return qbuf[guard:guard + rows], sbuf[guard:guard + rows]
 
 
-@pytest.mark.parametrize("name", ["dsv3", "kimi"])
+@pytest.mark.parametrize("name", ["dsv3", "kimi", "dsv3_shared"])
 def test_dispatch_fp8_parity_full(moe, name):
     wl = workload(name)
     q, s = _gpu_fp8(moe, wl)
@@ -177,7 +182,7 @@ def test_dispatch_fp8_parity_prefill_sampled(moe):
 
 # ---------------------------------------------------------------- combine
 
-@pytest.mark.parametrize("name", ["tiny", "mixtral", "dsv3", "kimi"])
+@pytest.mark.parametrize("name", ["tiny", "mixtral", "dsv3", "kimi", "dsv3_shared"])
 def test_combine_parity_full(moe, name):
     """y = the workload's stand-in expert applied (on the CPU) to the oracle's
     dispatch output; the same y and the oracle's weights go to both sides."""
@@ -232,8 +237,8 @@ def test_whole_path_on_gpu_vs_oracle(moe, name):
     wl = workload(name)
     cfg = wl["cfg"]
     x = to_dev(wl["x"])
-    idx, w = moe.moe_route_topk(to_dev(wl["logits"]), cfg.k)
-    lay = moe.moe_dispatch_layout(idx, cfg.E, cfg.R, capacity=wl["cap"], rows=wl["rows"])
+    idx, w = gpu_route(moe, wl)
+    lay = moe.moe_dispatch_layout(idx, wl["E_lay"], cfg.R, capacity=wl["cap"], rows=wl["rows"])
     pos_o = wl["layout"]["dispatch_pos"]
     if cfg.dispatch == "bf16":
         recv = moe.moe_dispatch_bf16(x, lay["dispatch_pos"], wl["rows"])
@@ -258,10 +263,11 @@ def test_whole_path_on_gpu_vs_oracle(moe, name):
     else:
         qt, st_ = oracle.quantize_tokens(wl["x_bits"], tokens)
         y_tok = stand_in_y_cpu(wl, recv_q=qt, recv_scale=st_)          # [n][H]
-        y_small = np.repeat(y_tok, cfg.k, 0)                             # row = i*k + j
-        pos_small = np.arange(len(tokens) * cfg.k, dtype=np.int32).reshape(len(tokens), cfg.k)
+        kk = wl["k"]
+        y_small = np.repeat(y_tok, kk, 0)                                # row = i*k + j
+        pos_small = np.arange(len(tokens) * kk, dtype=np.int32).reshape(len(tokens), kk)
         acc, _ = oracle.combine(y_small, pos_small, wl["w"][tokens])
-        yf = bf16_to_f64(y_small).reshape(len(tokens), cfg.k, cfg.H)
+        yf = bf16_to_f64(y_small).reshape(len(tokens), kk, cfg.H)
         terms = np.abs(wl["w"][tokens].astype(np.float64))[:, :, None] * np.abs(yf)
     got = bf16_to_f64(gpu_bits(out)[tokens])
     tol = ulp_bf16(acc) + 2.0 ** -19 * terms.sum(1)

@@ -79,3 +79,62 @@ def test_route_zipf_bias_makes_expert0_hottest():
     b = inputs.zipf_bias(cfg.E, cfg.zipf).double()
     assert abs(torch.logsumexp(b, 0).item()) < 1e-6
     assert torch.all(b[1:] < b[:-1])
+
+
+# ------------------------------------------------ shared experts and replicas
+
+def test_route_ex_hand_case(oracle_mod):
+    fx = load_golden("route_ex_hand.json")
+    logits = np.array(fx["logits"], np.float32)
+    idx, w, st = oracle_mod.route_ex(logits, fx["k"], fx["n_shared"], fx["shared_weight"],
+                                     fx["replica_offsets"], fx["replica_ids"], fx["E_phys"],
+                                     fx["T_r"])
+    assert st == oracle_mod.OK
+    assert idx.tolist() == fx["topk_idx"]
+    assert w[:, fx["k"]:].ravel().tolist() == fx["shared_w"]
+    # the routed weights are those of the plain route
+    _, w_plain = oracle_mod.route(logits, fx["k"])
+    assert np.array_equal(w[:, :fx["k"]], w_plain)
+
+
+def test_route_ex_workload_invariants(oracle_mod):
+    cfg = inputs.CONFIGS["dsv3_shared"]
+    logits = inputs.make_logits(cfg).numpy()
+    offs, ids = inputs.expert_placement(cfg)
+    idx, w, st = oracle_mod.route_ex(logits, cfg.k, cfg.n_shared, 1.0, offs, ids, cfg.E_phys,
+                                     cfg.T_r)
+    assert st == oracle_mod.OK and idx.shape == (cfg.T, cfg.k_total)
+    plain_idx, plain_w = oracle_mod.route(logits, cfg.k)
+    L, per = cfg.E // cfg.R, cfg.E // cfg.R + cfg.n_shared
+    # routed slots: the plain top-k mapped to their physical ids, same weights
+    assert np.array_equal(idx[:, :cfg.k], (plain_idx // L) * per + plain_idx % L)
+    assert np.array_equal(w[:, :cfg.k], plain_w)
+    # shared slot: weight 1, the replica on the token's own logical rank
+    ranks = np.arange(cfg.T) // cfg.T_r
+    assert np.array_equal(idx[:, cfg.k], ranks * per + L)
+    assert np.all(w[:, cfg.k] == 1.0)
+    # every rank now receives exactly its own T_r shared slots
+    lay = oracle_mod.layout(idx, cfg.E_phys, cfg.R)
+    shared_rows = lay["expert_counts"].reshape(cfg.R, per)[:, L]
+    assert np.all(shared_rows == cfg.T_r)
+
+
+def test_route_ex_multi_replica_choice_and_bad_table(oracle_mod):
+    logits, _ = inputs.make_random_case(24, 8, 6, 2, seed=31)
+    # expert 0 has 3 replicas (ids 6, 7, 8), the others one each (ids 0..5)
+    offs = np.array([0, 3, 4, 5, 6, 7, 8], np.int32)
+    ids = np.array([6, 7, 8, 1, 2, 3, 4, 5], np.int32)
+    idx, _, st = oracle_mod.route_ex(logits.numpy(), 2, 0, 1.0, offs, ids, 9, 4)
+    assert st == oracle_mod.OK
+    plain, _ = oracle_mod.route(logits.numpy(), 2)
+    for g in range(24):
+        for j in range(2):
+            if plain[g, j] == 0:
+                assert idx[g, j] == [6, 7, 8][(g // 4) % 3]
+            else:
+                assert idx[g, j] == plain[g, j]
+    bad = ids.copy()
+    bad[4] = 99                        # expert 2's only replica is out of range
+    idx_b, _, st_b = oracle_mod.route_ex(logits.numpy(), 2, 0, 1.0, offs, bad, 9, 4)
+    assert st_b == oracle_mod.ERR_INVALID
+    assert np.all(idx_b[plain == 2] == -1) and np.all(idx_b[plain != 2] == idx[plain != 2])
