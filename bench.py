@@ -51,7 +51,7 @@ METRIC = "dispatch+combine µs/layer and effective HBM GB/s (% of B200 roofline)
 SPEC_HBM_GBS = 8000.0          # B200 HBM3e bandwidth the roofline target is quoted against
 FALLBACK_HBM_GBS = 6650.0      # earlier measured copy bandwidth on this machine
 L2_FLUSH_BYTES = 512 << 20
-KERNELS_PER_STEP = 5           # route, layout (2 kernels), dispatch, combine
+KERNELS_PER_STEP = 5           # route, layout (2 kernels), dispatch, combine (+1 compaction, two-phase)
 STEPS_PER_GRAPH = 10           # consecutive steps captured in one CUDA graph (no-flush workloads)
 
 
@@ -345,6 +345,17 @@ def run_ours(args) -> None:
             del probe
         rows = T * k if cap == 0 else E_lay * cap
         lay = moe.moe_dispatch_layout(idx, E_lay, R, capacity=cap, rows=rows, workspace=ws)
+        if args.two_phase:
+            if cap:
+                raise SystemExit("--two-phase needs a packed-layout workload")
+            max_m = cfg.T_r                      # a rank sends at most T_r tokens to an expert
+            lay["private_pos"] = torch.empty(T, k, dtype=torch.int32, device=dev)
+            moe.moe_dispatch_layout_private(idx, E_lay, R, max_m, out=lay, workspace=ws)
+            prows = E_lay * R * max_m
+        if args.two_phase and cfg.dispatch == "fp8":
+            priv_q, priv_scale = moe.moe_dispatch_fp8(x, lay["private_pos"], prows)
+        elif args.two_phase:
+            priv_x = moe.moe_dispatch_bf16(x, lay["private_pos"], prows)
         if cfg.dispatch == "fp8":
             recv_q, recv_scale = moe.moe_dispatch_fp8(x, lay["dispatch_pos"], rows)
             y = experts.dequantise(recv_q, recv_scale)
@@ -368,20 +379,43 @@ def run_ours(args) -> None:
                                  w.data_ptr(), None, sp))
         if cfg.n_shared else
         (lib.moe_route_topk, (logits.data_ptr(), T, E, k, 0, idx.data_ptr(), w.data_ptr(), sp)))
-    calls = [
-        route_call,
-        (lib.moe_dispatch_layout, (idx.data_ptr(), T, k, E_lay, R, cap, rows,
-                                   lay["expert_counts"].data_ptr(), lay["expert_src_counts"].data_ptr(),
-                                   lay["rank_counts"].data_ptr(), lay["expert_offsets"].data_ptr(),
-                                   pos.data_ptr(), lay["recv_src"].data_ptr(), ws_buf.data_ptr(),
-                                   ws_buf.numel(), None, sp)),
-        (lib.moe_dispatch_fp8, (x.data_ptr(), T, H, k, pos.data_ptr(), recv_q.data_ptr(),
-                                recv_scale.data_ptr(), rows, None, sp)) if cfg.dispatch == "fp8" else
-        (lib.moe_dispatch_bf16, (x.data_ptr(), T, H, k, pos.data_ptr(), recv_x.data_ptr(), rows,
-                                 None, sp)),
-        (lib.moe_combine_bf16, (y.data_ptr(), pos.data_ptr(), w.data_ptr(), T, H, k, rows,
-                                out.data_ptr(), None, sp)),
-    ]
+    lay_args = (idx.data_ptr(), T, k, E_lay, R, cap, rows, lay["expert_counts"].data_ptr(),
+                lay["expert_src_counts"].data_ptr(), lay["rank_counts"].data_ptr(),
+                lay["expert_offsets"].data_ptr(), pos.data_ptr(), lay["recv_src"].data_ptr())
+    if not args.two_phase:
+        layout_call = (lib.moe_dispatch_layout, lay_args + (ws_buf.data_ptr(), ws_buf.numel(), None, sp))
+        dispatch_calls = [
+            (lib.moe_dispatch_fp8, (x.data_ptr(), T, H, k, pos.data_ptr(), recv_q.data_ptr(),
+                                    recv_scale.data_ptr(), rows, None, sp)) if cfg.dispatch == "fp8" else
+            (lib.moe_dispatch_bf16, (x.data_ptr(), T, H, k, pos.data_ptr(), recv_x.data_ptr(), rows,
+                                     None, sp))]
+    else:
+        # the pages' two-phase form: private-region layout, send into the private
+        # regions, receiver compaction into the packed rows
+        ppos = lay["private_pos"]
+        layout_call = (lib.moe_dispatch_layout_private,
+                       lay_args[:5] + (max_m,) + lay_args[6:] +
+                       (ppos.data_ptr(), ws_buf.data_ptr(), ws_buf.numel(), None, sp))
+        if cfg.dispatch == "fp8":
+            dispatch_calls = [
+                (lib.moe_dispatch_fp8, (x.data_ptr(), T, H, k, ppos.data_ptr(), priv_q.data_ptr(),
+                                        priv_scale.data_ptr(), prows, None, sp)),
+                (lib.moe_compact_fp8, (priv_q.data_ptr(), priv_scale.data_ptr(), prows,
+                                       ppos.data_ptr(), pos.data_ptr(), T, H, k, recv_q.data_ptr(),
+                                       recv_scale.data_ptr(), rows, None, sp))]
+        else:
+            dispatch_calls = [
+                (lib.moe_dispatch_bf16, (x.data_ptr(), T, H, k, ppos.data_ptr(), priv_x.data_ptr(),
+                                         prows, None, sp)),
+                (lib.moe_compact_bf16, (priv_x.data_ptr(), prows, ppos.data_ptr(), pos.data_ptr(),
+                                        T, H, k, recv_x.data_ptr(), rows, None, sp))]
+    calls = [route_call, layout_call, *dispatch_calls,
+             (lib.moe_combine_bf16, (y.data_ptr(), pos.data_ptr(), w.data_ptr(), T, H, k, rows,
+                                     out.data_ptr(), None, sp))]
+    n_dispatch_calls = len(dispatch_calls)
+
+    # stage j ends after these call indices: route, layout, dispatch (1 or 2 calls)
+    stage_end = [0, 1, 1 + n_dispatch_calls]
 
     def step(ev=None):
         """One pass of the path; with `ev`, events ev[1..3] mark the stage ends."""
@@ -389,8 +423,8 @@ def run_ours(args) -> None:
             rc = fn(*a)
             if rc != 0:
                 raise moe.MoeError(rc, fn.__name__)
-            if ev is not None and j < 3:
-                ev[j + 1].record(s)
+            if ev is not None and j in stage_end:
+                ev[stage_end.index(j) + 1].record(s)
 
     nb = algorithmic_bytes(cfg, rows, kept)
     K, W = args.steps, args.warmup
@@ -500,10 +534,12 @@ def run_ours(args) -> None:
         stage_ms = None
     if stage_ms is None:  # one graph per stage, events between replays
         gs = []
-        for j, (fn, a) in enumerate(calls):
+        bounds = [0, *[j + 1 for j in stage_end], len(calls)]
+        for j in range(4):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=s):
-                fn(*a)
+                for fn, a in calls[bounds[j]:bounds[j + 1]]:
+                    fn(*a)
             gs.append(g)
         rows_ms = []
         with torch.cuda.stream(s):
@@ -573,7 +609,10 @@ def run_ours(args) -> None:
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": cfg.describe(), "parallelism": f"replicas x{n_gpus}",
                        "l2": l2_mode,
-                       "capacity": cap, "rows": rows, "timing": (f"CUDA events around K steps run as replays of CUDA graphs of "
+                       "capacity": cap, "rows": rows,
+                       "pipeline": ("two-phase: private-region layout, send into E*R private "
+                                    "regions of T_r rows, receiver compaction" if args.two_phase
+                                    else "direct scatter into the packed rows"), "timing": (f"CUDA events around K steps run as replays of CUDA graphs of "
                                   f"{G} consecutive step(s)")},
             "us_per_layer": ms_step * 1e3,
             "stages_us": {"route": ms_route * 1e3, "layout": ms_layout * 1e3,
@@ -594,7 +633,7 @@ def run_ours(args) -> None:
             "e2e": {"value": n_gpus * nb["step"] / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
                     "us_per_step": e2e_ms * 1e3, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
-            "gpu_launches": KERNELS_PER_STEP * K,
+            "gpu_launches": (KERNELS_PER_STEP + (1 if args.two_phase else 0)) * K,
             "clocks": clocks,
         }
         if world == 1 and not args.no_cpu_baseline:
@@ -614,6 +653,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", choices=sorted(inputs.CONFIGS), default="dsv3")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--two-phase", action="store_true",
+                    help="dispatch as the pages' two-phase form (private regions + compaction)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -20,7 +20,9 @@ __all__ = [
     "MoeError", "lib", "moe_status_string", "moe_route_topk", "moe_route_topk_ex",
     "moe_layout_workspace_bytes",
     "moe_dispatch_layout", "moe_dispatch_bf16", "moe_dispatch_fp8", "moe_combine_bf16",
-    "moe_quantize_e4m3", "moe_dispatch_layout_noalloc", "Workspace", "LIB_PATH",
+    "moe_quantize_e4m3", "moe_dispatch_layout_noalloc", "moe_dispatch_fp8_ex", "Workspace",
+    "LIB_PATH", "MOE_SCALE_ROW_MAJOR", "MOE_SCALE_COL_MAJOR", "moe_dispatch_layout_private",
+    "moe_compact_fp8", "moe_compact_bf16",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_route.so")
@@ -50,10 +52,19 @@ lib.moe_dispatch_layout.restype = _i32
 lib.moe_dispatch_layout_noalloc.argtypes = [_P, _i32, _i32, _i32, _i32, _i32, _i64, _P, _P, _P,
                                             _P, _P, _P, _P, _P]
 lib.moe_dispatch_layout_noalloc.restype = _i32
+lib.moe_dispatch_layout_private.argtypes = [_P, _i32, _i32, _i32, _i32, _i32, _i64, _P, _P, _P, _P,
+                                            _P, _P, _P, _P, _sz, _P, _P]
+lib.moe_dispatch_layout_private.restype = _i32
+lib.moe_compact_fp8.argtypes = [_P, _P, _i64, _P, _P, _i32, _i32, _i32, _P, _P, _i64, _P, _P]
+lib.moe_compact_fp8.restype = _i32
+lib.moe_compact_bf16.argtypes = [_P, _i64, _P, _P, _i32, _i32, _i32, _P, _i64, _P, _P]
+lib.moe_compact_bf16.restype = _i32
 lib.moe_dispatch_bf16.argtypes = [_P, _i32, _i32, _i32, _P, _P, _i64, _P, _P]
 lib.moe_dispatch_bf16.restype = _i32
 lib.moe_dispatch_fp8.argtypes = [_P, _i32, _i32, _i32, _P, _P, _P, _i64, _P, _P]
 lib.moe_dispatch_fp8.restype = _i32
+lib.moe_dispatch_fp8_ex.argtypes = [_P, _i32, _i32, _i32, _P, _P, _P, _i64, _i32, _i64, _P, _P]
+lib.moe_dispatch_fp8_ex.restype = _i32
 lib.moe_combine_bf16.argtypes = [_P, _P, _P, _i32, _i32, _i32, _i64, _P, _P, _P]
 lib.moe_combine_bf16.restype = _i32
 lib.moe_quantize_e4m3.argtypes = [_P, _i64, _P, _P]
@@ -66,6 +77,8 @@ MOE_ERR_CAPACITY = 3
 MOE_ERR_WORKSPACE = 4
 MOE_ERR_TIMEOUT = 5
 MOE_ERR_CUDA = 6
+MOE_SCALE_ROW_MAJOR = 0
+MOE_SCALE_COL_MAJOR = 1
 
 
 class MoeError(RuntimeError):
@@ -239,6 +252,77 @@ def moe_dispatch_layout_noalloc(topk_idx: torch.Tensor, E: int, R: int, capacity
     return out
 
 
+def moe_dispatch_layout_private(topk_idx: torch.Tensor, E: int, R: int, max_m: int,
+                                rows: int | None = None, out: dict | None = None,
+                                workspace: Workspace | None = None,
+                                dev_status: torch.Tensor | None = None, stream=None) -> dict:
+    """Two-phase layout: everything moe_dispatch_layout (packed) returns plus
+    private_pos [T][k], the row of each slot in its (expert, source rank)
+    private region of max_m rows (E*R*max_m private rows in all)."""
+    assert topk_idx.dtype == torch.int32 and topk_idx.dim() == 2
+    T, k = topk_idx.shape
+    dev = topk_idx.device
+    if rows is None:
+        rows = T * k
+    if out is None:
+        out = dict(
+            expert_counts=torch.empty(E, dtype=torch.int32, device=dev),
+            expert_src_counts=torch.empty(E, R, dtype=torch.int32, device=dev),
+            rank_counts=torch.empty(R, dtype=torch.int32, device=dev),
+            expert_offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
+            dispatch_pos=torch.empty(T, k, dtype=torch.int32, device=dev),
+            recv_src=torch.empty(max(rows, 1), dtype=torch.int32, device=dev),
+            private_pos=torch.empty(T, k, dtype=torch.int32, device=dev),
+        )
+    if workspace is None:
+        workspace = _default_ws.setdefault(dev, Workspace(dev))
+    nbytes = moe_layout_workspace_bytes(T, k, E, R)
+    if nbytes == 0:
+        raise MoeError(MOE_ERR_INVALID_ARG, "moe_layout_workspace_bytes")
+    ws = workspace.get(nbytes)
+    _check(lib.moe_dispatch_layout_private(
+        _ptr(topk_idx), T, k, E, R, max_m, rows,
+        _ptr(out["expert_counts"]), _ptr(out["expert_src_counts"]), _ptr(out["rank_counts"]),
+        _ptr(out["expert_offsets"]), _ptr(out["dispatch_pos"]), _ptr(out["recv_src"]),
+        _ptr(out["private_pos"]), _ptr(ws), ws.numel(), _ptr(dev_status), _stream(stream)),
+        "moe_dispatch_layout_private")
+    out["rows"] = rows
+    out["private_rows"] = E * R * max_m
+    return out
+
+
+def moe_compact_fp8(priv_q: torch.Tensor, priv_scale: torch.Tensor, private_pos: torch.Tensor,
+                    dispatch_pos: torch.Tensor, rows: int, recv_q: torch.Tensor | None = None,
+                    recv_scale: torch.Tensor | None = None, dev_status: torch.Tensor | None = None,
+                    stream=None):
+    """Receive phase: copy each slot's private fp8 row and scales to its packed row."""
+    prows, H = priv_q.shape
+    T, k = dispatch_pos.shape
+    if recv_q is None:
+        recv_q = torch.empty(rows, H, dtype=torch.uint8, device=priv_q.device)
+    if recv_scale is None:
+        recv_scale = torch.empty(rows, max(H // 128, 1), dtype=torch.float32, device=priv_q.device)
+    _check(lib.moe_compact_fp8(_ptr(priv_q), _ptr(priv_scale), prows, _ptr(private_pos),
+                               _ptr(dispatch_pos), T, H, k, _ptr(recv_q), _ptr(recv_scale), rows,
+                               _ptr(dev_status), _stream(stream)), "moe_compact_fp8")
+    return recv_q, recv_scale
+
+
+def moe_compact_bf16(priv_x: torch.Tensor, private_pos: torch.Tensor, dispatch_pos: torch.Tensor,
+                     rows: int, recv_x: torch.Tensor | None = None,
+                     dev_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Receive phase: copy each slot's private bf16 row to its packed row."""
+    priv_x = _bits16(priv_x)
+    prows, H = priv_x.shape
+    T, k = dispatch_pos.shape
+    if recv_x is None:
+        recv_x = torch.empty(rows, H, dtype=priv_x.dtype, device=priv_x.device)
+    _check(lib.moe_compact_bf16(_ptr(priv_x), prows, _ptr(private_pos), _ptr(dispatch_pos), T, H, k,
+                                _ptr(recv_x), rows, _ptr(dev_status), _stream(stream)),
+           "moe_compact_bf16")
+    return recv_x
+
+
 def moe_dispatch_bf16(x: torch.Tensor, dispatch_pos: torch.Tensor, rows: int,
                       recv_x: torch.Tensor | None = None, dev_status: torch.Tensor | None = None,
                       stream=None) -> torch.Tensor:
@@ -268,6 +352,30 @@ def moe_dispatch_fp8(x: torch.Tensor, dispatch_pos: torch.Tensor, rows: int,
     _check(lib.moe_dispatch_fp8(_ptr(x), T, H, k, _ptr(dispatch_pos), _ptr(recv_q),
                                 _ptr(recv_scale), rows, _ptr(dev_status), _stream(stream)),
            "moe_dispatch_fp8")
+    return recv_q, recv_scale
+
+
+def moe_dispatch_fp8_ex(x: torch.Tensor, dispatch_pos: torch.Tensor, rows: int,
+                        scale_layout: int = MOE_SCALE_COL_MAJOR, scale_ld: int | None = None,
+                        recv_q: torch.Tensor | None = None, recv_scale: torch.Tensor | None = None,
+                        dev_status: torch.Tensor | None = None, stream=None):
+    """moe_dispatch_fp8 with the scales column-major [H/128][scale_ld]
+    (scale_ld = rows rounded up to a multiple of 4 by default) or row-major.
+    Returns (recv_q uint8 [rows][H], recv_scale)."""
+    x = _bits16(x)
+    T, H = x.shape
+    k = dispatch_pos.shape[1]
+    S = max(H // 128, 1)
+    if scale_ld is None:
+        scale_ld = (rows + 3) // 4 * 4 if scale_layout == MOE_SCALE_COL_MAJOR else 0
+    if recv_q is None:
+        recv_q = torch.empty(rows, H, dtype=torch.uint8, device=x.device)
+    if recv_scale is None:
+        shape = (S, scale_ld) if scale_layout == MOE_SCALE_COL_MAJOR else (rows, S)
+        recv_scale = torch.empty(shape, dtype=torch.float32, device=x.device)
+    _check(lib.moe_dispatch_fp8_ex(_ptr(x), T, H, k, _ptr(dispatch_pos), _ptr(recv_q),
+                                   _ptr(recv_scale), rows, scale_layout, scale_ld,
+                                   _ptr(dev_status), _stream(stream)), "moe_dispatch_fp8_ex")
     return recv_q, recv_scale
 
 

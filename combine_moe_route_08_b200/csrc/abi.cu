@@ -130,8 +130,79 @@ int moe_dispatch_layout(const int32_t *topk_idx, int T, int k, int E, int R, int
         return MOE_ERR_WORKSPACE;
     return launched(moe::dispatch_layout(topk_idx, g, capacity, rows, expert_counts,
                                          expert_src_counts, rank_counts, expert_offsets,
-                                         dispatch_pos, recv_src, workspace, dev_status,
+                                         dispatch_pos, recv_src, nullptr, workspace, dev_status,
                                          as_stream(stream)));
+}
+
+int moe_dispatch_layout_private(const int32_t *topk_idx, int T, int k, int E, int R, int max_m,
+                                int64_t rows, int32_t *expert_counts, int32_t *expert_src_counts,
+                                int32_t *rank_counts, int32_t *expert_offsets,
+                                int32_t *dispatch_pos, int32_t *recv_src, int32_t *private_pos,
+                                void *workspace, size_t ws_bytes, int32_t *dev_status,
+                                void *stream)
+{
+    if (!valid_layout_sizes(T, k, E, R) || max_m < 1 || rows < static_cast<int64_t>(T) * k ||
+        rows >= kMaxIndex || static_cast<int64_t>(E) * R * max_m >= kMaxIndex)
+        return MOE_ERR_INVALID_ARG;
+    const void *arrays[] = {expert_counts, expert_src_counts, rank_counts, expert_offsets};
+    for (const void *p : arrays)
+        if (!p || !aligned(p, 4))
+            return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!topk_idx || !dispatch_pos || !private_pos || !aligned(topk_idx, 4) ||
+                  !aligned(dispatch_pos, 4) || !aligned(private_pos, 4)))
+        return MOE_ERR_INVALID_ARG;
+    if (rows > 0 && (!recv_src || !aligned(recv_src, 4)))
+        return MOE_ERR_INVALID_ARG;
+    if (dev_status && !aligned(dev_status, 4))
+        return MOE_ERR_INVALID_ARG;
+    moe::LayoutGeom g = moe::layout_geom(T, k, E, R);
+    g.max_m = max_m;
+    if (!workspace || !aligned(workspace, 256) || ws_bytes < moe::layout_workspace_bytes(g))
+        return MOE_ERR_WORKSPACE;
+    return launched(moe::dispatch_layout(topk_idx, g, 0, rows, expert_counts, expert_src_counts,
+                                         rank_counts, expert_offsets, dispatch_pos, recv_src,
+                                         private_pos, workspace, dev_status, as_stream(stream)));
+}
+
+int moe_compact_fp8(const uint8_t *priv_q, const float *priv_scale, int64_t private_rows,
+                    const int32_t *private_pos, const int32_t *dispatch_pos, int T, int H, int k,
+                    uint8_t *recv_q, float *recv_scale, int64_t rows, int32_t *dev_status,
+                    void *stream)
+{
+    const int st = check_rows_args(T, H, k, dispatch_pos, rows);
+    if (st != MOE_OK)
+        return st;
+    if (H % 128 != 0)
+        return MOE_ERR_UNSUPPORTED;
+    if (private_rows < 0 || private_rows >= kMaxIndex)
+        return MOE_ERR_INVALID_ARG;
+    if (T == 0)
+        return MOE_OK;
+    if (!priv_q || !priv_scale || !private_pos || !recv_q || !recv_scale || !aligned(priv_q, 16) ||
+        !aligned(recv_q, 16) || !aligned(priv_scale, 4) || !aligned(recv_scale, 4) ||
+        !aligned(private_pos, 4) || (dev_status && !aligned(dev_status, 4)))
+        return MOE_ERR_INVALID_ARG;
+    return launched(moe::compact_fp8(priv_q, priv_scale, private_rows, private_pos, dispatch_pos, T,
+                                     H, k, recv_q, recv_scale, rows, dev_status,
+                                     as_stream(stream)));
+}
+
+int moe_compact_bf16(const uint16_t *priv_x, int64_t private_rows, const int32_t *private_pos,
+                     const int32_t *dispatch_pos, int T, int H, int k, uint16_t *recv_x,
+                     int64_t rows, int32_t *dev_status, void *stream)
+{
+    const int st = check_rows_args(T, H, k, dispatch_pos, rows);
+    if (st != MOE_OK)
+        return st;
+    if (private_rows < 0 || private_rows >= kMaxIndex)
+        return MOE_ERR_INVALID_ARG;
+    if (T == 0)
+        return MOE_OK;
+    if (!priv_x || !private_pos || !recv_x || !aligned(priv_x, 16) || !aligned(recv_x, 16) ||
+        !aligned(private_pos, 4) || (dev_status && !aligned(dev_status, 4)))
+        return MOE_ERR_INVALID_ARG;
+    return launched(moe::compact_bf16(priv_x, private_rows, private_pos, dispatch_pos, T, H, k,
+                                      recv_x, rows, dev_status, as_stream(stream)));
 }
 
 int moe_dispatch_bf16(const uint16_t *x, int T, int H, int k, const int32_t *dispatch_pos,
@@ -163,7 +234,31 @@ int moe_dispatch_fp8(const uint16_t *x, int T, int H, int k, const int32_t *disp
     if (!x || !recv_q || !recv_scale || !aligned(x, 16) || !aligned(recv_q, 16) ||
         !aligned(recv_scale, 4) || (dev_status && !aligned(dev_status, 4)))
         return MOE_ERR_INVALID_ARG;
-    return launched(moe::dispatch_fp8(x, T, H, k, dispatch_pos, recv_q, recv_scale, rows,
+    return launched(moe::dispatch_fp8(x, T, H, k, dispatch_pos, recv_q, recv_scale, rows, 0,
+                                      dev_status, as_stream(stream)));
+}
+
+int moe_dispatch_fp8_ex(const uint16_t *x, int T, int H, int k, const int32_t *dispatch_pos,
+                        uint8_t *recv_q, float *recv_scale, int64_t rows, int scale_layout,
+                        int64_t scale_ld, int32_t *dev_status, void *stream)
+{
+    if (scale_layout == MOE_SCALE_ROW_MAJOR)
+        return moe_dispatch_fp8(x, T, H, k, dispatch_pos, recv_q, recv_scale, rows, dev_status,
+                                stream);
+    if (scale_layout != MOE_SCALE_COL_MAJOR || scale_ld < rows || scale_ld % 4 != 0 ||
+        scale_ld >= kMaxIndex)
+        return MOE_ERR_INVALID_ARG;
+    const int st = check_rows_args(T, H, k, dispatch_pos, rows);
+    if (st != MOE_OK)
+        return st;
+    if (H % 128 != 0)
+        return MOE_ERR_UNSUPPORTED;
+    if (T == 0)
+        return MOE_OK;
+    if (!x || !recv_q || !recv_scale || !aligned(x, 16) || !aligned(recv_q, 16) ||
+        !aligned(recv_scale, 16) || (dev_status && !aligned(dev_status, 4)))
+        return MOE_ERR_INVALID_ARG;
+    return launched(moe::dispatch_fp8(x, T, H, k, dispatch_pos, recv_q, recv_scale, rows, scale_ld,
                                       dev_status, as_stream(stream)));
 }
 

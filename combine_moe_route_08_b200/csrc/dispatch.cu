@@ -62,10 +62,14 @@ __global__ void __launch_bounds__(kMaxThreads)
 // 128-channel block are 8 consecutive lanes, so the block's amax is a 3-step
 // xor shuffle.  s = amax / 448 and every x / s are IEEE binary32 divisions
 // (__fdiv_rn), then the hardware converts to e4m3 with RNE + saturation.
+// Scales go to recv_scale[r * S + b] (row-major) or, with scale_ld > 0, to
+// recv_scale[b * scale_ld + r] (column-major: each 128-channel block's scales
+// contiguous over the rows, the operand layout of a grouped FP8 GEMM).
 __global__ void __launch_bounds__(kMaxThreads)
     k_dispatch_fp8(const uint4 *__restrict__ x, int H, int k,
                    const int32_t *__restrict__ dispatch_pos, uint8_t *__restrict__ recv_q,
-                   float *__restrict__ recv_scale, int64_t rows, int32_t *__restrict__ dev_status)
+                   float *__restrict__ recv_scale, int64_t rows, int64_t scale_ld,
+                   int32_t *__restrict__ dev_status)
 {
     __shared__ int32_t srow[kMaxK];
     const int g = blockIdx.x;
@@ -112,8 +116,12 @@ __global__ void __launch_bounds__(kMaxThreads)
                 if (r < 0)
                     continue;
                 st_stream_v4(recv_q + static_cast<size_t>(r) * H + 16 * t, q);
-                if ((t & 7) == 0)
-                    __stcs(recv_scale + static_cast<size_t>(r) * S + (t >> 3), s);
+                if ((t & 7) == 0) {
+                    const size_t at = (scale_ld > 0)
+                                          ? static_cast<size_t>(t >> 3) * scale_ld + r
+                                          : static_cast<size_t>(r) * S + (t >> 3);
+                    __stcs(recv_scale + at, s);
+                }
             }
         }
     }
@@ -155,12 +163,12 @@ cudaError_t dispatch_bf16(const uint16_t *x, int T, int H, int k, const int32_t 
 }
 
 cudaError_t dispatch_fp8(const uint16_t *x, int T, int H, int k, const int32_t *dispatch_pos,
-                         uint8_t *recv_q, float *recv_scale, int64_t rows, int32_t *dev_status,
-                         cudaStream_t s)
+                         uint8_t *recv_q, float *recv_scale, int64_t rows, int64_t scale_ld,
+                         int32_t *dev_status, cudaStream_t s)
 {
     return launch_pdl(k_dispatch_fp8, dim3(T), dim3(threads_for(H / 16)), 0, s,
                       reinterpret_cast<const uint4 *>(x), H, k, dispatch_pos, recv_q, recv_scale,
-                      rows, dev_status);
+                      rows, scale_ld, dev_status);
 }
 
 cudaError_t quantize_e4m3(const float *v, int64_t n, uint8_t *q, cudaStream_t s)

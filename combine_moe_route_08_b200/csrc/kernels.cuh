@@ -17,6 +17,7 @@ struct LayoutGeom {
     int CT;       // tokens per chunk
     int cpr;      // chunks per rank
     int nchunks;  // R * cpr
+    int max_m;    // > 0: also place every slot in its private (expert, source rank) region
 };
 
 LayoutGeom layout_geom(int T, int k, int E, int R);
@@ -39,18 +40,31 @@ struct RouteEx {
 cudaError_t route_topk(const float *logits, int T, int E, int k, int renormalize,
                        int32_t *topk_idx, float *topk_w, const RouteEx *ex, cudaStream_t s);
 
+// private_pos: [T][k] private rows when g.max_m > 0 (else unused, may be null).
 cudaError_t dispatch_layout(const int32_t *topk_idx, const LayoutGeom &g, int capacity,
                             int64_t rows, int32_t *expert_counts, int32_t *expert_src_counts,
                             int32_t *rank_counts, int32_t *expert_offsets,
-                            int32_t *dispatch_pos, int32_t *recv_src, void *workspace,
-                            int32_t *dev_status, cudaStream_t s);
+                            int32_t *dispatch_pos, int32_t *recv_src, int32_t *private_pos,
+                            void *workspace, int32_t *dev_status, cudaStream_t s);
+
+// Receiver side of the two-phase dispatch: copy every slot's private row to
+// its packed row (codes and scales / bf16 rows).
+cudaError_t compact_fp8(const uint8_t *priv_q, const float *priv_scale, int64_t private_rows,
+                        const int32_t *private_pos, const int32_t *dispatch_pos, int T, int H,
+                        int k, uint8_t *recv_q, float *recv_scale, int64_t rows,
+                        int32_t *dev_status, cudaStream_t s);
+cudaError_t compact_bf16(const uint16_t *priv_x, int64_t private_rows, const int32_t *private_pos,
+                         const int32_t *dispatch_pos, int T, int H, int k, uint16_t *recv_x,
+                         int64_t rows, int32_t *dev_status, cudaStream_t s);
 
 cudaError_t dispatch_bf16(const uint16_t *x, int T, int H, int k, const int32_t *dispatch_pos,
                           uint16_t *recv_x, int64_t rows, int32_t *dev_status, cudaStream_t s);
 
+// scale_ld == 0: scales row-major [rows][H/128]; > 0: column-major
+// [H/128][scale_ld] (scale_ld >= rows).
 cudaError_t dispatch_fp8(const uint16_t *x, int T, int H, int k, const int32_t *dispatch_pos,
-                         uint8_t *recv_q, float *recv_scale, int64_t rows, int32_t *dev_status,
-                         cudaStream_t s);
+                         uint8_t *recv_q, float *recv_scale, int64_t rows, int64_t scale_ld,
+                         int32_t *dev_status, cudaStream_t s);
 
 cudaError_t combine_bf16(const uint16_t *y, const int32_t *dispatch_pos, const float *topk_w,
                          int T, int H, int k, int64_t rows, uint16_t *out, int32_t *dev_status,

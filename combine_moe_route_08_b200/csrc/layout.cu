@@ -197,7 +197,8 @@ __global__ void __launch_bounds__(kThreads)
                     const int32_t *__restrict__ ws_hist, int32_t *__restrict__ expert_counts,
                     int32_t *__restrict__ expert_src_counts, int32_t *__restrict__ rank_counts,
                     int32_t *__restrict__ expert_offsets, int32_t *__restrict__ dispatch_pos,
-                    int32_t *__restrict__ recv_src, int32_t *__restrict__ dev_status)
+                    int32_t *__restrict__ recv_src, int32_t *__restrict__ private_pos,
+                    int32_t *__restrict__ dev_status)
 {
     extern __shared__ int32_t sm[];
     const int E = G.E, lane = threadIdx.x & 31, w = threadIdx.x >> 5;
@@ -205,7 +206,8 @@ __global__ void __launch_bounds__(kThreads)
     int32_t *wh = sm;                   // [kWarps][E] per-warp counts, then bases
     int32_t *off = wh + kWarps * E;     // [E + 1] expert totals, then their scan
     int32_t *chb = off + E + 1;         // [E] slots of e in earlier chunks
-    int32_t *tot = chb + E;             // [kWarps + 1]
+    int32_t *rbs = chb + E;             // [E] slots of e in chunks of earlier ranks
+    int32_t *tot = rbs + E;             // [kWarps + 1]
     const int c = blockIdx.x;
 
     int64_t w0, w1;
@@ -214,7 +216,7 @@ __global__ void __launch_bounds__(kThreads)
     int e[kMaxSteps];
     load_run(topk_idx, w0, w1, e);  // in flight while the columns are summed
 
-    for (int x = threadIdx.x + 3 * max(1, min(kThreads / E, kWarps / 3)) * E; x < kWarps * E;
+    for (int x = threadIdx.x + 4 * max(1, min(kThreads / E, kWarps / 4)) * E; x < kWarps * E;
          x += kThreads)
         wh[x] = 0;
 
@@ -224,14 +226,14 @@ __global__ void __launch_bounds__(kThreads)
     // part of the chunks (coalesced over experts); the parts meet in shared
     // memory (the per-warp rows, not yet used).
     const int n = G.nchunks;
-    const int P = max(1, min(kThreads / E, kWarps / 3));
+    const int P = max(1, min(kThreads / E, kWarps / 4));
     const int r = c / G.cpr;
     {
         const int x = threadIdx.x % E, part = threadIdx.x / E;
         if (part < P) {
             const int per = ceil_div(n, P);
             const int cb = part * per, ce = min(n, cb + per);
-            int before = 0, total = 0, mine = 0;
+            int before = 0, total = 0, mine = 0, rstart = 0;
             for (int c0 = cb; c0 < ce; c0 += kColBatch) {
                 int v[kColBatch];
 #pragma unroll
@@ -241,32 +243,36 @@ __global__ void __launch_bounds__(kThreads)
                 for (int u = 0; u < kColBatch; ++u) {
                     const int cc = c0 + u;
                     before += (cc < c) ? v[u] : 0;
+                    rstart += (cc < r * G.cpr) ? v[u] : 0;
                     total += v[u];
                     mine += (cc >= r * G.cpr && cc < (r + 1) * G.cpr) ? v[u] : 0;
                 }
             }
-            wh[(3 * part) * E + x] = before;
-            wh[(3 * part + 1) * E + x] = total;
-            wh[(3 * part + 2) * E + x] = mine;
+            wh[(4 * part) * E + x] = before;
+            wh[(4 * part + 1) * E + x] = total;
+            wh[(4 * part + 2) * E + x] = mine;
+            wh[(4 * part + 3) * E + x] = rstart;
         }
     }
     __syncthreads();
     for (int x = threadIdx.x; x < E; x += kThreads) {
-        int before = 0, total = 0, mine = 0;
+        int before = 0, total = 0, mine = 0, rstart = 0;
         for (int part = 0; part < P; ++part) {
-            before += wh[(3 * part) * E + x];
-            total += wh[(3 * part + 1) * E + x];
-            mine += wh[(3 * part + 2) * E + x];
+            before += wh[(4 * part) * E + x];
+            total += wh[(4 * part + 1) * E + x];
+            mine += wh[(4 * part + 2) * E + x];
+            rstart += wh[(4 * part + 3) * E + x];
         }
         off[x] = total;
         chb[x] = before;
+        rbs[x] = rstart;
         if (c == 0)
             expert_counts[x] = total;
         if (c == r * G.cpr)  // first chunk of its rank writes the rank's column
             expert_src_counts[static_cast<size_t>(x) * G.R + r] = mine;
     }
     __syncthreads();
-    for (int x = threadIdx.x; x < 3 * P * E; x += kThreads)
+    for (int x = threadIdx.x; x < 4 * P * E; x += kThreads)
         wh[x] = 0;
     __syncthreads();
 
@@ -318,7 +324,8 @@ __global__ void __launch_bounds__(kThreads)
             mywh[e[s]] += __popc(mask);
         __syncwarp();
         if (i < w1) {
-            int64_t row = -1;
+            int64_t row = -1, prow = -1;
+            bool hole = false;  // private mode: packed row left empty by a dropped slot
             if (valid) {
                 if (capacity == 0)
                     row = off[e[s]] + p;
@@ -326,14 +333,26 @@ __global__ void __launch_bounds__(kThreads)
                     row = static_cast<int64_t>(e[s]) * capacity + p;
                 else
                     dropped = true;
+                if (G.max_m > 0 && row >= 0) {
+                    // position among this rank's slots of the expert
+                    const int pr = p - rbs[e[s]];
+                    if (pr < G.max_m) {
+                        prow = (static_cast<int64_t>(e[s]) * G.R + r) * G.max_m + pr;
+                    } else {
+                        dropped = true;
+                        hole = true;
+                    }
+                }
             }
             if (row >= rows) {  // cannot happen for a consistent layout; never write past rows
                 bad_row = true;
                 row = -1;
             }
-            dispatch_pos[i] = static_cast<int32_t>(row);
+            dispatch_pos[i] = hole ? -1 : static_cast<int32_t>(row);
             if (row >= 0)
-                recv_src[row] = static_cast<int32_t>(i);
+                recv_src[row] = hole ? -1 : static_cast<int32_t>(i);
+            if (G.max_m > 0)
+                private_pos[i] = static_cast<int32_t>(prow);
         }
     }
     if (dropped)
@@ -359,7 +378,7 @@ __global__ void __launch_bounds__(kThreads)
     pdl_trigger();
 }
 
-size_t assign_smem_bytes(int E) { return (static_cast<size_t>(kWarps + 2) * E + 1 + kWarps + 1) * sizeof(int32_t); }
+size_t assign_smem_bytes(int E) { return (static_cast<size_t>(kWarps + 3) * E + 1 + kWarps + 1) * sizeof(int32_t); }
 
 }  // namespace
 
@@ -374,6 +393,7 @@ LayoutGeom layout_geom(int T, int k, int E, int R)
     g.CT = std::max(1, kChunkSlots / k);  // at most 8192 slots per chunk
     g.cpr = std::max(1, ceil_div(g.Tr, g.CT));
     g.nchunks = R * g.cpr;
+    g.max_m = 0;
     return g;
 }
 
@@ -386,8 +406,8 @@ size_t layout_workspace_bytes(const LayoutGeom &g)
 cudaError_t dispatch_layout(const int32_t *topk_idx, const LayoutGeom &g, int capacity, int64_t rows,
                             int32_t *expert_counts, int32_t *expert_src_counts,
                             int32_t *rank_counts, int32_t *expert_offsets, int32_t *dispatch_pos,
-                            int32_t *recv_src, void *workspace, int32_t *dev_status,
-                            cudaStream_t s)
+                            int32_t *recv_src, int32_t *private_pos, void *workspace,
+                            int32_t *dev_status, cudaStream_t s)
 {
     int32_t *hist = static_cast<int32_t *>(workspace);
     cudaError_t err = launch_pdl(k_layout_hist, dim3(g.nchunks), dim3(kThreads), g.E * sizeof(int32_t),
@@ -403,7 +423,7 @@ cudaError_t dispatch_layout(const int32_t *topk_idx, const LayoutGeom &g, int ca
     }
     return launch_pdl(k_layout_assign, dim3(g.nchunks), dim3(kThreads), smem, s, topk_idx, g, capacity,
                       rows, hist, expert_counts, expert_src_counts, rank_counts, expert_offsets,
-                      dispatch_pos, recv_src, dev_status);
+                      dispatch_pos, recv_src, private_pos, dev_status);
 }
 
 }  // namespace moe

@@ -178,6 +178,54 @@ int moe_dispatch_layout(const int32_t *topk_idx, int T, int k, int E, int R,
                         int32_t *dev_status, void *stream);
 
 /*
+ * Two-phase dispatch (the pages' own design, for comparison with the direct
+ * scatter above).  "Efficient and portable mixture-of-experts
+ * communication", "Kernels portáteis": each rank keeps private storage to
+ * receive from every other rank; the number of tokens a source rank may
+ * dispatch is fixed, which bounds what a rank receives for each local expert
+ * from each source rank, so senders derive unique addresses without
+ * synchronising; after receiving, the tokens are reorganised into the layout
+ * the expert kernels need ("Despacho": copied into contiguous buffers).
+ *
+ * moe_dispatch_layout_private -- everything moe_dispatch_layout (packed,
+ * capacity 0) outputs, identically, plus
+ *   private_pos [T][k] int32 out: the slot's row in the private region of
+ *               (its expert e, its source rank r): rows
+ *               [(e*R + r)*max_m, (e*R + r + 1)*max_m), position = number of
+ *               earlier slots of the same source rank routed to e.  A slot at
+ *               position >= max_m is dropped: private_pos and dispatch_pos -1,
+ *               its packed row left empty (recv_src -1), MOE_ERR_CAPACITY
+ *               through dev_status.  max_m = T/R never drops (a token picks an
+ *               expert at most once).
+ * The private rows hold E*R*max_m rows (< 2^31).  Send phase: moe_dispatch_fp8
+ * (or _bf16) with private_pos as dispatch_pos and rows = E*R*max_m.
+ */
+int moe_dispatch_layout_private(const int32_t *topk_idx, int T, int k, int E, int R, int max_m,
+                                int64_t rows, int32_t *expert_counts, int32_t *expert_src_counts,
+                                int32_t *rank_counts, int32_t *expert_offsets,
+                                int32_t *dispatch_pos, int32_t *recv_src, int32_t *private_pos,
+                                void *workspace, size_t ws_bytes, int32_t *dev_status,
+                                void *stream);
+
+/*
+ * moe_compact_fp8 / moe_compact_bf16 -- receive phase of the two-phase
+ * dispatch: for every slot with private_pos >= 0, copy its private row
+ * (codes and 1x128 scales, or bf16 row) to row dispatch_pos of the packed
+ * buffers.  The result is byte-for-byte what moe_dispatch_fp8 / _bf16 write
+ * with dispatch_pos directly.  A row outside [0, private_rows) or [0, rows)
+ * is skipped and reported (MOE_ERR_INVALID_ARG via dev_status).
+ *   priv_q [private_rows][H] u8, priv_scale [private_rows][H/128] fp32 (or
+ *   priv_x [private_rows][H] bf16) -> recv_q / recv_scale (recv_x) [rows][...].
+ */
+int moe_compact_fp8(const uint8_t *priv_q, const float *priv_scale, int64_t private_rows,
+                    const int32_t *private_pos, const int32_t *dispatch_pos, int T, int H, int k,
+                    uint8_t *recv_q, float *recv_scale, int64_t rows, int32_t *dev_status,
+                    void *stream);
+int moe_compact_bf16(const uint16_t *priv_x, int64_t private_rows, const int32_t *private_pos,
+                     const int32_t *dispatch_pos, int T, int H, int k, uint16_t *recv_x,
+                     int64_t rows, int32_t *dev_status, void *stream);
+
+/*
  * moe_dispatch_layout_noalloc -- moe_dispatch_layout for callers that cannot
  * allocate device memory.  The pages have no counterpart: this is a
  * deployment variant of the entry point above, not a step of the method.
@@ -253,6 +301,28 @@ int moe_dispatch_fp8(const uint16_t *x, int T, int H, int k,
                      const int32_t *dispatch_pos, uint8_t *recv_q,
                      float *recv_scale, int64_t rows, int32_t *dev_status,
                      void *stream);
+
+/*
+ * moe_dispatch_fp8_ex -- moe_dispatch_fp8 with a choice of scale layout for
+ * the grouped GEMM that consumes the rows.  The codes, the scale values and
+ * the rows written are exactly those of moe_dispatch_fp8 (DeepSeek-V3
+ * fragments: 1x128 activation tiles); only where each scale is stored
+ * changes.
+ *   scale_layout MOE_SCALE_ROW_MAJOR: recv_scale [rows][H/128] (scale_ld
+ *                ignored), as moe_dispatch_fp8.
+ *   scale_layout MOE_SCALE_COL_MAJOR: recv_scale [H/128][scale_ld], the scale
+ *                of row r and block b at recv_scale[b * scale_ld + r];
+ *                scale_ld >= rows and scale_ld % 4 == 0 so every block's
+ *                column starts 16-byte aligned (recv_scale itself 16-byte
+ *                aligned), the layout a tile load along the rows needs.
+ *                Entries of rows no slot fills are not written.
+ */
+#define MOE_SCALE_ROW_MAJOR 0
+#define MOE_SCALE_COL_MAJOR 1
+
+int moe_dispatch_fp8_ex(const uint16_t *x, int T, int H, int k, const int32_t *dispatch_pos,
+                        uint8_t *recv_q, float *recv_scale, int64_t rows, int scale_layout,
+                        int64_t scale_ld, int32_t *dev_status, void *stream);
 
 /*
  * moe_combine_bf16 -- gather each token's k expert outputs and form the

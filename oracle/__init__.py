@@ -54,6 +54,8 @@ def _load():
         lib.oracle_route_ex.restype = i32
         lib.oracle_layout.argtypes = [P, i32, i32, i32, i32, i32, i64, P, P, P, P, P, P]
         lib.oracle_layout.restype = i32
+        lib.oracle_private_layout.argtypes = [P, i32, i32, i32, i32, i32, P, P, P]
+        lib.oracle_private_layout.restype = i32
         lib.oracle_dispatch_bf16.argtypes = [P, i32, i32, i32, P, P, i64]
         lib.oracle_dispatch_bf16.restype = i32
         lib.oracle_dispatch_fp8.argtypes = [P, i32, i32, i32, P, P, P, i64]
@@ -159,6 +161,21 @@ def layout(topk_idx: np.ndarray, E: int, R: int, capacity: int = 0, rows: int | 
         raise ValueError("bad rows")
     out["status"] = st
     return out
+
+
+def private_layout(topk_idx: np.ndarray, E: int, R: int, max_m: int):
+    """Two-phase layout: private row of each slot in the (expert, source rank)
+    regions of max_m rows, the packed row base of each region, and the slot
+    held by each private row.  Returns (private_pos [T][k], region_base
+    [E][R], recv_src_private [E*R*max_m], status)."""
+    topk_idx = _c(topk_idx, np.int32)
+    T, k = topk_idx.shape
+    pos = np.empty((T, k), np.int32)
+    base = np.empty((E, R), np.int32)
+    src = np.empty(E * R * max_m, np.int32)
+    st = _load().oracle_private_layout(_ptr(topk_idx), T, k, E, R, max_m, _ptr(pos), _ptr(base),
+                                       _ptr(src))
+    return pos, base, src, st
 
 
 # --------------------------------------------------------------------------

@@ -414,6 +414,79 @@ int oracle_layout(const int32_t *topk_idx, int T, int k, int E, int R,
     return status;
 }
 
+/* Two-phase form [EPMC "Kernels portáteis": each rank keeps private storage
+ * to receive from every other rank; the number of tokens a DP group may
+ * dispatch is fixed, which bounds what a rank receives for each local
+ * expert from each source rank, so senders derive unique addresses without
+ * synchronising; after receiving, tokens are reorganised into the layout the
+ * expert kernels need.  EFA "Dağıtım ve Birleştirme": the receiver computes
+ * the offsets once all counts are known].
+ *
+ * Private region of (expert e, source rank r): rows
+ * [(e*R + r)*max_m, (e*R + r + 1)*max_m).  A slot's position p in it is the
+ * number of earlier slots (smaller flat index) of the same source rank
+ * routed to the same expert; p >= max_m drops the slot (-1,
+ * ORACLE_ERR_CAPACITY).  region_base[e][r] is the row, in the packed layout
+ * of oracle_layout, of the first slot of that region:
+ *   expert_offsets[e] + sum_{r' < r} expert_src_counts[e][r'].
+ * recv_src_private[rows] (rows = E*R*max_m) holds the slot of each private
+ * row, -1 elsewhere.  Masked (-1) and invalid ids as in oracle_layout. */
+int oracle_private_layout(const int32_t *topk_idx, int T, int k, int E, int R,
+                          int max_m, int32_t *private_pos, int32_t *region_base,
+                          int32_t *recv_src_private)
+{
+    if (T < 0 || k < 1 || E < 1 || R < 1 || E % R != 0 || (T > 0 && T % R != 0) ||
+        max_m < 1)
+        return ORACLE_ERR_INVALID;
+    const int Tr = (T > 0) ? T / R : 1;
+    int status = ORACLE_OK;
+    int32_t *src = (int32_t *)calloc((size_t)E * R, sizeof(int32_t));
+    int32_t *seen = (int32_t *)calloc((size_t)E * R, sizeof(int32_t));
+    if (!src || !seen) {
+        free(src);
+        free(seen);
+        return ORACLE_ERR_INVALID;
+    }
+    for (int64_t i = 0; i < (int64_t)T * k; ++i) {
+        int32_t e = topk_idx[i];
+        if (e >= 0 && e < E)
+            src[(size_t)e * R + (i / k) / Tr] += 1;
+    }
+    /* packed offsets, then the base of each (expert, rank) region in them */
+    int32_t run = 0;
+    for (int e = 0; e < E; ++e)
+        for (int r = 0; r < R; ++r) {
+            region_base[(size_t)e * R + r] = run;
+            run += src[(size_t)e * R + r];
+        }
+    const int64_t rows = (int64_t)E * R * max_m;
+    for (int64_t x = 0; x < rows; ++x)
+        recv_src_private[x] = -1;
+    for (int64_t i = 0; i < (int64_t)T * k; ++i) {
+        int32_t e = topk_idx[i];
+        if (e < 0 || e >= E) {
+            if (e != -1)
+                status = ORACLE_ERR_INVALID;
+            private_pos[i] = -1;
+            continue;
+        }
+        int r = (int)((i / k) / Tr);
+        int32_t p = seen[(size_t)e * R + r]++;
+        if (p >= max_m) {
+            private_pos[i] = -1;
+            if (status == ORACLE_OK)
+                status = ORACLE_ERR_CAPACITY;
+            continue;
+        }
+        int64_t row = ((int64_t)e * R + r) * max_m + p;
+        private_pos[i] = (int32_t)row;
+        recv_src_private[row] = (int32_t)i;
+    }
+    free(src);
+    free(seen);
+    return status;
+}
+
 /* ------------------------------------------------------------------------ */
 /* Dispatch [EFA "Dağıtım ve Birleştirme"; EPMC "Despacho"; DSV3 1x128]      */
 /* ------------------------------------------------------------------------ */

@@ -122,3 +122,31 @@ def test_valid_call_without_a_device_reports_cuda_error(moe):
     # arguments pass validation; the launch fails (no device) and is reported
     st = moe.lib.moe_route_topk(A4, 4, 8, 2, 0, A4, A4, None)
     assert st == moe.MOE_ERR_CUDA
+
+
+def test_dispatch_fp8_ex_rejects_bad_scale_layouts(moe):
+    f = moe.lib.moe_dispatch_fp8_ex
+    C = moe.MOE_SCALE_COL_MAJOR
+    assert f(A16, 4, 256, 2, A4, A16, A16, 8, 7, 8, None, None) == moe.MOE_ERR_INVALID_ARG  # layout
+    assert f(A16, 4, 256, 2, A4, A16, A16, 8, C, 6, None, None) == moe.MOE_ERR_INVALID_ARG  # ld < rows
+    assert f(A16, 4, 256, 2, A4, A16, A16, 8, C, 10, None, None) == moe.MOE_ERR_INVALID_ARG  # ld % 4
+    assert f(A16, 4, 256, 2, A4, A16, A4, 8, C, 8, None, None) == moe.MOE_ERR_INVALID_ARG  # align 16
+    assert f(A16, 4, 200, 2, A4, A16, A16, 8, C, 8, None, None) == moe.MOE_ERR_UNSUPPORTED
+    assert f(None, 0, 256, 2, None, None, None, 0, C, 0, None, None) == moe.MOE_OK
+
+
+def test_two_phase_entries_reject_bad_arguments(moe):
+    f = moe.lib.moe_dispatch_layout_private
+    ws = moe.moe_layout_workspace_bytes(8, 2, 4, 2)
+    args = lambda max_m=2, rows=16, wsb=ws: (A4, 8, 2, 4, 2, max_m, rows, A4, A4, A4, A4, A4, A4, A4,
+                                             A16 * 16, wsb, None, None)
+    assert f(*args(max_m=0)) == moe.MOE_ERR_INVALID_ARG
+    assert f(*args(rows=15)) == moe.MOE_ERR_INVALID_ARG
+    assert f(*args(max_m=1 << 28)) == moe.MOE_ERR_INVALID_ARG     # E*R*max_m >= 2^31
+    assert f(*args(wsb=ws - 4)) == moe.MOE_ERR_WORKSPACE
+    c8, c16 = moe.lib.moe_compact_fp8, moe.lib.moe_compact_bf16
+    assert c8(A16, A4, 8, A4, A4, 4, 200, 2, A16, A4, 8, None, None) == moe.MOE_ERR_UNSUPPORTED
+    assert c8(A16, A4, -1, A4, A4, 4, 256, 2, A16, A4, 8, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert c8(A16 + 4, A4, 8, A4, A4, 4, 256, 2, A16, A4, 8, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert c16(A16, 8, None, A4, 4, 256, 2, A16, 8, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert c16(None, 0, None, None, 0, 256, 2, None, 0, None, None) == moe.MOE_OK

@@ -327,3 +327,101 @@ def test_whole_path_in_a_cuda_graph_replayed_on_new_inputs(moe, name):
         for key in want:
             assert torch.equal(got[key], want[key]), (name, seed, key)
     del g
+
+
+# ------------------------------------------- column-major scales (grouped GEMM)
+
+@pytest.mark.parametrize("name", ["dsv3", "prefill"])
+def test_dispatch_fp8_column_major_scales(moe, name):
+    """Same codes as moe_dispatch_fp8; scale (row r, block b) at
+    recv_scale[b * ld + r], ld = rows rounded up to 4; entries of unfilled
+    rows and the padding columns stay untouched."""
+    wl = workload(name)
+    cfg = wl["cfg"]
+    rows = wl["rows"]
+    S = cfg.H // 128
+    ld = (rows + 3) // 4 * 4 + (4 if name == "prefill" else 0)
+    pos = to_dev(wl["layout"]["dispatch_pos"])
+    sbuf = torch.full((S * ld + 64,), -2.0, dtype=torch.float32, device="cuda")
+    st = _status()
+    q, sc = moe.moe_dispatch_fp8_ex(to_dev(wl["x"]), pos, rows, moe.MOE_SCALE_COL_MAJOR, ld,
+                                    recv_scale=sbuf[:S * ld], dev_status=st)
+    q_ref, s_ref = moe.moe_dispatch_fp8(to_dev(wl["x"]), pos, rows)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    filled = torch.from_numpy(wl["layout"]["recv_src"] >= 0).cuda()
+    assert torch.equal(q[filled], q_ref[filled])
+    colmaj = sbuf[:S * ld].view(S, ld)
+    assert torch.equal(colmaj[:, :rows].t()[filled], s_ref[filled])
+    assert torch.all(colmaj[:, rows:] == -2.0)
+    assert torch.all(colmaj[:, :rows].t()[~filled] == -2.0)
+    assert torch.all(sbuf[S * ld:] == -2.0)
+    if name == "dsv3":   # against the oracle too (transposed)
+        _, want_s = oracle.dispatch_fp8(wl["x_bits"], wl["layout"]["dispatch_pos"], rows)
+        assert np.array_equal(colmaj[:, :rows].t().contiguous().cpu().numpy().view(np.uint32),
+                              want_s.view(np.uint32))
+
+
+# ------------------------------------------ two-phase dispatch (private regions)
+
+@pytest.mark.parametrize("name", ["dsv3", "kimi", "dsv3_shared"])
+def test_private_layout_parity(moe, name):
+    wl = workload(name)
+    cfg = wl["cfg"]
+    E, R, max_m = wl["E_lay"], cfg.R, cfg.T_r
+    st = _status()
+    lay = moe.moe_dispatch_layout_private(to_dev(wl["idx"]), E, R, max_m, dev_status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    want = oracle.layout(wl["idx"], E, R)
+    for key in LAYOUT_KEYS:
+        assert np.array_equal(lay[key].cpu().numpy(), want[key].reshape(lay[key].shape)), key
+    ppos, _, _, st_o = oracle.private_layout(wl["idx"], E, R, max_m)
+    assert st_o == oracle.OK
+    assert np.array_equal(lay["private_pos"].cpu().numpy(), ppos)
+
+
+def test_private_layout_drops_beyond_max_m(moe):
+    wl = workload("kimi")                       # skewed routing: hot (expert, rank) regions
+    cfg = wl["cfg"]
+    E, R, max_m = cfg.E, cfg.R, 3
+    st = _status()
+    lay = moe.moe_dispatch_layout_private(to_dev(wl["idx"]), E, R, max_m, dev_status=st)
+    torch.cuda.synchronize()
+    ppos, _, _, st_o = oracle.private_layout(wl["idx"], E, R, max_m)
+    assert st_o == oracle.ERR_CAPACITY and st.item() == moe.MOE_ERR_CAPACITY
+    assert np.array_equal(lay["private_pos"].cpu().numpy(), ppos)
+    packed = wl["layout"]
+    want_pos = np.where(ppos >= 0, packed["dispatch_pos"], -1)
+    want_src = packed["recv_src"].copy()
+    want_src[packed["dispatch_pos"][ppos < 0]] = -1          # holes left by dropped slots
+    assert np.array_equal(lay["dispatch_pos"].cpu().numpy(), want_pos)
+    assert np.array_equal(lay["recv_src"].cpu().numpy(), want_src)
+    assert np.array_equal(lay["expert_counts"].cpu().numpy(), packed["expert_counts"])
+
+
+@pytest.mark.parametrize("name", ["dsv3", "mixtral"])
+def test_two_phase_dispatch_equals_direct(moe, name):
+    """send into private regions, then compact: the packed buffers equal the
+    direct dispatch byte for byte."""
+    wl = workload(name)
+    cfg = wl["cfg"]
+    E, R, max_m, rows = cfg.E, cfg.R, cfg.T_r, wl["rows"]
+    x = to_dev(wl["x"])
+    st = _status()
+    lay = moe.moe_dispatch_layout_private(to_dev(wl["idx"]), E, R, max_m, dev_status=st)
+    prows = lay["private_rows"]
+    if cfg.dispatch == "fp8":
+        pq, ps = moe.moe_dispatch_fp8(x, lay["private_pos"], prows, dev_status=st)
+        q, s = moe.moe_compact_fp8(pq, ps, lay["private_pos"], lay["dispatch_pos"], rows,
+                                   dev_status=st)
+        q_ref, s_ref = moe.moe_dispatch_fp8(x, lay["dispatch_pos"], rows)
+        torch.cuda.synchronize()
+        assert torch.equal(q, q_ref) and torch.equal(s, s_ref)
+    else:
+        px = moe.moe_dispatch_bf16(x, lay["private_pos"], prows, dev_status=st)
+        rx = moe.moe_compact_bf16(px, lay["private_pos"], lay["dispatch_pos"], rows, dev_status=st)
+        rx_ref = moe.moe_dispatch_bf16(x, lay["dispatch_pos"], rows)
+        torch.cuda.synchronize()
+        assert torch.equal(rx.view(torch.int16), rx_ref.view(torch.int16))
+    assert st.item() == 0

@@ -136,3 +136,37 @@ def test_layout_masked_slots_and_empty(oracle_mod):
     assert empty["status"] == oracle_mod.OK
     assert empty["expert_counts"].tolist() == [0] * 8
     assert empty["expert_offsets"].tolist() == [0] * 9
+
+
+# ------------------------------------------------- two-phase (private regions)
+
+@pytest.mark.parametrize("case", load_golden("private_layout_hand.json")["cases"],
+                         ids=lambda c: f"max_m{c['max_m']}")
+def test_private_layout_hand_cases(oracle_mod, case):
+    fx = load_golden("private_layout_hand.json")
+    idx = np.array(fx["topk_idx"], np.int32)
+    pos, base, src, st = oracle_mod.private_layout(idx, fx["E"], fx["R"], case["max_m"])
+    assert st == case["status"]
+    assert pos.tolist() == case["private_pos"]
+    assert base.tolist() == fx["region_base"]
+    kept = pos.ravel() >= 0
+    assert np.array_equal(src[pos.ravel()[kept]], np.nonzero(kept)[0])
+    assert np.sum(src >= 0) == kept.sum()
+
+
+@pytest.mark.parametrize("name", ["tiny", "dsv3", "kimi"])
+def test_private_layout_reproduces_packed_rows(oracle_mod, name):
+    """region_base[e][r] + (position in the private region) is the slot's
+    packed row: compacting the private regions gives the direct layout."""
+    cfg = inputs.CONFIGS[name]
+    idx, _ = oracle_mod.route(inputs.make_logits(cfg).numpy(), cfg.k)
+    packed = oracle_mod.layout(idx, cfg.E, cfg.R)
+    pos, base, src, st = oracle_mod.private_layout(idx, cfg.E, cfg.R, cfg.T_r)
+    assert st == oracle_mod.OK
+    max_m = cfg.T_r
+    region = pos // max_m
+    p = pos - region * max_m
+    assert np.array_equal(base.ravel()[region] + p, packed["dispatch_pos"])
+    # regions are (expert, source rank) pairs
+    ranks = (np.arange(cfg.T) // cfg.T_r)[:, None]
+    assert np.array_equal(region, idx * cfg.R + ranks)
