@@ -345,6 +345,8 @@ def run_ours(args) -> None:
             del probe
         rows = T * k if cap == 0 else E_lay * cap
         lay = moe.moe_dispatch_layout(idx, E_lay, R, capacity=cap, rows=rows, workspace=ws)
+        if args.fused and (args.two_phase or cfg.n_shared):
+            raise SystemExit("--fused runs the plain route on the direct layout")
         if args.two_phase:
             if cap:
                 raise SystemExit("--two-phase needs a packed-layout workload")
@@ -409,13 +411,23 @@ def run_ours(args) -> None:
                                          prows, None, sp)),
                 (lib.moe_compact_bf16, (priv_x.data_ptr(), prows, ppos.data_ptr(), pos.data_ptr(),
                                         T, H, k, recv_x.data_ptr(), rows, None, sp))]
-    calls = [route_call, layout_call, *dispatch_calls,
-             (lib.moe_combine_bf16, (y.data_ptr(), pos.data_ptr(), w.data_ptr(), T, H, k, rows,
-                                     out.data_ptr(), None, sp))]
-    n_dispatch_calls = len(dispatch_calls)
-
-    # stage j ends after these call indices: route, layout, dispatch (1 or 2 calls)
-    stage_end = [0, 1, 1 + n_dispatch_calls]
+    combine_call = (lib.moe_combine_bf16, (y.data_ptr(), pos.data_ptr(), w.data_ptr(), T, H, k,
+                                           rows, out.data_ptr(), None, sp))
+    if args.fused:
+        # route + layout + dispatch in one cooperative launch, then combine
+        fws_buf = moe.Workspace(dev).get(moe.moe_route_dispatch_workspace_bytes(T, k, E, R))
+        head = (logits.data_ptr(), T, E, k, 0, R, cap, x.data_ptr(), H, idx.data_ptr(),
+                w.data_ptr(), *lay_args[7:])
+        tail = (rows, fws_buf.data_ptr(), fws_buf.numel(), None, sp)
+        fused_call = ((lib.moe_route_dispatch_fp8, head + (recv_q.data_ptr(), recv_scale.data_ptr())
+                       + tail) if cfg.dispatch == "fp8" else
+                      (lib.moe_route_dispatch_bf16, head + (recv_x.data_ptr(),) + tail))
+        calls = [fused_call, combine_call]
+        stage_end = [0, 0, 0]      # route, layout and dispatch all end with the fused call
+    else:
+        calls = [route_call, layout_call, *dispatch_calls, combine_call]
+        # stage j ends after these call indices: route, layout, dispatch (1 or 2 calls)
+        stage_end = [0, 1, 1 + len(dispatch_calls)]
 
     def step(ev=None):
         """One pass of the path; with `ev`, events ev[1..3] mark the stage ends."""
@@ -423,8 +435,10 @@ def run_ours(args) -> None:
             rc = fn(*a)
             if rc != 0:
                 raise moe.MoeError(rc, fn.__name__)
-            if ev is not None and j in stage_end:
-                ev[stage_end.index(j) + 1].record(s)
+            if ev is not None:
+                for q, end in enumerate(stage_end):
+                    if end == j:
+                        ev[q + 1].record(s)
 
     nb = algorithmic_bytes(cfg, rows, kept)
     K, W = args.steps, args.warmup
@@ -536,6 +550,9 @@ def run_ours(args) -> None:
         gs = []
         bounds = [0, *[j + 1 for j in stage_end], len(calls)]
         for j in range(4):
+            if bounds[j] == bounds[j + 1]:
+                gs.append(None)   # a stage merged into the previous call
+                continue
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=s):
                 for fn, a in calls[bounds[j]:bounds[j + 1]]:
@@ -548,7 +565,8 @@ def run_ours(args) -> None:
                 e = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
                 e[0].record(s)
                 for j, g in enumerate(gs):
-                    g.replay()
+                    if g is not None:
+                        g.replay()
                     e[j + 1].record(s)
                 rows_ms.append(e)
             s.synchronize()
@@ -557,8 +575,10 @@ def run_ours(args) -> None:
         del gs
     # dispatch+combine as the pages count it (layout + dispatch + combine,
     # route excluded): its own graphs, timed the same way
+    dc_calls = calls if args.fused else calls[1:]   # fused: the route cannot be left out
+
     def dc_step():
-        for fn, a in calls[1:]:
+        for fn, a in dc_calls:
             rc = fn(*a)
             if rc != 0:
                 raise moe.MoeError(rc, fn.__name__)
@@ -602,6 +622,22 @@ def run_ours(args) -> None:
     dc_ms = ms_dc
     dc_bytes = nb["layout"] + nb["dispatch"] + nb["combine"]
 
+    if args.fused:
+        pipeline = ("fused: route + layout + dispatch in one cooperative launch "
+                    "(moe_route_dispatch), then combine")
+        stages = {"route+layout+dispatch": (ms_route + ms_layout + ms_dispatch) * 1e3,
+                  "combine": ms_combine * 1e3}
+        dc_how = ("CUDA graphs of the fused route+layout+dispatch launch + combine (the route "
+                  "is inside the fused launch, so it is included), K steps timed like the step")
+        launches = 2 * K
+    else:
+        pipeline = ("two-phase: private-region layout, send into E*R private regions of T_r "
+                    "rows, receiver compaction" if args.two_phase
+                    else "direct scatter into the packed rows")
+        stages = {"route": ms_route * 1e3, "layout": ms_layout * 1e3,
+                  "dispatch": ms_dispatch * 1e3, "combine": ms_combine * 1e3}
+        dc_how = "CUDA graphs of layout + dispatch + combine, K steps timed like the step"
+        launches = (KERNELS_PER_STEP + (1 if args.two_phase else 0)) * K
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": n_gpus, "steps": K,
@@ -610,15 +646,12 @@ def run_ours(args) -> None:
             "config": {"workload": cfg.describe(), "parallelism": f"replicas x{n_gpus}",
                        "l2": l2_mode,
                        "capacity": cap, "rows": rows,
-                       "pipeline": ("two-phase: private-region layout, send into E*R private "
-                                    "regions of T_r rows, receiver compaction" if args.two_phase
-                                    else "direct scatter into the packed rows"), "timing": (f"CUDA events around K steps run as replays of CUDA graphs of "
+                       "pipeline": pipeline, "timing": (f"CUDA events around K steps run as replays of CUDA graphs of "
                                   f"{G} consecutive step(s)")},
             "us_per_layer": ms_step * 1e3,
-            "stages_us": {"route": ms_route * 1e3, "layout": ms_layout * 1e3,
-                          "dispatch": ms_dispatch * 1e3, "combine": ms_combine * 1e3},
+            "stages_us": stages,
             "dispatch_combine": {"us": dc_ms * 1e3, "bytes": dc_bytes,
-                                 "how": "CUDA graphs of layout + dispatch + combine, K steps timed like the step",
+                                 "how": dc_how,
                                  "gbs": dc_bytes / (dc_ms * 1e-3) / 1e9,
                                  "frac_of_8tbs": dc_bytes / (dc_ms * 1e-3) / 1e9 / SPEC_HBM_GBS,
                                  "frac_of_measured": dc_bytes / (dc_ms * 1e-3) / 1e9 / peak},
@@ -633,7 +666,7 @@ def run_ours(args) -> None:
             "e2e": {"value": n_gpus * nb["step"] / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
                     "us_per_step": e2e_ms * 1e3, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
-            "gpu_launches": (KERNELS_PER_STEP + (1 if args.two_phase else 0)) * K,
+            "gpu_launches": launches,
             "clocks": clocks,
         }
         if world == 1 and not args.no_cpu_baseline:
@@ -655,6 +688,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--two-phase", action="store_true",
                     help="dispatch as the pages' two-phase form (private regions + compaction)")
+    ap.add_argument("--fused", action="store_true",
+                    help="route + layout + dispatch as one cooperative launch, then combine")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -22,7 +22,8 @@ __all__ = [
     "moe_dispatch_layout", "moe_dispatch_bf16", "moe_dispatch_fp8", "moe_combine_bf16",
     "moe_quantize_e4m3", "moe_dispatch_layout_noalloc", "moe_dispatch_fp8_ex", "Workspace",
     "LIB_PATH", "MOE_SCALE_ROW_MAJOR", "MOE_SCALE_COL_MAJOR", "moe_dispatch_layout_private",
-    "moe_compact_fp8", "moe_compact_bf16",
+    "moe_compact_fp8", "moe_compact_bf16", "moe_route_dispatch_workspace_bytes",
+    "moe_route_dispatch_fp8", "moe_route_dispatch_bf16",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_route.so")
@@ -67,6 +68,14 @@ lib.moe_dispatch_fp8_ex.argtypes = [_P, _i32, _i32, _i32, _P, _P, _P, _i64, _i32
 lib.moe_dispatch_fp8_ex.restype = _i32
 lib.moe_combine_bf16.argtypes = [_P, _P, _P, _i32, _i32, _i32, _i64, _P, _P, _P]
 lib.moe_combine_bf16.restype = _i32
+lib.moe_route_dispatch_workspace_bytes.argtypes = [_i32, _i32, _i32, _i32]
+lib.moe_route_dispatch_workspace_bytes.restype = _sz
+lib.moe_route_dispatch_fp8.argtypes = [_P, _i32, _i32, _i32, _i32, _i32, _i32, _P, _i32, _P, _P,
+                                       _P, _P, _P, _P, _P, _P, _P, _P, _i64, _P, _sz, _P, _P]
+lib.moe_route_dispatch_fp8.restype = _i32
+lib.moe_route_dispatch_bf16.argtypes = [_P, _i32, _i32, _i32, _i32, _i32, _i32, _P, _i32, _P, _P,
+                                        _P, _P, _P, _P, _P, _P, _P, _i64, _P, _sz, _P, _P]
+lib.moe_route_dispatch_bf16.restype = _i32
 lib.moe_quantize_e4m3.argtypes = [_P, _i64, _P, _P]
 lib.moe_quantize_e4m3.restype = _i32
 
@@ -392,6 +401,87 @@ def moe_combine_bf16(y: torch.Tensor, dispatch_pos: torch.Tensor, topk_w: torch.
     _check(lib.moe_combine_bf16(_ptr(y), _ptr(dispatch_pos), _ptr(topk_w), T, H, k, rows,
                                 _ptr(out), _ptr(dev_status), _stream(stream)), "moe_combine_bf16")
     return out
+
+
+def moe_route_dispatch_workspace_bytes(T: int, k: int, E: int, R: int) -> int:
+    return int(lib.moe_route_dispatch_workspace_bytes(T, k, E, R))
+
+
+# The fused entry keeps its grid barrier in the first 256 bytes of its
+# workspace (zero before first use, left ready by every completed call), so it
+# gets workspaces of its own, never shared with the layout's.
+_default_fused_ws: dict[torch.device, Workspace] = {}
+
+
+def _route_dispatch(fp8: bool, logits, x, k, R, capacity, rows, renormalize, out, workspace,
+                    dev_status, stream) -> dict:
+    assert logits.dtype == torch.float32 and logits.dim() == 2
+    x = _bits16(x)
+    T, E = logits.shape
+    H = x.shape[1]
+    assert x.shape[0] == T
+    dev = logits.device
+    if rows is None:
+        rows = T * k if capacity == 0 else E * capacity
+    if out is None:
+        out = dict(
+            topk_idx=torch.empty(T, k, dtype=torch.int32, device=dev),
+            topk_w=torch.empty(T, k, dtype=torch.float32, device=dev),
+            expert_counts=torch.empty(E, dtype=torch.int32, device=dev),
+            expert_src_counts=torch.empty(E, R, dtype=torch.int32, device=dev),
+            rank_counts=torch.empty(R, dtype=torch.int32, device=dev),
+            expert_offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
+            dispatch_pos=torch.empty(T, k, dtype=torch.int32, device=dev),
+            recv_src=torch.empty(max(rows, 1), dtype=torch.int32, device=dev),
+        )
+        if fp8:
+            out["recv_q"] = torch.empty(max(rows, 1), H, dtype=torch.uint8, device=dev)
+            out["recv_scale"] = torch.empty(max(rows, 1), H // 128, dtype=torch.float32,
+                                            device=dev)
+        else:
+            out["recv_x"] = torch.empty(max(rows, 1), H, dtype=x.dtype, device=dev)
+    if workspace is None:
+        workspace = _default_fused_ws.setdefault(dev, Workspace(dev))
+    nbytes = moe_route_dispatch_workspace_bytes(T, k, E, R)
+    if nbytes == 0:
+        raise MoeError(MOE_ERR_INVALID_ARG, "moe_route_dispatch_workspace_bytes")
+    ws = workspace.get(nbytes)
+    common = (_ptr(logits), T, E, k, int(renormalize), R, capacity, _ptr(x), H,
+              _ptr(out["topk_idx"]), _ptr(out["topk_w"]), _ptr(out["expert_counts"]),
+              _ptr(out["expert_src_counts"]), _ptr(out["rank_counts"]),
+              _ptr(out["expert_offsets"]), _ptr(out["dispatch_pos"]), _ptr(out["recv_src"]))
+    if fp8:
+        _check(lib.moe_route_dispatch_fp8(*common, _ptr(out["recv_q"]), _ptr(out["recv_scale"]),
+                                          rows, _ptr(ws), ws.numel(), _ptr(dev_status),
+                                          _stream(stream)), "moe_route_dispatch_fp8")
+    else:
+        _check(lib.moe_route_dispatch_bf16(*common, _ptr(out["recv_x"]), rows, _ptr(ws),
+                                           ws.numel(), _ptr(dev_status), _stream(stream)),
+               "moe_route_dispatch_bf16")
+    out["rows"] = rows
+    return out
+
+
+def moe_route_dispatch_fp8(logits: torch.Tensor, x: torch.Tensor, k: int, R: int,
+                           capacity: int = 0, rows: int | None = None, renormalize: bool = False,
+                           out: dict | None = None, workspace: Workspace | None = None,
+                           dev_status: torch.Tensor | None = None, stream=None) -> dict:
+    """Route + layout + FP8 dispatch in one cooperative launch.  Returns a dict
+    with topk_idx, topk_w, the layout arrays of moe_dispatch_layout, recv_q
+    [rows][H] uint8 and recv_scale [rows][H/128] fp32, and ``rows``.  A given
+    ``workspace`` must be used by this entry (and _bf16) only."""
+    return _route_dispatch(True, logits, x, k, R, capacity, rows, renormalize, out, workspace,
+                           dev_status, stream)
+
+
+def moe_route_dispatch_bf16(logits: torch.Tensor, x: torch.Tensor, k: int, R: int,
+                            capacity: int = 0, rows: int | None = None, renormalize: bool = False,
+                            out: dict | None = None, workspace: Workspace | None = None,
+                            dev_status: torch.Tensor | None = None, stream=None) -> dict:
+    """Route + layout + bf16 dispatch in one cooperative launch (see
+    moe_route_dispatch_fp8); the rows are returned as recv_x [rows][H]."""
+    return _route_dispatch(False, logits, x, k, R, capacity, rows, renormalize, out, workspace,
+                           dev_status, stream)
 
 
 def moe_quantize_e4m3(v: torch.Tensor, q: torch.Tensor | None = None, stream=None) -> torch.Tensor:

@@ -279,6 +279,84 @@ int moe_combine_bf16(const uint16_t *y, const int32_t *dispatch_pos, const float
                                       as_stream(stream)));
 }
 
+size_t moe_route_dispatch_workspace_bytes(int T, int k, int E, int R)
+{
+    if (!valid_layout_sizes(T, k, E, R))
+        return 0;
+    const size_t a = moe::route_dispatch_workspace_bytes(T, k, E, R, true);
+    const size_t b = moe::route_dispatch_workspace_bytes(T, k, E, R, false);
+    return (a == 0 || b == 0) ? 0 : (a > b ? a : b);
+}
+
+static int route_dispatch_common(const float *logits, int T, int E, int k, int renormalize, int R,
+                                 int capacity, const uint16_t *x, int H, bool fp8,
+                                 int32_t *topk_idx, float *topk_w, int32_t *expert_counts,
+                                 int32_t *expert_src_counts, int32_t *rank_counts,
+                                 int32_t *expert_offsets, int32_t *dispatch_pos,
+                                 int32_t *recv_src, void *recv, float *recv_scale, int64_t rows,
+                                 void *workspace, size_t ws_bytes, int32_t *dev_status,
+                                 void *stream)
+{
+    if (!valid_layout_sizes(T, k, E, R) || capacity < 0 || rows < 0 || rows >= kMaxIndex ||
+        H < 8 || H % 8 != 0 || H > (1 << 20) || static_cast<int64_t>(T) * H > (int64_t(1) << 40))
+        return MOE_ERR_INVALID_ARG;
+    if ((fp8 && H % 128 != 0) || (!fp8 && H < 64))
+        return MOE_ERR_UNSUPPORTED;
+    const int64_t needed = (capacity == 0) ? static_cast<int64_t>(T) * k
+                                           : static_cast<int64_t>(E) * capacity;
+    if (rows < needed)
+        return MOE_ERR_INVALID_ARG;
+    const void *arrays[] = {expert_counts, expert_src_counts, rank_counts, expert_offsets};
+    for (const void *p : arrays)
+        if (!p || !aligned(p, 4))
+            return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!logits || !x || !topk_idx || !topk_w || !dispatch_pos || !aligned(logits, 4) ||
+                  !aligned(x, 16) || !aligned(topk_idx, 4) || !aligned(topk_w, 4) ||
+                  !aligned(dispatch_pos, 4)))
+        return MOE_ERR_INVALID_ARG;
+    if (rows > 0 && (!recv_src || !recv || !aligned(recv_src, 4) || !aligned(recv, 16) ||
+                     (fp8 && (!recv_scale || !aligned(recv_scale, 4)))))
+        return MOE_ERR_INVALID_ARG;
+    if (dev_status && !aligned(dev_status, 4))
+        return MOE_ERR_INVALID_ARG;
+    if (!workspace || !aligned(workspace, 256))
+        return MOE_ERR_WORKSPACE;
+    bool small = false;
+    const cudaError_t err = moe::route_dispatch(
+        logits, T, E, k, renormalize != 0, R, capacity, x, H, fp8, topk_idx, topk_w, expert_counts,
+        expert_src_counts, rank_counts, expert_offsets, dispatch_pos, recv_src, recv, recv_scale,
+        rows, workspace, ws_bytes, dev_status, as_stream(stream), &small);
+    if (small)
+        return MOE_ERR_WORKSPACE;
+    return launched(err);
+}
+
+int moe_route_dispatch_fp8(const float *logits, int T, int E, int k, int renormalize, int R,
+                           int capacity, const uint16_t *x, int H, int32_t *topk_idx,
+                           float *topk_w, int32_t *expert_counts, int32_t *expert_src_counts,
+                           int32_t *rank_counts, int32_t *expert_offsets, int32_t *dispatch_pos,
+                           int32_t *recv_src, uint8_t *recv_q, float *recv_scale, int64_t rows,
+                           void *workspace, size_t ws_bytes, int32_t *dev_status, void *stream)
+{
+    return route_dispatch_common(logits, T, E, k, renormalize, R, capacity, x, H, true, topk_idx,
+                                 topk_w, expert_counts, expert_src_counts, rank_counts,
+                                 expert_offsets, dispatch_pos, recv_src, recv_q, recv_scale, rows,
+                                 workspace, ws_bytes, dev_status, stream);
+}
+
+int moe_route_dispatch_bf16(const float *logits, int T, int E, int k, int renormalize, int R,
+                            int capacity, const uint16_t *x, int H, int32_t *topk_idx,
+                            float *topk_w, int32_t *expert_counts, int32_t *expert_src_counts,
+                            int32_t *rank_counts, int32_t *expert_offsets, int32_t *dispatch_pos,
+                            int32_t *recv_src, uint16_t *recv_x, int64_t rows, void *workspace,
+                            size_t ws_bytes, int32_t *dev_status, void *stream)
+{
+    return route_dispatch_common(logits, T, E, k, renormalize, R, capacity, x, H, false, topk_idx,
+                                 topk_w, expert_counts, expert_src_counts, rank_counts,
+                                 expert_offsets, dispatch_pos, recv_src, recv_x, nullptr, rows,
+                                 workspace, ws_bytes, dev_status, stream);
+}
+
 int moe_quantize_e4m3(const float *v, int64_t n, uint8_t *q, void *stream)
 {
     if (n < 0)

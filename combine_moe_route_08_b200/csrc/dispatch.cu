@@ -12,6 +12,7 @@
 // quantised once, and written k times with 16-byte streaming stores, each
 // destination row by the whole CTA in one coalesced sweep.
 #include "common.cuh"
+#include "dispatch_dev.cuh"
 #include "kernels.cuh"
 
 namespace moe {
@@ -58,10 +59,7 @@ __global__ void __launch_bounds__(kMaxThreads)
     pdl_trigger();
 }
 
-// Thread t of the token owns channels [16t, 16t + 16); the 8 threads of one
-// 128-channel block are 8 consecutive lanes, so the block's amax is a 3-step
-// xor shuffle.  s = amax / 448 and every x / s are IEEE binary32 divisions
-// (__fdiv_rn), then the hardware converts to e4m3 with RNE + saturation.
+// Thread t of the token owns channels [16t, 16t + 16) (quant_e4m3_x16).
 // Scales go to recv_scale[r * S + b] (row-major) or, with scale_ld > 0, to
 // recv_scale[b * scale_ld + r] (column-major: each 128-channel block's scales
 // contiguous over the rows, the operand layout of a grouped FP8 GEMM).
@@ -86,30 +84,8 @@ __global__ void __launch_bounds__(kMaxThreads)
             a = ld_stream_v4(xr + 2 * t);
             b = ld_stream_v4(xr + 2 * t + 1);
         }
-        const uint32_t wds[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-        float f[16];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            f[2 * i] = bf16_lo(wds[i]);
-            f[2 * i + 1] = bf16_hi(wds[i]);
-        }
-        float amax = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-            amax = fmaxf(amax, fabsf(f[i]));
-        amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 1));
-        amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 2));
-        amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 4));
-        const float s = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 448.0f);
-
-        uint32_t c[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const uint32_t lo = e4m3x2(__fdiv_rn(f[4 * i], s), __fdiv_rn(f[4 * i + 1], s));
-            const uint32_t hi = e4m3x2(__fdiv_rn(f[4 * i + 2], s), __fdiv_rn(f[4 * i + 3], s));
-            c[i] = lo | (hi << 16);
-        }
-        const uint4 q = make_uint4(c[0], c[1], c[2], c[3]);
+        float s;
+        const uint4 q = quant_e4m3_x16(a, b, s);
         if (act) {
             for (int j = 0; j < k; ++j) {
                 const int r = srow[j];

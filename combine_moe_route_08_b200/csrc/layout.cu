@@ -34,14 +34,13 @@
 // The kernel boundary between the two is the only grid-wide ordering; nothing
 // waits on another CTA.
 //
-// The equality mask of a warp step ("which lanes hold my expert") is built
-// from one __ballot_sync per key bit; __match_any_sync would give the same
-// mask but costs about 2000 cycles per call on this part (measured with
-// clock64 stamps), which dominated the kernel.
+// The warp-level pieces (equality masks, per-warp histograms and bases, the
+// block scan) are in layout_dev.cuh.
 #include <algorithm>
 
 #include "common.cuh"
 #include "kernels.cuh"
+#include "layout_dev.cuh"
 
 namespace moe {
 
@@ -74,13 +73,6 @@ __device__ __forceinline__ void warp_run(const LayoutGeom &G, int c, int64_t &w0
     w1 = min(w0 + seg, i1);
 }
 
-__device__ __forceinline__ unsigned lanemask_lt()
-{
-    unsigned m;
-    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
-    return m;
-}
-
 // The lane's slots of its warp run, loaded in one go (-1 past the end).
 __device__ __forceinline__ void load_run(const int32_t *__restrict__ topk_idx, int64_t w0,
                                          int64_t w1, int (&e)[kMaxSteps])
@@ -91,32 +83,6 @@ __device__ __forceinline__ void load_run(const int32_t *__restrict__ topk_idx, i
         const int64_t i = w0 + 32 * s + lane;
         e[s] = (i < w1) ? __ldg(topk_idx + i) : -1;
     }
-}
-
-// Lanes of the warp holding the same key as this lane.  __match_any_sync is
-// slow on this part (thousands of cycles per call), so the equality mask is
-// built from one ballot per key bit: a lane matches where every bit agrees.
-__device__ __forceinline__ unsigned match_mask(int key, int nbits)
-{
-    unsigned mask = kFullMask;
-    for (int b = 0; b < nbits; ++b) {
-        const bool bit = (key >> b) & 1;
-        const unsigned bal = __ballot_sync(kFullMask, bit);
-        mask &= bit ? bal : ~bal;
-    }
-    return mask;
-}
-
-// Key bits: enough for max(E - 1, 31), plus one bit that marks a slot that
-// is empty, masked or invalid (key = lane | that bit, unique in the warp).
-__device__ __forceinline__ int key_bits(int E)
-{
-    return 32 - __clz(max(E - 1, 31)) + 1;
-}
-
-__device__ __forceinline__ int match_key(int e, int E, int lane, int nbits)
-{
-    return (static_cast<unsigned>(e) < static_cast<unsigned>(E)) ? e : (lane | (1 << (nbits - 1)));
 }
 
 __global__ void __launch_bounds__(kThreads)
@@ -153,43 +119,6 @@ __global__ void __launch_bounds__(kThreads)
     for (int x = threadIdx.x; x < E; x += kThreads)
         ws_hist[static_cast<size_t>(c) * E + x] = h[x];
     pdl_trigger();
-}
-
-// In-place exclusive scan of a[0..n) (n <= kThreads) by the whole CTA; a[n]
-// receives the total.  `tot` is kWarps + 1 ints of shared scratch.
-__device__ void block_exclusive_scan(int32_t *a, int n, int32_t *tot)
-{
-    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-    const int v = (tid < n) ? a[tid] : 0;
-    int incl = v;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        const int t = __shfl_up_sync(kFullMask, incl, off);
-        if (lane >= off)
-            incl += t;
-    }
-    if (lane == 31)
-        tot[w] = incl;
-    __syncthreads();
-    if (w == 0) {
-        const int t = tot[lane];
-        int x = t;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int y = __shfl_up_sync(kFullMask, x, off);
-            if (lane >= off)
-                x += y;
-        }
-        tot[lane] = x - t;  // exclusive over warps
-        if (lane == 31)
-            tot[kWarps] = x;
-    }
-    __syncthreads();
-    if (tid < n)
-        a[tid] = tot[w] + incl - v;
-    if (tid == 0)
-        a[n] = tot[kWarps];
-    __syncthreads();
 }
 
 __global__ void __launch_bounds__(kThreads)
@@ -278,17 +207,8 @@ __global__ void __launch_bounds__(kThreads)
 
     // per-warp histogram of this CTA's slots (warp-private rows: no atomics)
     int32_t *mywh = wh + w * E;
-#pragma unroll
-    for (int s = 0; s < kMaxSteps; ++s) {
-        if (w0 + 32 * s >= w1)
-            break;
-        const bool valid = static_cast<unsigned>(e[s]) < static_cast<unsigned>(E);
-        const unsigned mask = match_mask(match_key(e[s], E, lane, nb), nb);
-        if (valid && lane == __ffs(mask) - 1)
-            mywh[e[s]] += __popc(mask);
-        __syncwarp();
-    }
-    block_exclusive_scan(off, E, tot);  // off[e] = slots of experts < e; off[E] = total
+    warp_histogram(e, w0, w1, E, nb, mywh);
+    block_exclusive_scan<kWarps>(off, E, tot);  // off[e] = slots of experts < e; off[E] = total
 
     if (c == 0) {
         for (int x = threadIdx.x; x <= E; x += kThreads)
@@ -298,15 +218,7 @@ __global__ void __launch_bounds__(kThreads)
             rank_counts[rr] = off[(rr + 1) * L] - off[rr * L];
     }
     // per-warp base of each expert's positions: earlier chunks + earlier warps
-    for (int x = threadIdx.x; x < E; x += kThreads) {
-        int run = chb[x];
-#pragma unroll 8
-        for (int ww = 0; ww < kWarps; ++ww) {
-            const int t = wh[ww * E + x];
-            wh[ww * E + x] = run;
-            run += t;
-        }
-    }
+    warp_bases<kWarps>(wh, chb, E);
     __syncthreads();
 
     // rank every slot among equal experts, in slot order
@@ -317,12 +229,7 @@ __global__ void __launch_bounds__(kThreads)
             break;
         const int64_t i = w0 + 32 * s + lane;
         const bool valid = static_cast<unsigned>(e[s]) < static_cast<unsigned>(E);
-        const unsigned mask = match_mask(match_key(e[s], E, lane, nb), nb);
-        const int p = valid ? mywh[e[s]] + __popc(mask & lanemask_lt()) : 0;
-        __syncwarp();
-        if (valid && lane == __ffs(mask) - 1)
-            mywh[e[s]] += __popc(mask);
-        __syncwarp();
+        const int p = rank_step(e[s], E, nb, mywh);
         if (i < w1) {
             int64_t row = -1, prow = -1;
             bool hole = false;  // private mode: packed row left empty by a dropped slot

@@ -325,6 +325,58 @@ int moe_dispatch_fp8_ex(const uint16_t *x, int T, int H, int k, const int32_t *d
                         int64_t scale_ld, int32_t *dev_status, void *stream);
 
 /*
+ * moe_route_dispatch_fp8 / moe_route_dispatch_bf16 -- moe_route_topk,
+ * moe_dispatch_layout and moe_dispatch_fp8 (or _bf16) in ONE launch.
+ * Follows "Enabling trillion-parameter models on AWS EFA", "Dağıtım ve
+ * Birleştirme" (the dispatch kernel counts the tokens of each expert itself,
+ * by atomic accumulation in shared memory within a block, sums the counts
+ * into offsets and packs the tokens at those offsets) and "Efficient and
+ * portable mixture-of-experts communication", "Despacho" (one routing warp
+ * counts while the others move the tokens).
+ *
+ * Outputs are bit-identical to the three separate calls with the same
+ * arguments (plain route, scales row-major):
+ *   topk_idx, topk_w            as moe_route_topk (logits [T][E] fp32);
+ *   expert_counts .. recv_src   as moe_dispatch_layout (capacity 0 = packed,
+ *                               > 0 = padded [E][capacity]);
+ *   recv_q + recv_scale         as moe_dispatch_fp8 (x [T][H] bf16 bits), or
+ *   recv_x                      as moe_dispatch_bf16.
+ * Extra constraints: H <= 2^20, T*H <= 2^40; bf16 needs H >= 64
+ * (MOE_ERR_UNSUPPORTED otherwise).
+ *
+ * The kernel is a cooperative launch (every CTA resident) with two
+ * grid-wide barriers kept in the workspace:
+ *   workspace   device memory, 256-byte aligned, at least
+ *               moe_route_dispatch_workspace_bytes(T, k, E, R) bytes (a
+ *               value for the CURRENT device: it depends on its SM count).
+ *               It carries state from call to call (a grid barrier, work
+ *               counters, per-rank totals), so it must be ZERO before the
+ *               first call and is then reserved for these two entry
+ *               points; every call that completes leaves it ready for the
+ *               next, whatever the sizes of either.  A wait inside the
+ *               kernel gives up after 1 s and records MOE_ERR_TIMEOUT in
+ *               *dev_status (the outputs are then incomplete); zero the
+ *               workspace again before reusing it.  Calls that share a
+ *               workspace must not overlap on the GPU.
+ * Returns MOE_ERR_WORKSPACE for a missing, misaligned or short workspace,
+ * MOE_ERR_CUDA if the device cannot run the cooperative launch.
+ * T == 0 still launches (counts, offsets and recv_src are written).
+ */
+size_t moe_route_dispatch_workspace_bytes(int T, int k, int E, int R);
+int moe_route_dispatch_fp8(const float *logits, int T, int E, int k, int renormalize, int R,
+                           int capacity, const uint16_t *x, int H, int32_t *topk_idx,
+                           float *topk_w, int32_t *expert_counts, int32_t *expert_src_counts,
+                           int32_t *rank_counts, int32_t *expert_offsets, int32_t *dispatch_pos,
+                           int32_t *recv_src, uint8_t *recv_q, float *recv_scale, int64_t rows,
+                           void *workspace, size_t ws_bytes, int32_t *dev_status, void *stream);
+int moe_route_dispatch_bf16(const float *logits, int T, int E, int k, int renormalize, int R,
+                            int capacity, const uint16_t *x, int H, int32_t *topk_idx,
+                            float *topk_w, int32_t *expert_counts, int32_t *expert_src_counts,
+                            int32_t *rank_counts, int32_t *expert_offsets, int32_t *dispatch_pos,
+                            int32_t *recv_src, uint16_t *recv_x, int64_t rows, void *workspace,
+                            size_t ws_bytes, int32_t *dev_status, void *stream);
+
+/*
  * moe_combine_bf16 -- gather each token's k expert outputs and form the
  * router-weighted sum.
  * Follows "Efficient and portable mixture-of-experts communication",

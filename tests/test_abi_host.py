@@ -150,3 +150,35 @@ def test_two_phase_entries_reject_bad_arguments(moe):
     assert c8(A16 + 4, A4, 8, A4, A4, 4, 256, 2, A16, A4, 8, None, None) == moe.MOE_ERR_INVALID_ARG
     assert c16(A16, 8, None, A4, 4, 256, 2, A16, 8, None, None) == moe.MOE_ERR_INVALID_ARG
     assert c16(None, 0, None, None, 0, 256, 2, None, 0, None, None) == moe.MOE_OK
+
+
+def test_fused_route_dispatch_rejects_bad_arguments(moe):
+    for bad in [(-1, 2, 8, 2), (64, 0, 8, 2), (64, 2, 8, 3), (63, 2, 8, 2)]:
+        assert moe.moe_route_dispatch_workspace_bytes(*bad) == 0, bad
+    f8, f16 = moe.lib.moe_route_dispatch_fp8, moe.lib.moe_route_dispatch_bf16
+    ws = 0x100000  # 256-byte aligned fake address
+
+    def call8(T=64, E=8, k=2, R=2, cap=0, x=A16, H=256, rows=128, wsp=ws, recv_q=A16,
+              scale=A4, logits=A4):
+        return f8(logits, T, E, k, 0, R, cap, x, H, A4, A4, A4, A4, A4, A4, A4, A4, recv_q,
+                  scale, rows, wsp, 1 << 20, None, None)
+
+    assert call8(k=0) == moe.MOE_ERR_INVALID_ARG
+    assert call8(k=9) == moe.MOE_ERR_INVALID_ARG            # k > E
+    assert call8(R=3) == moe.MOE_ERR_INVALID_ARG            # E % R != 0
+    assert call8(T=63) == moe.MOE_ERR_INVALID_ARG           # T % R != 0
+    assert call8(H=204) == moe.MOE_ERR_INVALID_ARG          # H % 8 != 0
+    assert call8(H=264) == moe.MOE_ERR_UNSUPPORTED          # fp8 needs H % 128 == 0
+    assert call8(H=1 << 21) == moe.MOE_ERR_INVALID_ARG      # H > 2^20
+    assert call8(rows=127) == moe.MOE_ERR_INVALID_ARG       # packed rows < T*k
+    assert call8(cap=4, rows=31) == moe.MOE_ERR_INVALID_ARG  # padded rows < E*cap
+    assert call8(x=A16 + 8) == moe.MOE_ERR_INVALID_ARG      # x not 16-byte aligned
+    assert call8(recv_q=A16 + 4) == moe.MOE_ERR_INVALID_ARG
+    assert call8(scale=None) == moe.MOE_ERR_INVALID_ARG
+    assert call8(logits=None) == moe.MOE_ERR_INVALID_ARG
+    assert call8(wsp=None) == moe.MOE_ERR_WORKSPACE
+    assert call8(wsp=ws + 128) == moe.MOE_ERR_WORKSPACE     # not 256-byte aligned
+    assert f16(A4, 64, 8, 2, 0, 2, 0, A16, 204, A4, A4, A4, A4, A4, A4, A4, A4, A16, 128, ws,
+               1 << 20, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert f16(A4, 64, 8, 2, 0, 2, 0, A16, 56, A4, A4, A4, A4, A4, A4, A4, A4, A16, 128, ws,
+               1 << 20, None, None) == moe.MOE_ERR_UNSUPPORTED   # bf16 needs H >= 64
