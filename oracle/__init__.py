@@ -64,6 +64,8 @@ def _load():
         lib.oracle_quantize_tokens.restype = i32
         lib.oracle_combine.argtypes = [P, P, P, i32, i32, i32, i64, P, i32, P, P]
         lib.oracle_combine.restype = i32
+        lib.oracle_combine_fp8.argtypes = [P, P, P, P, i32, i32, i32, i64, P, i32, P, P]
+        lib.oracle_combine_fp8.restype = i32
         lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
         lib.oracle_e4m3_encode.restype = ctypes.c_uint8
         lib.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
@@ -256,6 +258,34 @@ def combine(y_bits: np.ndarray, dispatch_pos: np.ndarray, topk_w: np.ndarray,
                                 _ptr(tok), n, _ptr(acc), _ptr(out))
     if st != OK:
         raise ValueError(f"oracle_combine status {st}")
+    return acc, out
+
+
+def combine_fp8(yq: np.ndarray, ys: np.ndarray, dispatch_pos: np.ndarray, topk_w: np.ndarray,
+                tokens=None):
+    """Combine with E4M3 expert rows: each element restored as decode(q) * s
+    (one binary32 product), then the router-weighted binary32 sum over j
+    ascending.  yq uint8 [rows][H], ys float32 [rows][H/128].  Returns (acc
+    float32 [n][H], out_bits uint16 [n][H])."""
+    yq = _c(yq, np.uint8)
+    rows, H = yq.shape
+    ys = _c(ys, np.float32)
+    assert ys.shape == (rows, H // 128)
+    pos = _c(dispatch_pos, np.int32)
+    T, k = pos.shape
+    w = _c(topk_w, np.float32)
+    assert w.shape == (T, k)
+    if tokens is None:
+        tok, n = None, T
+    else:
+        tok = _c(tokens, np.int32)
+        n = tok.shape[0]
+    acc = np.empty((n, H), np.float32)
+    out = np.empty((n, H), np.uint16)
+    st = _load().oracle_combine_fp8(_ptr(yq), _ptr(ys), _ptr(pos), _ptr(w), T, H, k, rows,
+                                    _ptr(tok), n, _ptr(acc), _ptr(out))
+    if st != OK:
+        raise ValueError(f"oracle_combine_fp8 status {st}")
     return acc, out
 
 

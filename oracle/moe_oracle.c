@@ -630,3 +630,47 @@ int oracle_combine(const uint16_t *y, const int32_t *dispatch_pos,
     }
     return ORACLE_OK;
 }
+
+/*
+ * Combine with an FP8 payload: the expert rows arrive as E4M3 codes with one
+ * binary32 scale per 1x128 block (the dispatch format, DeepSeek-V3
+ * fragments: activations scaled per token per 128 channels).  Each element
+ * is first restored as one binary32 product, v = decode(q) * s (decode is
+ * exact in binary32), then summed as in oracle_combine: acc = acc + w_j * v
+ * over j ascending, one multiply and one add per term, -1 slots skipped.
+ *   yq [rows][H] codes, ys [rows][H/128] scales.
+ */
+int oracle_combine_fp8(const uint8_t *yq, const float *ys, const int32_t *dispatch_pos,
+                       const float *topk_w, int T, int H, int k, int64_t rows,
+                       const int32_t *tokens, int n, float *acc_out, uint16_t *out)
+{
+    if (H % 128 != 0)
+        return ORACLE_ERR_INVALID;
+    int S = H / 128;
+    int count = tokens ? n : T;
+    for (int i = 0; i < count; ++i) {
+        int g = tokens ? tokens[i] : i;
+        if (g < 0 || g >= T)
+            return ORACLE_ERR_INVALID;
+        for (int j = 0; j < k; ++j) {
+            int32_t row = dispatch_pos[(size_t)g * k + j];
+            if (row >= rows)
+                return ORACLE_ERR_INVALID;
+        }
+        for (int h = 0; h < H; ++h) {
+            float acc = 0.0f;
+            for (int j = 0; j < k; ++j) {
+                int32_t row = dispatch_pos[(size_t)g * k + j];
+                if (row < 0)
+                    continue;
+                float v = e4m3_decode(yq[(size_t)row * H + h]) * ys[(size_t)row * S + h / 128];
+                float prod = topk_w[(size_t)g * k + j] * v;
+                acc = acc + prod;
+            }
+            if (acc_out)
+                acc_out[(size_t)i * H + h] = acc;
+            out[(size_t)i * H + h] = float_to_bf16_rne(acc);
+        }
+    }
+    return ORACLE_OK;
+}

@@ -161,3 +161,69 @@ def test_dispatch_identity_combine_returns_weight_scaled_input(oracle_mod, renor
         outf = _f(out).astype(np.float64)
         ulp = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(xf), 2.0 ** -126))) - 7)
         assert np.all(np.abs(outf - xf) <= ulp + cfg.k * 2 ** -23 * np.abs(xf))
+
+
+# ------------------------------------------------------- combine, FP8 payload
+
+def _fp8_case_arrays(case):
+    H, rows = case["H"], case["rows"]
+    yq = np.zeros((rows, H), np.uint8)
+    for r, cols in case["codes"].items():
+        for h, code in cols.items():
+            yq[int(r), int(h)] = code
+    ys = np.array(case["scales"], np.float32)
+    pos = np.array(case["dispatch_pos"], np.int32)
+    w = np.array(case["topk_w"], np.float32)
+    return yq, ys, pos, w
+
+
+@pytest.mark.parametrize("case", load_golden("combine_fp8_hand.json")["cases"],
+                         ids=lambda c: c["name"][:24])
+def test_combine_fp8_hand_cases(oracle_mod, case):
+    yq, ys, pos, w = _fp8_case_arrays(case)
+    acc, out = oracle_mod.combine_fp8(yq, ys, pos, w)
+    want = np.zeros(case["H"], np.float32)
+    for h, v in case["expect_acc"].items():
+        want[int(h)] = v
+    assert np.array_equal(acc[0], want)
+    if "wrong_order_acc" in case:
+        assert acc[0][0] != np.float32(case["wrong_order_acc"])
+    assert np.array_equal(out[0], oracle_mod.float_to_bf16_bits(want))
+
+
+def test_combine_fp8_power_of_two_scales_equal_bf16_combine(oracle_mod):
+    """With power-of-two scales decode(q) * s is exact and representable in
+    bf16, so the FP8-payload combine must equal the pinned bf16 combine of the
+    restored rows, bit for bit."""
+    rng = np.random.default_rng(21)
+    T, k, H, rows = 24, 4, 256, 70
+    yq = rng.integers(0, 256, (rows, H)).astype(np.uint8)
+    yq[(yq & 0x7F) == 0x7F] = 0x11                   # no NaN codes
+    ys = (2.0 ** rng.integers(-8, 8, (rows, H // 128))).astype(np.float32)
+    pos = rng.integers(-1, rows, (T, k)).astype(np.int32)
+    w = rng.random((T, k)).astype(np.float32)
+    restored = oracle_mod.e4m3_decode(yq) * np.repeat(ys, 128, axis=1)
+    y_bits = oracle_mod.float_to_bf16_bits(restored)
+    assert np.array_equal(_f(y_bits), restored)   # exact in bf16
+    acc8, out8 = oracle_mod.combine_fp8(yq, ys, pos, w)
+    acc16, out16 = oracle_mod.combine(y_bits, pos, w)
+    assert np.array_equal(acc8, acc16) and np.array_equal(out8, out16)
+
+
+def test_combine_fp8_of_dispatched_tokens_is_weighted_input(oracle_mod):
+    """dispatch (fp8) -> identity expert -> FP8-payload combine returns
+    sum_j w_j * x within the E4M3 error (half an ulp: 2^-4 relative above the
+    subnormal range, s * 2^-10 below) plus the binary32 rounding of k terms."""
+    T, H, k, E = 40, 256, 3, 8
+    logits, x = inputs.make_random_case(T, H, E, k, seed=23)
+    idx, w = oracle_mod.route(logits.numpy(), k)
+    lay = oracle_mod.layout(idx, E, 2)
+    xb = inputs.bf16_bits(x)
+    q, s = oracle_mod.dispatch_fp8(xb, lay["dispatch_pos"], T * k)
+    acc, _ = oracle_mod.combine_fp8(q, s, lay["dispatch_pos"], w)
+    xf = x.float().numpy().astype(np.float64)
+    wsum = w.astype(np.float64).sum(1, keepdims=True)
+    scale_tok = np.repeat(oracle_mod.quantize_tokens(xb, np.arange(T, dtype=np.int32))[1], 128, 1)
+    bound = wsum * (2.0 ** -4 * np.abs(xf) + scale_tok * 2.0 ** -10) * (1 + 2 ** -20) \
+        + 2 * k * 2.0 ** -24 * wsum * (np.abs(xf) * (1 + 2 ** -4) + scale_tok)
+    assert np.all(np.abs(acc - wsum * xf) <= bound)
