@@ -59,9 +59,10 @@ STEPS_PER_GRAPH = 10           # consecutive steps captured in one CUDA graph (n
 # algorithmic bytes
 # --------------------------------------------------------------------------
 
-def algorithmic_bytes(cfg: inputs.Config, rows: int, kept: int) -> dict:
+def algorithmic_bytes(cfg: inputs.Config, rows: int, kept: int, combine_fp8: bool = False) -> dict:
     """Minimal bytes each stage must move.  kept = slots that have a row
-    (T*k when nothing is dropped); rows = receive rows laid out."""
+    (T*k when nothing is dropped); rows = receive rows laid out.  With
+    combine_fp8 the expert rows come back as E4M3 codes + 1x128 scales."""
     T, H, E, k, R = cfg.T, cfg.H, cfg.E, cfg.k_total, cfg.R
     E_lay = cfg.E_phys if cfg.n_shared else E
     S = H // 128
@@ -71,7 +72,10 @@ def algorithmic_bytes(cfg: inputs.Config, rows: int, kept: int) -> dict:
         dispatch = T * H * 2 + T * k * 4 + kept * H + kept * S * 4
     else:
         dispatch = T * H * 2 + T * k * 4 + kept * H * 2
-    combine = kept * H * 2 + T * k * 8 + T * H * 2
+    if combine_fp8:
+        combine = kept * H + kept * S * 4 + T * k * 8 + T * H * 2
+    else:
+        combine = kept * H * 2 + T * k * 8 + T * H * 2
     return dict(route=route, layout=layout, dispatch=dispatch, combine=combine,
                 step=route + layout + dispatch + combine)
 
@@ -85,11 +89,12 @@ def load_peak() -> tuple[float, str]:
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def combine_traffic(cfg_name: str):
+def combine_traffic(cfg_name: str, fp8: bool = False):
     """DRAM bytes per launch of the combine kernel from the committed ncu
     summary, or None when that summary is missing or the kernel source has
     changed since it was taken."""
-    path = os.path.join(ROOT, "profiles", f"combine_{cfg_name}_traffic.json")
+    kind = "combine_fp8" if fp8 else "combine"
+    path = os.path.join(ROOT, "profiles", f"{kind}_{cfg_name}_traffic.json")
     src = os.path.join(ROOT, "combine_moe_route_08_b200", "csrc", "combine.cu")
     try:
         with open(path) as f:
@@ -345,6 +350,8 @@ def run_ours(args) -> None:
             del probe
         rows = T * k if cap == 0 else E_lay * cap
         lay = moe.moe_dispatch_layout(idx, E_lay, R, capacity=cap, rows=rows, workspace=ws)
+        if args.combine_fp8 and cfg.dispatch != "fp8":
+            raise SystemExit("--combine-fp8 needs an FP8-dispatch workload")
         if args.fused and (args.two_phase or cfg.n_shared):
             raise SystemExit("--fused runs the plain route on the direct layout")
         if args.two_phase:
@@ -411,8 +418,15 @@ def run_ours(args) -> None:
                                          prows, None, sp)),
                 (lib.moe_compact_bf16, (priv_x.data_ptr(), prows, ppos.data_ptr(), pos.data_ptr(),
                                         T, H, k, recv_x.data_ptr(), rows, None, sp))]
-    combine_call = (lib.moe_combine_bf16, (y.data_ptr(), pos.data_ptr(), w.data_ptr(), T, H, k,
-                                           rows, out.data_ptr(), None, sp))
+    if args.combine_fp8:
+        # the expert rows come back in the dispatch's FP8 format: the stand-in
+        # expert returns its input, the dispatched codes and scales
+        combine_call = (lib.moe_combine_fp8, (recv_q.data_ptr(), recv_scale.data_ptr(),
+                                              pos.data_ptr(), w.data_ptr(), T, H, k, rows,
+                                              out.data_ptr(), None, sp))
+    else:
+        combine_call = (lib.moe_combine_bf16, (y.data_ptr(), pos.data_ptr(), w.data_ptr(), T, H,
+                                               k, rows, out.data_ptr(), None, sp))
     if args.fused:
         # route + layout + dispatch in one cooperative launch, then combine
         fws_buf = moe.Workspace(dev).get(moe.moe_route_dispatch_workspace_bytes(T, k, E, R))
@@ -440,7 +454,7 @@ def run_ours(args) -> None:
                     if end == j:
                         ev[q + 1].record(s)
 
-    nb = algorithmic_bytes(cfg, rows, kept)
+    nb = algorithmic_bytes(cfg, rows, kept, args.combine_fp8)
     K, W = args.steps, args.warmup
     l2 = getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 126 << 20)
     flush_needed = nb["step"] < 2 * l2
@@ -646,7 +660,9 @@ def run_ours(args) -> None:
             "config": {"workload": cfg.describe(), "parallelism": f"replicas x{n_gpus}",
                        "l2": l2_mode,
                        "capacity": cap, "rows": rows,
-                       "pipeline": pipeline, "timing": (f"CUDA events around K steps run as replays of CUDA graphs of "
+                       "pipeline": pipeline,
+                       "combine_payload": ("fp8 e4m3 + 1x128 fp32 scales (the dispatched rows)"
+                                           if args.combine_fp8 else "bf16 (stand-in expert output)"), "timing": (f"CUDA events around K steps run as replays of CUDA graphs of "
                                   f"{G} consecutive step(s)")},
             "us_per_layer": ms_step * 1e3,
             "stages_us": stages,
@@ -657,11 +673,13 @@ def run_ours(args) -> None:
                                  "frac_of_measured": dc_bytes / (dc_ms * 1e-3) / 1e9 / peak},
             "stage_timing": stage_how,
             "bytes_per_step": nb,
-            "roofline": {"bound": "hbm", "kernel": "k_combine_bf16", "achieved": comb_gbs,
+            "roofline": {"bound": "hbm",
+                         "kernel": "k_combine_fp8" if args.combine_fp8 else "k_combine_bf16",
+                         "achieved": comb_gbs,
                          "peak": peak, "unit": "GB/s", "frac": comb_gbs / peak,
                          "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
                          else "fallback 6650 GB/s",
-                         "traffic": combine_traffic(cfg.name),
+                         "traffic": combine_traffic(cfg.name, args.combine_fp8),
                          "algorithmic_bytes_per_launch": nb["combine"]},
             "e2e": {"value": n_gpus * nb["step"] / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
                     "us_per_step": e2e_ms * 1e3, "h2d_bytes_per_step": h2d,
@@ -690,6 +708,8 @@ def main(argv=None):
                     help="dispatch as the pages' two-phase form (private regions + compaction)")
     ap.add_argument("--fused", action="store_true",
                     help="route + layout + dispatch as one cooperative launch, then combine")
+    ap.add_argument("--combine-fp8", action="store_true",
+                    help="expert rows come back as E4M3 + 1x128 scales (moe_combine_fp8)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

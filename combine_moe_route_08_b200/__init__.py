@@ -23,7 +23,7 @@ __all__ = [
     "moe_quantize_e4m3", "moe_dispatch_layout_noalloc", "moe_dispatch_fp8_ex", "Workspace",
     "LIB_PATH", "MOE_SCALE_ROW_MAJOR", "MOE_SCALE_COL_MAJOR", "moe_dispatch_layout_private",
     "moe_compact_fp8", "moe_compact_bf16", "moe_route_dispatch_workspace_bytes",
-    "moe_route_dispatch_fp8", "moe_route_dispatch_bf16",
+    "moe_route_dispatch_fp8", "moe_route_dispatch_bf16", "moe_combine_fp8",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_route.so")
@@ -76,6 +76,8 @@ lib.moe_route_dispatch_fp8.restype = _i32
 lib.moe_route_dispatch_bf16.argtypes = [_P, _i32, _i32, _i32, _i32, _i32, _i32, _P, _i32, _P, _P,
                                         _P, _P, _P, _P, _P, _P, _P, _i64, _P, _sz, _P, _P]
 lib.moe_route_dispatch_bf16.restype = _i32
+lib.moe_combine_fp8.argtypes = [_P, _P, _P, _P, _i32, _i32, _i32, _i64, _P, _P, _P]
+lib.moe_combine_fp8.restype = _i32
 lib.moe_quantize_e4m3.argtypes = [_P, _i64, _P, _P]
 lib.moe_quantize_e4m3.restype = _i32
 
@@ -400,6 +402,23 @@ def moe_combine_bf16(y: torch.Tensor, dispatch_pos: torch.Tensor, topk_w: torch.
         out = torch.empty(T, H, dtype=y.dtype, device=y.device)
     _check(lib.moe_combine_bf16(_ptr(y), _ptr(dispatch_pos), _ptr(topk_w), T, H, k, rows,
                                 _ptr(out), _ptr(dev_status), _stream(stream)), "moe_combine_bf16")
+    return out
+
+
+def moe_combine_fp8(y_q: torch.Tensor, y_scale: torch.Tensor, dispatch_pos: torch.Tensor,
+                    topk_w: torch.Tensor, out: torch.Tensor | None = None,
+                    dev_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """out[g] = bf16(sum_j w[g, j] * (decode(y_q[row]) * y_scale[row])) in fp32,
+    ascending j.  y_q uint8 [rows][H] (E4M3), y_scale fp32 [rows][H/128]."""
+    assert y_q.dtype == torch.uint8 and y_scale.dtype == torch.float32
+    rows, H = y_q.shape
+    T, k = dispatch_pos.shape
+    assert topk_w.dtype == torch.float32 and tuple(topk_w.shape) == (T, k)
+    if out is None:
+        out = torch.empty(T, H, dtype=torch.bfloat16, device=y_q.device)
+    _check(lib.moe_combine_fp8(_ptr(y_q), _ptr(y_scale), _ptr(dispatch_pos), _ptr(topk_w), T, H,
+                               k, rows, _ptr(out), _ptr(dev_status), _stream(stream)),
+           "moe_combine_fp8")
     return out
 
 

@@ -357,6 +357,26 @@ int moe_route_dispatch_bf16(const float *logits, int T, int E, int k, int renorm
                                  workspace, ws_bytes, dev_status, stream);
 }
 
+int moe_combine_fp8(const uint8_t *y_q, const float *y_scale, const int32_t *dispatch_pos,
+                    const float *topk_w, int T, int H, int k, int64_t rows, uint16_t *out,
+                    int32_t *dev_status, void *stream)
+{
+    const int st = check_rows_args(T, H, k, dispatch_pos, rows);
+    if (st != MOE_OK)
+        return st;
+    if (H % 128 != 0)
+        return MOE_ERR_UNSUPPORTED;
+    if (T == 0)
+        return MOE_OK;
+    if (!out || !topk_w || !aligned(out, 16) || !aligned(topk_w, 4) ||
+        (dev_status && !aligned(dev_status, 4)))
+        return MOE_ERR_INVALID_ARG;
+    if (rows > 0 && (!y_q || !y_scale || !aligned(y_q, 16) || !aligned(y_scale, 4)))
+        return MOE_ERR_INVALID_ARG;
+    return launched(moe::combine_fp8(y_q, y_scale, dispatch_pos, topk_w, T, H, k, rows, out,
+                                     dev_status, as_stream(stream)));
+}
+
 int moe_quantize_e4m3(const float *v, int64_t n, uint8_t *q, void *stream)
 {
     if (n < 0)

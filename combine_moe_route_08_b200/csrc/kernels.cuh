@@ -83,6 +83,11 @@ cudaError_t route_dispatch(const float *logits, int T, int E, int k, int renorma
                            void *workspace, size_t ws_bytes, int32_t *dev_status, cudaStream_t s,
                            bool *ws_too_small);
 
+// Combine with E4M3 rows yq [rows][H] and row-major 1x128 scales ys [rows][H/128].
+cudaError_t combine_fp8(const uint8_t *yq, const float *ys, const int32_t *dispatch_pos,
+                        const float *topk_w, int T, int H, int k, int64_t rows, uint16_t *out,
+                        int32_t *dev_status, cudaStream_t s);
+
 cudaError_t quantize_e4m3(const float *v, int64_t n, uint8_t *q, cudaStream_t s);
 
 }  // namespace moe

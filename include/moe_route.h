@@ -400,6 +400,23 @@ int moe_combine_bf16(const uint16_t *y, const int32_t *dispatch_pos,
                      uint16_t *out, int32_t *dev_status, void *stream);
 
 /*
+ * moe_combine_fp8 -- moe_combine_bf16 with the expert rows in the dispatch's
+ * FP8 format: E4M3 codes and one fp32 scale per 1x128 block (DeepSeek-V3
+ * fragments: activations scaled per token per 128 channels), a payload of
+ * H + H/32 bytes per row instead of 2H.
+ *   out[g][h] = bf16_rne( acc ), acc = 0; for j = 0..k-1 ascending, slots
+ *   with dispatch_pos == -1 skipped: acc = acc + (topk_w[g][j] *
+ *   (decode(y_q[row][h]) * y_scale[row][h / 128])), each product and sum one
+ *   binary32 operation (decode is exact), no fused multiply-add.
+ *   y_q      [rows][H] E4M3 codes (16-byte aligned rows).
+ *   y_scale  [rows][H/128] fp32, row-major.
+ * H % 128 != 0 -> MOE_ERR_UNSUPPORTED.  T == 0 enqueues nothing.
+ */
+int moe_combine_fp8(const uint8_t *y_q, const float *y_scale, const int32_t *dispatch_pos,
+                    const float *topk_w, int T, int H, int k, int64_t rows, uint16_t *out,
+                    int32_t *dev_status, void *stream);
+
+/*
  * moe_quantize_e4m3 -- q[i] = e4m3(v[i]) with the converter moe_dispatch_fp8
  * uses (round to nearest even, saturating at +-448, NaN -> 0x7F).  Exposed
  * so the converter can be checked on every binary32 bit pattern.

@@ -182,3 +182,12 @@ def test_fused_route_dispatch_rejects_bad_arguments(moe):
                1 << 20, None, None) == moe.MOE_ERR_INVALID_ARG
     assert f16(A4, 64, 8, 2, 0, 2, 0, A16, 56, A4, A4, A4, A4, A4, A4, A4, A4, A16, 128, ws,
                1 << 20, None, None) == moe.MOE_ERR_UNSUPPORTED   # bf16 needs H >= 64
+
+
+def test_combine_fp8_rejects_bad_arguments(moe):
+    f = moe.lib.moe_combine_fp8
+    assert f(A16, A4, A4, A4, 4, 200, 2, 8, A16, None, None) == moe.MOE_ERR_UNSUPPORTED  # H % 128
+    assert f(A16, A4, A4, A4, 4, 128, 0, 8, A16, None, None) == moe.MOE_ERR_INVALID_ARG  # k = 0
+    assert f(A16 + 4, A4, A4, A4, 4, 128, 2, 8, A16, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert f(A16, None, A4, A4, 4, 128, 2, 8, A16, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert f(None, None, None, None, 0, 128, 2, 0, None, None, None) == moe.MOE_OK  # T = 0

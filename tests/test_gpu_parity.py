@@ -425,3 +425,78 @@ def test_two_phase_dispatch_equals_direct(moe, name):
         torch.cuda.synchronize()
         assert torch.equal(rx.view(torch.int16), rx_ref.view(torch.int16))
     assert st.item() == 0
+
+
+# ------------------------------------------------------- combine, FP8 payload
+
+def _fp8_payload(cfg_H, rows, seed, bank=2048):
+    """Seeded E4M3 rows for the FP8-payload combine: a bank of random codes
+    (no NaN codes) and positive scales, rows mapped onto the bank."""
+    rng = np.random.default_rng(seed)
+    q = rng.integers(0, 256, (bank, cfg_H)).astype(np.uint8)
+    q[(q & 0x7F) == 0x7F] = 0x3C
+    s = (rng.random((bank, cfg_H // 128)) * 0.05 + 1e-3).astype(np.float32)
+    rmap = np.arange(rows) % bank
+    return q, s, rmap
+
+
+@pytest.mark.parametrize("name", ["dsv3", "kimi", "dsv3_shared"])
+def test_combine_fp8_parity_full(moe, name):
+    """The dispatched FP8 rows come straight back (identity expert on the FP8
+    payload); GPU and oracle use the same codes, scales and weights."""
+    wl = workload(name)
+    pos = wl["layout"]["dispatch_pos"]
+    rq, rs = oracle.dispatch_fp8(wl["x_bits"], pos, wl["rows"])
+    acc, out_o = oracle.combine_fp8(rq, rs, pos, wl["w"])
+    st = _status()
+    out = moe.moe_combine_fp8(to_dev(rq), to_dev(rs), to_dev(pos), to_dev(wl["w"]), dev_status=st)
+    torch.cuda.synchronize()
+    exact = check_combine(gpu_bits(out), acc, out_o, name)
+    assert exact == 1.0, f"{name}: {exact:.6f} bit-identical"
+    assert st.item() == 0
+
+
+def test_combine_fp8_parity_prefill_sampled(moe):
+    """Prefill at full size (padded rows) with a seeded code/scale bank; the
+    oracle recomputes a sample of tokens."""
+    wl = workload("prefill")
+    cfg = wl["cfg"]
+    q, s, rmap = _fp8_payload(cfg.H, wl["rows"], seed=31)
+    qd = torch.from_numpy(q).cuda()[torch.from_numpy(rmap).cuda()]
+    sd = torch.from_numpy(s).cuda()[torch.from_numpy(rmap).cuda()]
+    pos = wl["layout"]["dispatch_pos"]
+    out = moe.moe_combine_fp8(qd, sd, to_dev(pos), to_dev(wl["w"]))
+    torch.cuda.synchronize()
+    del qd, sd
+    rng = np.random.default_rng(4)
+    tokens = np.unique(np.concatenate([[0, cfg.T - 1], rng.choice(cfg.T, 300, replace=False)]))
+    tokens = tokens.astype(np.int32)
+    used = pos[tokens].ravel()
+    ok = used >= 0
+    q_small = q[rmap[used[ok]]]
+    s_small = s[rmap[used[ok]]]
+    pos_small = np.full(used.shape, -1, np.int32)
+    pos_small[ok] = np.arange(int(ok.sum()), dtype=np.int32)
+    acc, out_o = oracle.combine_fp8(q_small, s_small, pos_small.reshape(len(tokens), cfg.k),
+                                    wl["w"][tokens])
+    assert check_combine(gpu_bits(out)[tokens], acc, out_o, "prefill fp8") == 1.0
+
+
+@pytest.mark.parametrize("k,T", [(1, 37), (3, 37), (8, 37), (11, 37), (32, 37), (8, 4099),
+                                 (2, 9001)])
+def test_combine_fp8_edges(moe, k, T):
+    """k beyond the register-held rows, -1 slots, one 128-channel block; T
+    large enough for several tokens per CTA with a ragged last CTA."""
+    rng = np.random.default_rng(40 + k + T)
+    H, rows = 128, 200
+    q, s, _ = _fp8_payload(H, 64, seed=50 + k, bank=64)
+    q = q[rng.integers(0, 64, rows)]
+    s = s[rng.integers(0, 64, rows)]
+    pos = rng.integers(-1, rows, (T, k)).astype(np.int32)
+    w = rng.random((T, k)).astype(np.float32)
+    acc, out_o = oracle.combine_fp8(q, s, pos, w)
+    st = _status()
+    out = moe.moe_combine_fp8(to_dev(q), to_dev(s), to_dev(pos), to_dev(w), dev_status=st)
+    torch.cuda.synchronize()
+    assert check_combine(gpu_bits(out), acc, out_o, f"k={k}") == 1.0
+    assert st.item() == 0
