@@ -608,24 +608,55 @@ def run_ours(args) -> None:
     del g_step1, g_stepG, g_dc1, g_dcG
 
     # ---- end to end through the public API, host buffers in and out ----
+    # Every step copies its inputs (logits, x) in from pinned host memory and
+    # its output out to pinned host memory, inside the timed region.  The
+    # copies run on their own streams (H2D and D2H have separate copy
+    # engines): step i+1's inputs arrive while step i computes and step
+    # i-1's output leaves, as a serving loop would overlap them.  Inputs and
+    # output are double-buffered; the step's intermediates are reused.
     logits_pin = logits_h.pin_memory()
     x_pin = x_h.pin_memory()
-    out_pin = torch.empty(T, H, dtype=torch.bfloat16).pin_memory()
-    e2e = []
-    with torch.cuda.stream(s):
-        for i in range(max(W, 3) + min(K, 100)):
-            flush(i)
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(s)
-            logits.copy_(logits_pin, non_blocking=True)
-            x.copy_(x_pin, non_blocking=True)
-            step()
-            out_pin.copy_(out, non_blocking=True)
-            b.record(s)
-            if i >= max(W, 3):
-                e2e.append((a, b))
-        s.synchronize()
-    e2e_ms = max_over_ranks([float(np.mean([a.elapsed_time(b) for a, b in e2e]))], world, dev)[0]
+    out_pins = [torch.empty(T, H, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    logits2, x2, out2 = torch.empty_like(logits), torch.empty_like(x), torch.empty_like(out)
+    swap = {logits.data_ptr(): logits2.data_ptr(), x.data_ptr(): x2.data_ptr(),
+            out.data_ptr(): out2.data_ptr()}
+    calls2 = [(fn, tuple(swap.get(v, v) if isinstance(v, int) else v for v in a))
+              for fn, a in calls]
+    sets = [(logits, x, out, calls), (logits2, x2, out2, calls2)]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_done = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    n_e2e = min(K, 100)
+    first, last = max(W, 3), max(W, 3) + n_e2e
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    for i in range(last):
+        lg, xx, oo, cl = sets[i % 2]
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(ev_done[i % 2])   # step i-2 has finished reading this set
+            if i == first:
+                t0.record(s_in)
+            lg.copy_(logits_pin, non_blocking=True)
+            xx.copy_(x_pin, non_blocking=True)
+            ev_in[i % 2].record(s_in)
+        s.wait_event(ev_in[i % 2])
+        if i >= 2:
+            s.wait_event(ev_out[i % 2])           # step i-2's output has left this buffer
+        for fn, a in cl:
+            rc = fn(*a)
+            if rc != 0:
+                raise moe.MoeError(rc, fn.__name__)
+        ev_done[i % 2].record(s)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_done[i % 2])
+            out_pins[i % 2].copy_(oo, non_blocking=True)
+            ev_out[i % 2].record(s_out)
+            if i == last - 1:
+                t1.record(s_out)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks([t0.elapsed_time(t1) / n_e2e], world, dev)[0]
     h2d = logits_h.numel() * 4 + x_h.numel() * 2
     d2h = out.numel() * 2
 
@@ -683,6 +714,10 @@ def run_ours(args) -> None:
                          "algorithmic_bytes_per_launch": nb["combine"]},
             "e2e": {"value": n_gpus * nb["step"] / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
                     "us_per_step": e2e_ms * 1e3, "h2d_bytes_per_step": h2d,
+                    "how": ("C ABI calls launched per step; every step's inputs copied in from "
+                            "pinned host memory and its output copied out, on two copy "
+                            "streams overlapping the neighbouring steps' compute; inputs and "
+                            "output double-buffered; no L2 flush"),
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": launches,
             "clocks": clocks,
