@@ -482,21 +482,28 @@ def test_combine_fp8_parity_prefill_sampled(moe):
     assert check_combine(gpu_bits(out)[tokens], acc, out_o, "prefill fp8") == 1.0
 
 
-@pytest.mark.parametrize("k,T", [(1, 37), (3, 37), (8, 37), (11, 37), (32, 37), (8, 4099),
-                                 (2, 9001)])
-def test_combine_fp8_edges(moe, k, T):
-    """k beyond the register-held rows, -1 slots, one 128-channel block; T
-    large enough for several tokens per CTA with a ragged last CTA."""
-    rng = np.random.default_rng(40 + k + T)
-    H, rows = 128, 200
-    q, s, _ = _fp8_payload(H, 64, seed=50 + k, bank=64)
+@pytest.mark.parametrize("k,T,H", [(1, 37, 128), (3, 37, 128), (8, 37, 128), (11, 37, 128),
+                                   (32, 37, 128), (8, 4099, 128), (2, 9001, 128),
+                                   (1, 37, 512), (8, 300, 512), (11, 37, 512), (32, 37, 512),
+                                   (8, 4099, 1024)])
+@pytest.mark.parametrize("scale_offset", [0, 1])
+def test_combine_fp8_edges(moe, k, T, H, scale_offset):
+    """k beyond the register-held rows, -1 slots, ragged token counts (several
+    tokens per CTA with a short last CTA), several hidden sizes, and a scale
+    plane that is only 4-byte aligned."""
+    rng = np.random.default_rng(40 + k + T + H + scale_offset)
+    rows = 200
+    q, s, _ = _fp8_payload(H, 64, seed=50 + k + H, bank=64)
     q = q[rng.integers(0, 64, rows)]
     s = s[rng.integers(0, 64, rows)]
     pos = rng.integers(-1, rows, (T, k)).astype(np.int32)
     w = rng.random((T, k)).astype(np.float32)
     acc, out_o = oracle.combine_fp8(q, s, pos, w)
     st = _status()
-    out = moe.moe_combine_fp8(to_dev(q), to_dev(s), to_dev(pos), to_dev(w), dev_status=st)
+    s_dev = torch.zeros(rows * (H // 128) + 4, dtype=torch.float32, device="cuda")
+    s_view = s_dev[scale_offset:scale_offset + rows * (H // 128)].view(rows, H // 128)
+    s_view.copy_(to_dev(s))
+    out = moe.moe_combine_fp8(to_dev(q), s_view, to_dev(pos), to_dev(w), dev_status=st)
     torch.cuda.synchronize()
-    assert check_combine(gpu_bits(out), acc, out_o, f"k={k}") == 1.0
+    assert check_combine(gpu_bits(out), acc, out_o, f"k={k} T={T} H={H}") == 1.0
     assert st.item() == 0
