@@ -8,20 +8,23 @@
 // precision (DeepSeek-V3 fragments): fp32 logits in, fp32 weights out.
 //
 // Each lane holds the logits e = i*32 + lane (a warp-wide load per i is one
-// coalesced 128-byte line), as order-preserving 32-bit keys.  k rounds of
-// warp arg-max under the order (logit descending, index ascending) pick the
-// experts: one warp-wide max of the lanes' best keys and one warp-wide min of
-// the indices holding it (redux.sync, a single instruction each), then the
-// winner's key is cleared.
+// coalesced 128-byte line), as order-preserving 32-bit keys, and tracks its
+// own best key.  k rounds of warp arg-max under the order (logit descending,
+// index ascending) pick the experts: one warp-wide max of the lanes' best
+// keys and one warp-wide min of the expert ids holding it (redux.sync, a
+// single instruction each); only the winning lane then clears that key and
+// rescans for its next best.
 //
-// The softmax is evaluated in fp32 with its error bounded (u = 2^-24):
+// The softmax is evaluated with its error bounded (u = 2^-24):
 //   d = l - m is split exactly into d_hi + d_lo (Knuth's TwoSum), so the
 //   exponent sees no rounding of the difference; t = expf(d_hi) * (1 + d_lo)
 //   has relative error <= 5u (expf is within 2 ulp = 4u, plus one rounding);
-//   the denominator is a compensated (Neumaier) sum of the positive t, within
-//   2u of their exact sum; w = t_j / S is one IEEE division (u).  Hence
-//   |w - p| <= 13u * p (+ O(u^2)) for the exact probability p, i.e. within 16
-//   fp32 ulps of the correctly rounded value; in practice 1-2 ulps.
+//   the denominator sums the positive t in binary64 (at most 1024 terms of at
+//   most 1: its error is below 2^-42 relative, far under u) and is rounded
+//   once to binary32 (u); w = t_j / S is one IEEE division (u).  Hence
+//   |w - p| <= 7u * p (+ O(u^2)) for the exact probability p; in practice
+//   1-2 ulps.  Lane 0's total is broadcast, so all of a token's weights
+//   share one denominator.
 #pragma once
 
 #include <cfloat>
@@ -39,14 +42,6 @@ __device__ __forceinline__ void two_sum(float a, float b, float &s, float &err)
     err = __fadd_rn(__fsub_rn(a, __fsub_rn(s, bb)), __fsub_rn(b, bb));
 }
 
-// Neumaier's compensated summation step: (sum + comp) absorbs t.
-__device__ __forceinline__ void neumaier_add(float &sum, float &comp, float t)
-{
-    float s, err;
-    two_sum(sum, t, s, err);
-    sum = s;
-    comp = __fadd_rn(comp, err);
-}
 
 // exp(l - m) for fp32 l <= m: the difference split exactly into hi + lo, the
 // exponential of hi by expf, the first-order factor (1 + lo) applied with one
@@ -62,17 +57,13 @@ __device__ __forceinline__ float exp_diff(float l, float m)
     return __fmaf_rn(t, lo, t);
 }
 
-// Warp-wide compensated sum of (sum, comp) pairs.
-__device__ __forceinline__ float warp_neumaier_total(float sum, float comp)
+// Warp-wide binary64 sum, rounded once to binary32; lane 0's value for all.
+__device__ __forceinline__ float warp_total_f64(double sum)
 {
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-        const float os = __shfl_xor_sync(kFullMask, sum, off);
-        const float oc = __shfl_xor_sync(kFullMask, comp, off);
-        comp = __fadd_rn(comp, oc);
-        neumaier_add(sum, comp, os);
-    }
-    return __fadd_rn(sum, comp);
+    for (int off = 16; off > 0; off >>= 1)
+        sum = __dadd_rn(sum, __shfl_xor_sync(kFullMask, sum, off));
+    return __shfl_sync(kFullMask, __double2float_rn(sum), 0);
 }
 
 // Route one token with the whole warp: on return lane j < k holds the j-th
@@ -110,32 +101,42 @@ __device__ __forceinline__ void route_warp(const float *__restrict__ row, int E,
             key[i] = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
         }
     }
+    // Each lane keeps its best key and that key's slot (the lowest slot among
+    // equal keys); a round is one warp max of the lanes' bests, one warp min
+    // of the expert ids holding it, and a rescan by the winning lane alone.
+    // The chosen logit is read back from the winning key (the map is
+    // invertible; -0 comes back as +0, which gives the same softmax terms).
+    uint32_t bk = 0u;
+    int bi = 0;
+#pragma unroll
+    for (int i = 0; i < NPL; ++i)
+        if (key[i] > bk) {
+            bk = key[i];
+            bi = i;
+        }
     my_e = 0;
     float my_v = 0.0f;
     float vmax = 0.0f;
     for (int j = 0; j < k; ++j) {
-        uint32_t best = 0u;
-#pragma unroll
-        for (int i = 0; i < NPL; ++i)
-            best = max(best, key[i]);
-        const uint32_t m = __reduce_max_sync(kFullMask, best);
-        uint32_t cand = 0xffffffffu;
-#pragma unroll
-        for (int i = NPL - 1; i >= 0; --i)
-            if (key[i] == m)
-                cand = static_cast<uint32_t>(i * 32 + lane);
+        const uint32_t m = __reduce_max_sync(kFullMask, bk);
+        const uint32_t cand = (bk == m) ? static_cast<uint32_t>(bi * 32 + lane) : 0xffffffffu;
         const uint32_t e = __reduce_min_sync(kFullMask, cand);
-        const int ei = static_cast<int>(e >> 5);
-        float ve = 0.0f;
+        const uint32_t u = (m & 0x80000000u) ? (m & 0x7fffffffu) : ~m;
+        const float ve = __uint_as_float(u);
+        if ((e & 31u) == static_cast<uint32_t>(lane)) {  // the winner takes its next best
+            const int taken = bi;
+            bk = 0u;
+            bi = 0;
 #pragma unroll
-        for (int i = 0; i < NPL; ++i) {
-            if (i == ei && (e & 31u) == static_cast<uint32_t>(lane)) {
-                key[i] = 0u;
+            for (int i = 0; i < NPL; ++i) {
+                if (i == taken)
+                    key[i] = 0u;
+                if (key[i] > bk) {
+                    bk = key[i];
+                    bi = i;
+                }
             }
-            if (i == ei)
-                ve = v[i];
         }
-        ve = __shfl_sync(kFullMask, ve, static_cast<int>(e & 31u));
         if (lane == j) {
             my_e = static_cast<int>(e);
             my_v = ve;
@@ -144,17 +145,17 @@ __device__ __forceinline__ void route_warp(const float *__restrict__ row, int E,
             vmax = ve;
     }
 
-    // softmax over all E logits, in fp32 with compensated summation
-    float sum = 0.0f, comp = 0.0f;
+    // softmax over all E logits: fp32 terms, binary64 sum
+    double sum = 0.0;
 #pragma unroll
     for (int i = 0; i < NPL; ++i)
         if (i * 32 + lane < E)
-            neumaier_add(sum, comp, exp_diff(v[i], vmax));
-    float denom = warp_neumaier_total(sum, comp);
+            sum = __dadd_rn(sum, static_cast<double>(exp_diff(v[i], vmax)));
+    float denom = warp_total_f64(sum);
 
     const float num = (lane < k) ? exp_diff(my_v, vmax) : 0.0f;
     if (renormalize)
-        denom = warp_neumaier_total(num, 0.0f);
+        denom = warp_total_f64(static_cast<double>(num));
     my_w = (lane < k) ? __fdiv_rn(num, denom) : 0.0f;
 }
 

@@ -85,9 +85,9 @@ const char *moe_status_string(int status);
  *             descending, expert index ascending); -0.0 and +0.0 are equal.
  *   topk_w    [T][k] fp32 out: p_e = exp(l_e - m) / sum_e' exp(l_e' - m),
  *             m = max logit; with renormalize != 0 the sum runs over the k
- *             chosen experts only (softmax restricted to the top-k).  Computed
- *             in fp32 (exact split of l - m, expf, compensated sum, one IEEE
- *             division): |topk_w - p| <= 14 * 2^-24 * p.
+ *             chosen experts only (softmax restricted to the top-k).  Terms in
+ *             fp32 (exact split of l - m, expf), their sum in binary64 rounded
+ *             once, one IEEE division: |topk_w - p| <= 7 * 2^-24 * p.
  * Logits must be finite.  T == 0 enqueues nothing.
  */
 int moe_route_topk(const float *logits, int T, int E, int k, int renormalize,
