@@ -138,3 +138,16 @@ def test_route_ex_multi_replica_choice_and_bad_table(oracle_mod):
     idx_b, _, st_b = oracle_mod.route_ex(logits.numpy(), 2, 0, 1.0, offs, bad, 9, 4)
     assert st_b == oracle_mod.ERR_INVALID
     assert np.all(idx_b[plain == 2] == -1) and np.all(idx_b[plain != 2] == idx[plain != 2])
+
+
+def test_route_ex_several_shared_experts_and_their_weight(oracle_mod):
+    """Shared experts E, E+1, ... follow the routed slots in that order, each
+    with the given shared weight; without a replica table every logical id is
+    its own physical id."""
+    logits, _ = inputs.make_random_case(20, 8, 10, 3, seed=41)
+    idx, w, st = oracle_mod.route_ex(logits.numpy(), 3, 2, 0.25, E_phys=12)
+    assert st == oracle_mod.OK and idx.shape == (20, 5)
+    plain_idx, plain_w = oracle_mod.route(logits.numpy(), 3)
+    assert np.array_equal(idx[:, :3], plain_idx) and np.array_equal(w[:, :3], plain_w)
+    assert np.all(idx[:, 3] == 10) and np.all(idx[:, 4] == 11)
+    assert np.all(w[:, 3:] == np.float32(0.25))
