@@ -717,14 +717,24 @@ int max_resident(KernelFn fn, size_t smem)
 
 int query_resident(KernelFn fn, size_t smem)
 {
-    int dev = 0, nsm = 0, per = 0, coop = 0;
+    int dev = 0, nsm = 0, per = 0, coop = 0, optin = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess || !coop)
+        cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess || !coop ||
+        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
         return 0;
-    if (smem > 48 * 1024 &&
-        cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
+    // The limit is a property of the kernel, shared by every geometry: it is
+    // raised to the most the device allows next to the kernel's static
+    // shared memory (never lowered to one geometry's need, which would break
+    // a larger geometry whose answer is already cached).
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess)
+        return 0;
+    const size_t limit = static_cast<size_t>(optin) - fa.sharedSizeBytes;
+    if (smem > limit)
+        return 0;
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(limit)) != cudaSuccess)
         return 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, fn, kThreads, smem) != cudaSuccess)
         return 0;

@@ -345,3 +345,45 @@ def test_fused_wait_gives_up_and_reports_timeout(moe):
     got = _fused(moe, logits, x, cfg.k, cfg.R, 0, wl["rows"], False, ws=ws, st=st2)
     assert st2.item() == 0
     assert np.array_equal(got["dispatch_pos"].cpu().numpy(), wl["layout"]["dispatch_pos"])
+
+
+def _random_shapes(n, seed):
+    """Seeded random (T, H, E, k, R, cap, fp8) with T % R == 0, E % R == 0."""
+    rng = np.random.default_rng(seed)
+    shapes = []
+    while len(shapes) < n:
+        E = int(rng.choice([4, 8, 16, 24, 37, 64, 96, 128, 256, 320, 384, 512, 1000, 1024]))
+        divs = [r for r in range(1, E + 1) if E % r == 0]
+        R = int(rng.choice(divs))
+        k = int(rng.integers(1, min(E, 32) + 1))
+        Tr = int(rng.choice([1, 2, 3, 7, 16, 33, 128, 400]))
+        T = Tr * R
+        if T * k > 400000 or T > 40000:
+            continue
+        fp8 = bool(rng.integers(0, 2))
+        H = int(rng.choice([128, 256, 512])) if fp8 else int(rng.choice([64, 136, 256]))
+        cap = 0 if rng.random() < 0.6 else int(rng.integers(1, max(2, T * k // E + 3)))
+        shapes.append((T, H, E, k, R, cap, fp8))
+    return shapes
+
+
+@pytest.mark.parametrize("case", _random_shapes(24, 2026),
+                         ids=lambda c: "T{}_H{}_E{}_k{}_R{}_cap{}_{}".format(
+                             c[0], c[1], c[2], c[3], c[4], c[5], "fp8" if c[6] else "bf16"))
+def test_fused_random_shapes_match_separate_and_oracle(moe, case):
+    T, H, E, k, R, cap, fp8 = case
+    logits, x = inputs.make_random_case(T, H, E, k, seed=T * 7 + E + k)
+    idx_o, _ = oracle.route(logits.numpy(), k)
+    lay_o = oracle.layout(idx_o, E, R, cap)
+    rows = lay_o["recv_src"].shape[0]
+    st = _status()
+    lg, xd = to_dev(logits), to_dev(x)
+    got = _fused(moe, lg, xd, k, R, cap, rows, fp8, st=st)
+    want_st = moe.MOE_ERR_CAPACITY if lay_o["status"] == oracle.ERR_CAPACITY else 0
+    assert st.item() == want_st
+    assert np.array_equal(got["topk_idx"].cpu().numpy(), idx_o)
+    for key in LAYOUT_KEYS:
+        assert np.array_equal(got[key].cpu().numpy(), lay_o[key].reshape(got[key].shape)), key
+    sep = _separate(moe, lg, xd, k, R, cap, rows, fp8)
+    _assert_same_as_separate(got, sep, fp8, str(case))
+    _assert_unfilled_untouched(got, fp8)
