@@ -318,3 +318,66 @@ def test_route_ex_replicas_and_bad_table(moe):
     torch.cuda.synchronize()
     assert st_o == oracle.ERR_INVALID and st.item() == moe.MOE_ERR_INVALID_ARG
     assert np.array_equal(got_i.cpu().numpy(), want_i)
+
+
+def _two_phase_shapes(n, seed):
+    """Seeded random (T, H, E, k, R, max_m, fp8) for the two-phase path."""
+    rng = np.random.default_rng(seed)
+    out = []
+    while len(out) < n:
+        E = int(rng.choice([4, 8, 16, 37, 64, 128, 256, 384]))
+        R = int(rng.choice([r for r in range(1, E + 1) if E % r == 0 and r <= 64]))
+        k = int(rng.integers(1, min(E, 12) + 1))
+        Tr = int(rng.choice([1, 2, 5, 16, 64, 130]))
+        T = Tr * R
+        if T * k > 200000 or E * R * Tr * 256 > 2 ** 31:
+            continue
+        max_m = int(rng.choice([1, 2, max(1, Tr // 2), Tr]))
+        fp8 = bool(rng.integers(0, 2))
+        H = int(rng.choice([128, 256])) if fp8 else int(rng.choice([8, 64, 136]))
+        out.append((T, H, E, k, R, max_m, fp8))
+    return out
+
+
+@pytest.mark.parametrize("case", _two_phase_shapes(16, 77),
+                         ids=lambda c: "T{}_H{}_E{}_k{}_R{}_m{}_{}".format(
+                             c[0], c[1], c[2], c[3], c[4], c[5], "fp8" if c[6] else "bf16"))
+def test_two_phase_random_shapes(moe, case):
+    """Private layout against the oracle (drops when max_m < the largest
+    per-(expert, rank) count); send + compact equals the direct dispatch on
+    the rows that were kept."""
+    T, H, E, k, R, max_m, fp8 = case
+    logits, x = inputs.make_random_case(T, H, E, k, seed=T + E * 3 + k)
+    idx_o, _ = oracle.route(logits.numpy(), k)
+    ppos_o, base_o, _, st_o = oracle.private_layout(idx_o, E, R, max_m)
+    st = _status()
+    lay = moe.moe_dispatch_layout_private(to_dev(idx_o), E, R, max_m, dev_status=st)
+    torch.cuda.synchronize()
+    want_st = moe.MOE_ERR_CAPACITY if st_o == oracle.ERR_CAPACITY else 0
+    assert st.item() == want_st
+    assert np.array_equal(lay["private_pos"].cpu().numpy(), ppos_o)
+    packed = oracle.layout(idx_o, E, R)
+    want_pos = np.where(ppos_o >= 0, packed["dispatch_pos"], -1)
+    assert np.array_equal(lay["dispatch_pos"].cpu().numpy(), want_pos)
+    prows, rows = lay["private_rows"], T * k
+    xd = to_dev(x)
+    st2 = _status()
+    if fp8:
+        pq, ps = moe.moe_dispatch_fp8(xd, lay["private_pos"], prows, dev_status=st2)
+        q, s = moe.moe_compact_fp8(pq, ps, lay["private_pos"], lay["dispatch_pos"], rows,
+                                   dev_status=st2)
+        q_ref, s_ref = moe.moe_dispatch_fp8(xd, lay["dispatch_pos"], rows)
+        torch.cuda.synchronize()
+        kept = torch.from_numpy(np.nonzero(lay["recv_src"].cpu().numpy() >= 0)[0]).cuda()
+        assert torch.equal(q.index_select(0, kept), q_ref.index_select(0, kept))
+        assert torch.equal(s.index_select(0, kept), s_ref.index_select(0, kept))
+    else:
+        px = moe.moe_dispatch_bf16(xd, lay["private_pos"], prows, dev_status=st2)
+        rx = moe.moe_compact_bf16(px, lay["private_pos"], lay["dispatch_pos"], rows,
+                                  dev_status=st2)
+        rx_ref = moe.moe_dispatch_bf16(xd, lay["dispatch_pos"], rows)
+        torch.cuda.synchronize()
+        kept = torch.from_numpy(np.nonzero(lay["recv_src"].cpu().numpy() >= 0)[0]).cuda()
+        assert torch.equal(rx.index_select(0, kept).view(torch.int16),
+                           rx_ref.index_select(0, kept).view(torch.int16))
+    assert st2.item() == 0
