@@ -352,8 +352,8 @@ def run_ours(args) -> None:
         lay = moe.moe_dispatch_layout(idx, E_lay, R, capacity=cap, rows=rows, workspace=ws)
         if args.combine_fp8 and cfg.dispatch != "fp8":
             raise SystemExit("--combine-fp8 needs an FP8-dispatch workload")
-        if args.fused and (args.two_phase or cfg.n_shared):
-            raise SystemExit("--fused runs the plain route on the direct layout")
+        if args.fused and args.two_phase:
+            raise SystemExit("--fused runs the direct layout")
         if args.two_phase:
             if cap:
                 raise SystemExit("--two-phase needs a packed-layout workload")
@@ -429,13 +429,21 @@ def run_ours(args) -> None:
                                                k, rows, out.data_ptr(), None, sp))
     if args.fused:
         # route + layout + dispatch in one cooperative launch, then combine
-        fws_buf = moe.Workspace(dev).get(moe.moe_route_dispatch_workspace_bytes(T, k, E, R))
-        head = (logits.data_ptr(), T, E, k, 0, R, cap, x.data_ptr(), H, idx.data_ptr(),
-                w.data_ptr(), *lay_args[7:])
+        # (with shared experts: the extended route, the layout over E_phys)
+        fws_buf = moe.Workspace(dev).get(moe.moe_route_dispatch_workspace_bytes(T, k, E_lay, R))
+        if cfg.n_shared:
+            head = (logits.data_ptr(), T, E, cfg.k, 0, cfg.n_shared, 1.0,
+                    replica_offsets.data_ptr(), replica_ids.data_ptr(), replica_ids.numel(),
+                    cfg.E_phys, R, cap, x.data_ptr(), H, idx.data_ptr(), w.data_ptr(),
+                    *lay_args[7:])
+            f8, f16 = lib.moe_route_dispatch_ex_fp8, lib.moe_route_dispatch_ex_bf16
+        else:
+            head = (logits.data_ptr(), T, E, k, 0, R, cap, x.data_ptr(), H, idx.data_ptr(),
+                    w.data_ptr(), *lay_args[7:])
+            f8, f16 = lib.moe_route_dispatch_fp8, lib.moe_route_dispatch_bf16
         tail = (rows, fws_buf.data_ptr(), fws_buf.numel(), None, sp)
-        fused_call = ((lib.moe_route_dispatch_fp8, head + (recv_q.data_ptr(), recv_scale.data_ptr())
-                       + tail) if cfg.dispatch == "fp8" else
-                      (lib.moe_route_dispatch_bf16, head + (recv_x.data_ptr(),) + tail))
+        fused_call = ((f8, head + (recv_q.data_ptr(), recv_scale.data_ptr()) + tail)
+                      if cfg.dispatch == "fp8" else (f16, head + (recv_x.data_ptr(),) + tail))
         calls = [fused_call, combine_call]
         stage_end = [0, 0, 0]      # route, layout and dispatch all end with the fused call
     else:

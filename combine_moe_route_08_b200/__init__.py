@@ -23,7 +23,8 @@ __all__ = [
     "moe_quantize_e4m3", "moe_dispatch_layout_noalloc", "moe_dispatch_fp8_ex", "Workspace",
     "LIB_PATH", "MOE_SCALE_ROW_MAJOR", "MOE_SCALE_COL_MAJOR", "moe_dispatch_layout_private",
     "moe_compact_fp8", "moe_compact_bf16", "moe_route_dispatch_workspace_bytes",
-    "moe_route_dispatch_fp8", "moe_route_dispatch_bf16", "moe_combine_fp8",
+    "moe_route_dispatch_fp8", "moe_route_dispatch_bf16", "moe_route_dispatch_ex_fp8",
+    "moe_route_dispatch_ex_bf16", "moe_combine_fp8",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_route.so")
@@ -76,6 +77,15 @@ lib.moe_route_dispatch_fp8.restype = _i32
 lib.moe_route_dispatch_bf16.argtypes = [_P, _i32, _i32, _i32, _i32, _i32, _i32, _P, _i32, _P, _P,
                                         _P, _P, _P, _P, _P, _P, _P, _i64, _P, _sz, _P, _P]
 lib.moe_route_dispatch_bf16.restype = _i32
+_EX = [_i32, ctypes.c_float, _P, _P, _i32, _i32]  # n_shared .. E_phys
+lib.moe_route_dispatch_ex_fp8.argtypes = ([_P, _i32, _i32, _i32, _i32] + _EX +
+                                          [_i32, _i32, _P, _i32] + [_P] * 10 +
+                                          [_i64, _P, _sz, _P, _P])
+lib.moe_route_dispatch_ex_fp8.restype = _i32
+lib.moe_route_dispatch_ex_bf16.argtypes = ([_P, _i32, _i32, _i32, _i32] + _EX +
+                                           [_i32, _i32, _P, _i32] + [_P] * 9 +
+                                           [_i64, _P, _sz, _P, _P])
+lib.moe_route_dispatch_ex_bf16.restype = _i32
 lib.moe_combine_fp8.argtypes = [_P, _P, _P, _P, _i32, _i32, _i32, _i64, _P, _P, _P]
 lib.moe_combine_fp8.restype = _i32
 lib.moe_quantize_e4m3.argtypes = [_P, _i64, _P, _P]
@@ -433,10 +443,16 @@ _default_fused_ws: dict[torch.device, Workspace] = {}
 
 
 def _route_dispatch(fp8: bool, logits, x, k, R, capacity, rows, renormalize, out, workspace,
-                    dev_status, stream) -> dict:
+                    dev_status, stream, ex: dict | None = None) -> dict:
     assert logits.dtype == torch.float32 and logits.dim() == 2
     x = _bits16(x)
-    T, E = logits.shape
+    T, E_route = logits.shape
+    k_route = k
+    if ex is not None:  # the layout's view: k + n_shared slots over E_phys experts
+        k = k_route + ex["n_shared"]
+        E = ex["E_phys"]
+    else:
+        E = E_route
     H = x.shape[1]
     assert x.shape[0] == T
     dev = logits.device
@@ -465,10 +481,26 @@ def _route_dispatch(fp8: bool, logits, x, k, R, capacity, rows, renormalize, out
     if nbytes == 0:
         raise MoeError(MOE_ERR_INVALID_ARG, "moe_route_dispatch_workspace_bytes")
     ws = workspace.get(nbytes)
-    common = (_ptr(logits), T, E, k, int(renormalize), R, capacity, _ptr(x), H,
-              _ptr(out["topk_idx"]), _ptr(out["topk_w"]), _ptr(out["expert_counts"]),
-              _ptr(out["expert_src_counts"]), _ptr(out["rank_counts"]),
-              _ptr(out["expert_offsets"]), _ptr(out["dispatch_pos"]), _ptr(out["recv_src"]))
+    tail = (_ptr(out["topk_idx"]), _ptr(out["topk_w"]), _ptr(out["expert_counts"]),
+            _ptr(out["expert_src_counts"]), _ptr(out["rank_counts"]),
+            _ptr(out["expert_offsets"]), _ptr(out["dispatch_pos"]), _ptr(out["recv_src"]))
+    if ex is not None:
+        ids = ex.get("replica_ids")
+        head = (_ptr(logits), T, E_route, k_route, int(renormalize), ex["n_shared"],
+                float(ex.get("shared_weight", 1.0)), _ptr(ex.get("replica_offsets")), _ptr(ids),
+                0 if ids is None else ids.numel(), E, R, capacity, _ptr(x), H) + tail
+        if fp8:
+            _check(lib.moe_route_dispatch_ex_fp8(*head, _ptr(out["recv_q"]),
+                                                 _ptr(out["recv_scale"]), rows, _ptr(ws),
+                                                 ws.numel(), _ptr(dev_status), _stream(stream)),
+                   "moe_route_dispatch_ex_fp8")
+        else:
+            _check(lib.moe_route_dispatch_ex_bf16(*head, _ptr(out["recv_x"]), rows, _ptr(ws),
+                                                  ws.numel(), _ptr(dev_status), _stream(stream)),
+                   "moe_route_dispatch_ex_bf16")
+        out["rows"] = rows
+        return out
+    common = (_ptr(logits), T, E, k, int(renormalize), R, capacity, _ptr(x), H) + tail
     if fp8:
         _check(lib.moe_route_dispatch_fp8(*common, _ptr(out["recv_q"]), _ptr(out["recv_scale"]),
                                           rows, _ptr(ws), ws.numel(), _ptr(dev_status),
@@ -501,6 +533,42 @@ def moe_route_dispatch_bf16(logits: torch.Tensor, x: torch.Tensor, k: int, R: in
     moe_route_dispatch_fp8); the rows are returned as recv_x [rows][H]."""
     return _route_dispatch(False, logits, x, k, R, capacity, rows, renormalize, out, workspace,
                            dev_status, stream)
+
+
+def _ex_spec(E, n_shared, shared_weight, replica_offsets, replica_ids, E_phys) -> dict:
+    return dict(n_shared=n_shared, shared_weight=shared_weight, replica_offsets=replica_offsets,
+                replica_ids=replica_ids, E_phys=E + n_shared if E_phys is None else E_phys)
+
+
+def moe_route_dispatch_ex_fp8(logits: torch.Tensor, x: torch.Tensor, k: int, R: int,
+                              n_shared: int = 0, shared_weight: float = 1.0,
+                              replica_offsets: torch.Tensor | None = None,
+                              replica_ids: torch.Tensor | None = None, E_phys: int | None = None,
+                              capacity: int = 0, rows: int | None = None,
+                              renormalize: bool = False, out: dict | None = None,
+                              workspace: Workspace | None = None,
+                              dev_status: torch.Tensor | None = None, stream=None) -> dict:
+    """moe_route_dispatch_fp8 with the routing of moe_route_topk_ex (shared
+    experts, replicas chosen by source rank = token // (T // R)); the layout
+    arrays are over E_phys experts and k + n_shared slots per token."""
+    ex = _ex_spec(logits.shape[1], n_shared, shared_weight, replica_offsets, replica_ids, E_phys)
+    return _route_dispatch(True, logits, x, k, R, capacity, rows, renormalize, out, workspace,
+                           dev_status, stream, ex)
+
+
+def moe_route_dispatch_ex_bf16(logits: torch.Tensor, x: torch.Tensor, k: int, R: int,
+                               n_shared: int = 0, shared_weight: float = 1.0,
+                               replica_offsets: torch.Tensor | None = None,
+                               replica_ids: torch.Tensor | None = None, E_phys: int | None = None,
+                               capacity: int = 0, rows: int | None = None,
+                               renormalize: bool = False, out: dict | None = None,
+                               workspace: Workspace | None = None,
+                               dev_status: torch.Tensor | None = None, stream=None) -> dict:
+    """moe_route_dispatch_bf16 with the routing of moe_route_topk_ex (see
+    moe_route_dispatch_ex_fp8)."""
+    ex = _ex_spec(logits.shape[1], n_shared, shared_weight, replica_offsets, replica_ids, E_phys)
+    return _route_dispatch(False, logits, x, k, R, capacity, rows, renormalize, out, workspace,
+                           dev_status, stream, ex)
 
 
 def moe_quantize_e4m3(v: torch.Tensor, q: torch.Tensor | None = None, stream=None) -> torch.Tensor:

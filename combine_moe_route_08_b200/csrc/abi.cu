@@ -283,9 +283,7 @@ size_t moe_route_dispatch_workspace_bytes(int T, int k, int E, int R)
 {
     if (!valid_layout_sizes(T, k, E, R))
         return 0;
-    const size_t a = moe::route_dispatch_workspace_bytes(T, k, E, R, true);
-    const size_t b = moe::route_dispatch_workspace_bytes(T, k, E, R, false);
-    return (a == 0 || b == 0) ? 0 : (a > b ? a : b);
+    return moe::route_dispatch_workspace_bytes(T, k, E, R);
 }
 
 static int route_dispatch_common(const float *logits, int T, int E, int k, int renormalize, int R,
@@ -295,15 +293,20 @@ static int route_dispatch_common(const float *logits, int T, int E, int k, int r
                                  int32_t *expert_offsets, int32_t *dispatch_pos,
                                  int32_t *recv_src, void *recv, float *recv_scale, int64_t rows,
                                  void *workspace, size_t ws_bytes, int32_t *dev_status,
-                                 void *stream)
+                                 void *stream, const moe::RouteEx *ex = nullptr)
 {
-    if (!valid_layout_sizes(T, k, E, R) || capacity < 0 || rows < 0 || rows >= kMaxIndex ||
+    // the layout's view: slots per token and experts after the extension
+    const int kl = k + (ex ? ex->n_shared : 0);
+    const int El = ex ? ex->E_phys : E;
+    if (ex && (E < 1 || E > kMaxE || k < 1 || k > E))
+        return MOE_ERR_INVALID_ARG;
+    if (!valid_layout_sizes(T, kl, El, R) || capacity < 0 || rows < 0 || rows >= kMaxIndex ||
         H < 8 || H % 8 != 0 || H > (1 << 20) || static_cast<int64_t>(T) * H > (int64_t(1) << 40))
         return MOE_ERR_INVALID_ARG;
     if ((fp8 && H % 128 != 0) || (!fp8 && H < 64))
         return MOE_ERR_UNSUPPORTED;
-    const int64_t needed = (capacity == 0) ? static_cast<int64_t>(T) * k
-                                           : static_cast<int64_t>(E) * capacity;
+    const int64_t needed = (capacity == 0) ? static_cast<int64_t>(T) * kl
+                                           : static_cast<int64_t>(El) * capacity;
     if (rows < needed)
         return MOE_ERR_INVALID_ARG;
     const void *arrays[] = {expert_counts, expert_src_counts, rank_counts, expert_offsets};
@@ -325,7 +328,7 @@ static int route_dispatch_common(const float *logits, int T, int E, int k, int r
     const cudaError_t err = moe::route_dispatch(
         logits, T, E, k, renormalize != 0, R, capacity, x, H, fp8, topk_idx, topk_w, expert_counts,
         expert_src_counts, rank_counts, expert_offsets, dispatch_pos, recv_src, recv, recv_scale,
-        rows, workspace, ws_bytes, dev_status, as_stream(stream), &small);
+        rows, workspace, ws_bytes, dev_status, as_stream(stream), &small, ex);
     if (small)
         return MOE_ERR_WORKSPACE;
     return launched(err);
@@ -375,6 +378,68 @@ int moe_combine_fp8(const uint8_t *y_q, const float *y_scale, const int32_t *dis
         return MOE_ERR_INVALID_ARG;
     return launched(moe::combine_fp8(y_q, y_scale, dispatch_pos, topk_w, T, H, k, rows, out,
                                      dev_status, as_stream(stream)));
+}
+
+// Shared experts and replicas for the fused launch: the same checks as
+// moe_route_topk_ex; the replica choice uses T / R tokens per source rank.
+static int route_dispatch_ex(const float *logits, int T, int E, int k, int renormalize,
+                             int n_shared, float shared_weight, const int32_t *replica_offsets,
+                             const int32_t *replica_ids, int n_replica_ids, int E_phys, int R,
+                             int capacity, const uint16_t *x, int H, bool fp8, int32_t *topk_idx,
+                             float *topk_w, int32_t *expert_counts, int32_t *expert_src_counts,
+                             int32_t *rank_counts, int32_t *expert_offsets, int32_t *dispatch_pos,
+                             int32_t *recv_src, void *recv, float *recv_scale, int64_t rows,
+                             void *workspace, size_t ws_bytes, int32_t *dev_status, void *stream)
+{
+    if (n_shared < 0 || n_shared > kMaxK || k < 1 || k + n_shared > kMaxK || E < 1 || E > kMaxE ||
+        E_phys < 1 || E_phys > kMaxE || R < 1)
+        return MOE_ERR_INVALID_ARG;
+    if (replica_offsets != nullptr &&
+        (replica_ids == nullptr || n_replica_ids < 1 || !aligned(replica_offsets, 4) ||
+         !aligned(replica_ids, 4)))
+        return MOE_ERR_INVALID_ARG;
+    if (replica_offsets == nullptr && E_phys < E + n_shared)
+        return MOE_ERR_INVALID_ARG;
+    const int tpr = (T >= R && T % R == 0) ? T / R : 1;
+    const moe::RouteEx ex{n_shared, shared_weight, replica_offsets, replica_ids, n_replica_ids,
+                          E_phys, tpr, dev_status};
+    return route_dispatch_common(logits, T, E, k, renormalize, R, capacity, x, H, fp8, topk_idx,
+                                 topk_w, expert_counts, expert_src_counts, rank_counts,
+                                 expert_offsets, dispatch_pos, recv_src, recv, recv_scale, rows,
+                                 workspace, ws_bytes, dev_status, stream, &ex);
+}
+
+int moe_route_dispatch_ex_fp8(const float *logits, int T, int E, int k, int renormalize,
+                              int n_shared, float shared_weight, const int32_t *replica_offsets,
+                              const int32_t *replica_ids, int n_replica_ids, int E_phys, int R,
+                              int capacity, const uint16_t *x, int H, int32_t *topk_idx,
+                              float *topk_w, int32_t *expert_counts, int32_t *expert_src_counts,
+                              int32_t *rank_counts, int32_t *expert_offsets, int32_t *dispatch_pos,
+                              int32_t *recv_src, uint8_t *recv_q, float *recv_scale, int64_t rows,
+                              void *workspace, size_t ws_bytes, int32_t *dev_status, void *stream)
+{
+    return route_dispatch_ex(logits, T, E, k, renormalize, n_shared, shared_weight,
+                             replica_offsets, replica_ids, n_replica_ids, E_phys, R, capacity, x, H,
+                             true, topk_idx, topk_w, expert_counts, expert_src_counts, rank_counts,
+                             expert_offsets, dispatch_pos, recv_src, recv_q, recv_scale, rows,
+                             workspace, ws_bytes, dev_status, stream);
+}
+
+int moe_route_dispatch_ex_bf16(const float *logits, int T, int E, int k, int renormalize,
+                               int n_shared, float shared_weight, const int32_t *replica_offsets,
+                               const int32_t *replica_ids, int n_replica_ids, int E_phys, int R,
+                               int capacity, const uint16_t *x, int H, int32_t *topk_idx,
+                               float *topk_w, int32_t *expert_counts, int32_t *expert_src_counts,
+                               int32_t *rank_counts, int32_t *expert_offsets,
+                               int32_t *dispatch_pos, int32_t *recv_src, uint16_t *recv_x,
+                               int64_t rows, void *workspace, size_t ws_bytes, int32_t *dev_status,
+                               void *stream)
+{
+    return route_dispatch_ex(logits, T, E, k, renormalize, n_shared, shared_weight,
+                             replica_offsets, replica_ids, n_replica_ids, E_phys, R, capacity, x, H,
+                             false, topk_idx, topk_w, expert_counts, expert_src_counts, rank_counts,
+                             expert_offsets, dispatch_pos, recv_src, recv_x, nullptr, rows,
+                             workspace, ws_bytes, dev_status, stream);
 }
 
 int moe_quantize_e4m3(const float *v, int64_t n, uint8_t *q, void *stream)

@@ -71,17 +71,20 @@ cudaError_t combine_bf16(const uint16_t *y, const int32_t *dispatch_pos, const f
                          cudaStream_t s);
 
 // Route + layout + dispatch in one cooperative launch (packed or padded
-// layout; plain route).  Workspace bytes depend on the current device's SM
-// count and the kernel's occupancy; 0 = cannot launch.  *ws_too_small is set
-// (and nothing launched) when ws_bytes is below what the geometry needs.
-size_t route_dispatch_workspace_bytes(int T, int k, int E, int R, bool fp8);
+// layout).  E, k: the router's experts and routed slots; with ex the layout
+// sees k + ex->n_shared slots over ex->E_phys experts, as after
+// route_topk(..., ex).  Workspace bytes depend on the current device's SM
+// count (0 = no device); they are given for the layout's (k, E).
+// *ws_too_small is set (and nothing launched) when ws_bytes is below what the
+// geometry needs.
+size_t route_dispatch_workspace_bytes(int T, int k, int E, int R);
 cudaError_t route_dispatch(const float *logits, int T, int E, int k, int renormalize, int R,
                            int capacity, const uint16_t *x, int H, bool fp8, int32_t *topk_idx,
                            float *topk_w, int32_t *expert_counts, int32_t *expert_src_counts,
                            int32_t *rank_counts, int32_t *expert_offsets, int32_t *dispatch_pos,
                            int32_t *recv_src, void *recv, float *recv_scale, int64_t rows,
                            void *workspace, size_t ws_bytes, int32_t *dev_status, cudaStream_t s,
-                           bool *ws_too_small);
+                           bool *ws_too_small, const RouteEx *ex = nullptr);
 
 // Combine with E4M3 rows yq [rows][H] and row-major 1x128 scales ys [rows][H/128].
 cudaError_t combine_fp8(const uint8_t *yq, const float *ys, const int32_t *dispatch_pos,

@@ -109,7 +109,16 @@ struct FusedGeom {
 
 struct FusedArgs {
     const float *logits;
+    int El;  // routed experts (logits per token)
+    int kr;  // routed slots per token; slots kr .. k-1 are the shared experts
     int renormalize;
+    // shared experts and replicas (as moe_route_topk_ex); ex_on = 0: the
+    // chosen logical experts are the layout's experts
+    int ex_on;
+    float shared_weight;
+    const int32_t *replica_offsets;  // [El + n_shared + 1] or nullptr
+    const int32_t *replica_ids;
+    int n_replica_ids;
     const uint4 *x;
     int H;
     int capacity;
@@ -332,14 +341,41 @@ __global__ void __launch_bounds__(kThreads, (NPL <= 12) ? 2 : 1)
         __syncthreads();
         int t0, t1;
         chunk_tokens(G, c, t0, t1);
+        const int src_r = c / G.cpr;  // a chunk's tokens share one source rank
         for (int g = t0 + w; g < t1; g += kWarps) {  // warp-uniform
             int my_e;
             float my_w;
-            route_warp<NPL>(A.logits + static_cast<size_t>(g) * E, E, k, A.renormalize, my_e, my_w);
+            if (A.ex_on)  // uniform; two call sites keep the plain form's registers
+                route_warp<NPL>(A.logits + static_cast<size_t>(g) * A.El, A.El, A.kr,
+                                A.renormalize, my_e, my_w);
+            else
+                route_warp<NPL>(A.logits + static_cast<size_t>(g) * E, E, k, A.renormalize,
+                                my_e, my_w);
             if (lane < k) {
-                A.topk_idx[static_cast<size_t>(g) * k + lane] = my_e;
-                A.topk_w[static_cast<size_t>(g) * k + lane] = my_w;
-                atomicAdd(&h[my_e], 1);
+                int phys = my_e;
+                float wt = my_w;
+                if (A.ex_on) {
+                    // shared experts El .. El + k - kr - 1 after the routed ones;
+                    // every logical expert mapped to the replica of the token's rank
+                    const int l = (lane < A.kr) ? my_e : A.El + (lane - A.kr);
+                    wt = (lane < A.kr) ? my_w : A.shared_weight;
+                    phys = l;
+                    if (A.replica_offsets != nullptr) {
+                        const int a = A.replica_offsets[l], b = A.replica_offsets[l + 1];
+                        if (a < 0 || b <= a || b > A.n_replica_ids)
+                            phys = -1;
+                        else
+                            phys = A.replica_ids[a + src_r % (b - a)];
+                    }
+                    if (phys < 0 || phys >= E) {
+                        report(A.dev_status, MOE_ERR_INVALID_ARG);
+                        phys = -1;
+                    }
+                }
+                A.topk_idx[static_cast<size_t>(g) * k + lane] = phys;
+                A.topk_w[static_cast<size_t>(g) * k + lane] = wt;
+                if (phys >= 0)
+                    atomicAdd(&h[phys], 1);
             }
         }
         __syncthreads();
@@ -741,11 +777,12 @@ int query_resident(KernelFn fn, size_t smem)
     return nsm * per;
 }
 
-// Geometry on the current device, the grid sized from the kernel's occupancy
-// (H = 0: chunks only, for the workspace size).
-bool device_geom(int T, int k, int E, int R, int H, bool fp8, FusedGeom &g, KernelFn &fn)
+// Geometry on the current device, the grid sized from the kernel's occupancy.
+// k and E are the layout's slots per token and experts; El, the logits per
+// token, picks the kernel (logits per lane).
+bool device_geom(int T, int k, int E, int R, int H, bool fp8, int El, FusedGeom &g, KernelFn &fn)
 {
-    fn = fp8 ? pick<true>(E) : pick<false>(E);
+    fn = fp8 ? pick<true>(El) : pick<false>(El);
     FusedGeom probe;
     probe.E = E;
     const int gmax = max_resident(fn, smem_bytes(probe));
@@ -758,12 +795,16 @@ bool device_geom(int T, int k, int E, int R, int H, bool fp8, FusedGeom &g, Kern
 
 }  // namespace
 
-size_t route_dispatch_workspace_bytes(int T, int k, int E, int R, bool fp8)
+size_t route_dispatch_workspace_bytes(int T, int k, int E, int R)
 {
-    FusedGeom g;
-    KernelFn fn;
-    if (!device_geom(T, k, E, R, 0, fp8, g, fn))
+    // Sized for the most CTAs any variant of the kernel can keep resident
+    // (2048 threads per SM / 512): the chunk count only grows with the grid,
+    // so every launch's geometry fits.
+    int dev = 0, nsm = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || nsm < 1)
         return 0;
+    const FusedGeom g = make_geom(T, k, E, R, nsm * (2048 / kThreads), 0);
     return (ws_layout(g).total * sizeof(int32_t) + 255) / 256 * 256;
 }
 
@@ -773,12 +814,14 @@ cudaError_t route_dispatch(const float *logits, int T, int E, int k, int renorma
                            int32_t *rank_counts, int32_t *expert_offsets, int32_t *dispatch_pos,
                            int32_t *recv_src, void *recv, float *recv_scale, int64_t rows,
                            void *workspace, size_t ws_bytes, int32_t *dev_status, cudaStream_t s,
-                           bool *ws_too_small)
+                           bool *ws_too_small, const RouteEx *ex)
 {
     FusedGeom g;
     KernelFn fn;
     *ws_too_small = false;
-    if (!device_geom(T, k, E, R, H, fp8, g, fn))
+    const int kk = k + (ex ? ex->n_shared : 0);   // slots per token
+    const int El = ex ? ex->E_phys : E;           // the layout's experts
+    if (!device_geom(T, kk, El, R, H, fp8, E, g, fn))
         return cudaErrorInvalidConfiguration;
     if (ws_bytes < ws_layout(g).total * sizeof(int32_t)) {
         *ws_too_small = true;
@@ -786,7 +829,14 @@ cudaError_t route_dispatch(const float *logits, int T, int E, int k, int renorma
     }
     FusedArgs a;
     a.logits = logits;
+    a.El = E;
+    a.kr = k;
     a.renormalize = renormalize;
+    a.ex_on = ex ? 1 : 0;
+    a.shared_weight = ex ? ex->shared_weight : 1.0f;
+    a.replica_offsets = ex ? ex->replica_offsets : nullptr;
+    a.replica_ids = ex ? ex->replica_ids : nullptr;
+    a.n_replica_ids = ex ? ex->n_replica_ids : 0;
     a.x = reinterpret_cast<const uint4 *>(x);
     a.H = H;
     a.capacity = capacity;

@@ -377,7 +377,39 @@ int moe_route_dispatch_bf16(const float *logits, int T, int E, int k, int renorm
                             size_t ws_bytes, int32_t *dev_status, void *stream);
 
 /*
- * moe_combine_bf16 -- gather each token's k expert outputs and form the
+ * moe_route_dispatch_ex_fp8 / moe_route_dispatch_ex_bf16 -- the same single
+ * launch with the routing of moe_route_topk_ex (shared experts, replicas):
+ * bit-identical to moe_route_topk_ex(..., tokens_per_rank = T / R), then
+ * moe_dispatch_layout with k + n_shared slots and E_phys experts, then
+ * moe_dispatch_fp8 (or _bf16).  logits stay [T][E] over the routed experts;
+ * topk_idx / topk_w are [T][k + n_shared]; the layout outputs are sized by
+ * E_phys (expert_counts [E_phys], expert_offsets [E_phys + 1],
+ * expert_src_counts [E_phys][R]) and R must divide E_phys.  The table
+ * arguments, their limits and their error behaviour are moe_route_topk_ex's;
+ * a slot that gets -1 is left out of the layout (no row).  The workspace is
+ * the one described above, at least moe_route_dispatch_workspace_bytes(T,
+ * k + n_shared, E_phys, R) bytes, shared with the plain entry points.
+ */
+int moe_route_dispatch_ex_fp8(const float *logits, int T, int E, int k, int renormalize,
+                              int n_shared, float shared_weight, const int32_t *replica_offsets,
+                              const int32_t *replica_ids, int n_replica_ids, int E_phys, int R,
+                              int capacity, const uint16_t *x, int H, int32_t *topk_idx,
+                              float *topk_w, int32_t *expert_counts, int32_t *expert_src_counts,
+                              int32_t *rank_counts, int32_t *expert_offsets, int32_t *dispatch_pos,
+                              int32_t *recv_src, uint8_t *recv_q, float *recv_scale, int64_t rows,
+                              void *workspace, size_t ws_bytes, int32_t *dev_status, void *stream);
+int moe_route_dispatch_ex_bf16(const float *logits, int T, int E, int k, int renormalize,
+                               int n_shared, float shared_weight, const int32_t *replica_offsets,
+                               const int32_t *replica_ids, int n_replica_ids, int E_phys, int R,
+                               int capacity, const uint16_t *x, int H, int32_t *topk_idx,
+                               float *topk_w, int32_t *expert_counts, int32_t *expert_src_counts,
+                               int32_t *rank_counts, int32_t *expert_offsets,
+                               int32_t *dispatch_pos, int32_t *recv_src, uint16_t *recv_x,
+                               int64_t rows, void *workspace, size_t ws_bytes, int32_t *dev_status,
+                               void *stream);
+
+/*
+ * moe_combine_bf16 --gather each token's k expert outputs and form the
  * router-weighted sum.
  * Follows "Efficient and portable mixture-of-experts communication",
  * "Combinação" (the receiver reads the routing table for which row to read

@@ -184,6 +184,33 @@ def test_fused_route_dispatch_rejects_bad_arguments(moe):
                1 << 20, None, None) == moe.MOE_ERR_UNSUPPORTED   # bf16 needs H >= 64
 
 
+def test_fused_route_dispatch_ex_rejects_bad_arguments(moe):
+    f8, f16 = moe.lib.moe_route_dispatch_ex_fp8, moe.lib.moe_route_dispatch_ex_bf16
+    ws = 0x100000
+
+    def call8(T=64, E=8, k=2, ns=1, offs=None, ids=None, nids=0, Ep=10, R=2, cap=0, H=256,
+              rows=192, wsp=ws):
+        return f8(A4, T, E, k, 0, ns, 1.0, offs, ids, nids, Ep, R, cap, A16, H, A4, A4, A4, A4,
+                  A4, A4, A4, A4, A16, A4, rows, wsp, 1 << 20, None, None)
+
+    assert call8(ns=-1) == moe.MOE_ERR_INVALID_ARG
+    assert call8(k=0) == moe.MOE_ERR_INVALID_ARG
+    assert call8(k=9) == moe.MOE_ERR_INVALID_ARG              # k > E
+    assert call8(k=30, E=64, ns=3, Ep=68) == moe.MOE_ERR_INVALID_ARG  # k + n_shared > 32
+    assert call8(Ep=8) == moe.MOE_ERR_INVALID_ARG             # no table: E_phys < E + n_shared
+    assert call8(Ep=1025) == moe.MOE_ERR_INVALID_ARG          # E_phys > 1024
+    assert call8(Ep=9) == moe.MOE_ERR_INVALID_ARG             # R = 2 does not divide E_phys
+    assert call8(offs=A4, ids=None, nids=4) == moe.MOE_ERR_INVALID_ARG  # table without ids
+    assert call8(offs=A4, ids=A4, nids=0) == moe.MOE_ERR_INVALID_ARG
+    assert call8(offs=A4 + 2, ids=A4, nids=4) == moe.MOE_ERR_INVALID_ARG  # misaligned table
+    assert call8(rows=191) == moe.MOE_ERR_INVALID_ARG         # packed rows < T * (k + n_shared)
+    assert call8(cap=4, rows=39) == moe.MOE_ERR_INVALID_ARG   # padded rows < E_phys * cap
+    assert call8(H=264) == moe.MOE_ERR_UNSUPPORTED
+    assert call8(wsp=None) == moe.MOE_ERR_WORKSPACE
+    assert f16(A4, 64, 8, 2, 0, 1, 1.0, None, None, 0, 10, 2, 0, A16, 56, A4, A4, A4, A4, A4, A4,
+               A4, A4, A16, 192, ws, 1 << 20, None, None) == moe.MOE_ERR_UNSUPPORTED
+
+
 def test_combine_fp8_rejects_bad_arguments(moe):
     f = moe.lib.moe_combine_fp8
     assert f(A16, A4, A4, A4, 4, 200, 2, 8, A16, None, None) == moe.MOE_ERR_UNSUPPORTED  # H % 128

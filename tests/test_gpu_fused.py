@@ -79,6 +79,11 @@ def _separate(moe, logits, x, k, R, cap, rows, fp8, renormalize=False):
     """The same step through the separate entry points."""
     E = logits.shape[1]
     idx, w = moe.moe_route_topk(logits, k, renormalize=renormalize)
+    return _separate_from(moe, idx, w, x, E, R, cap, rows, fp8)
+
+
+def _separate_from(moe, idx, w, x, E, R, cap, rows, fp8):
+    """Layout and dispatch of a given route through the separate entry points."""
     lay = moe.moe_dispatch_layout(idx, E, R, capacity=cap, rows=rows)
     got = dict(topk_idx=idx, topk_w=w, **{key: lay[key] for key in LAYOUT_KEYS})
     if fp8:
@@ -387,3 +392,176 @@ def test_fused_random_shapes_match_separate_and_oracle(moe, case):
     sep = _separate(moe, lg, xd, k, R, cap, rows, fp8)
     _assert_same_as_separate(got, sep, fp8, str(case))
     _assert_unfilled_untouched(got, fp8)
+
+
+# ------------------------------------------- shared experts and replicas
+
+def _fused_ex(moe, logits, x, k, R, ex, cap, rows, fp8, renormalize=False, st=None):
+    T = logits.shape[0]
+    out, guards = _out_buffers(T, ex["E_phys"], k + ex["n_shared"], R, x.shape[1], rows, fp8)
+    f = moe.moe_route_dispatch_ex_fp8 if fp8 else moe.moe_route_dispatch_ex_bf16
+    f(logits, x, k, R, n_shared=ex["n_shared"], shared_weight=ex["shared_weight"],
+      replica_offsets=ex["offs"], replica_ids=ex["ids"], E_phys=ex["E_phys"], capacity=cap,
+      rows=rows, renormalize=renormalize, out=out, dev_status=st)
+    torch.cuda.synchronize()
+    _check_guards(guards, rows)
+    return out
+
+
+def _separate_ex(moe, logits, x, k, R, ex, cap, rows, fp8, renormalize=False):
+    """moe_route_topk_ex with T / R tokens per source rank, then the
+    separate layout and dispatch over E_phys experts."""
+    T = logits.shape[0]
+    idx, w = moe.moe_route_topk_ex(logits, k, ex["n_shared"], ex["shared_weight"], ex["offs"],
+                                   ex["ids"], ex["E_phys"], max(1, T // R),
+                                   renormalize=renormalize)
+    return _separate_from(moe, idx, w, x, ex["E_phys"], R, cap, rows, fp8)
+
+
+def _np(t):
+    return None if t is None else t.cpu().numpy()
+
+
+def _check_ex_against_oracle(got, logits, x, k, R, ex, cap, rows, fp8, renormalize, st,
+                             moe, where):
+    T = logits.shape[0]
+    idx_o, w_o, st_o = oracle.route_ex(logits.numpy(), k, ex["n_shared"], ex["shared_weight"],
+                                       _np(ex["offs"]), _np(ex["ids"]), ex["E_phys"],
+                                       max(1, T // R), renormalize=renormalize)
+    lay_o = oracle.layout(idx_o, ex["E_phys"], R, cap, rows)
+    want_st = 0
+    if st_o != oracle.OK:
+        want_st = moe.MOE_ERR_INVALID_ARG
+    elif lay_o["status"] == oracle.ERR_CAPACITY:
+        want_st = moe.MOE_ERR_CAPACITY
+    assert st.item() == want_st, where
+    assert np.array_equal(got["topk_idx"].cpu().numpy(), idx_o), where
+    gw = got["topk_w"].cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(gw - w_o) <= route_w_tol(w_o)), where
+    for key in LAYOUT_KEYS:
+        assert np.array_equal(got[key].cpu().numpy(),
+                              lay_o[key].reshape(got[key].shape)), f"{where}: {key}"
+    filled = lay_o["recv_src"] >= 0
+    x_bits = inputs.bf16_bits(x)
+    if fp8:
+        qo, so = oracle.dispatch_fp8(x_bits, lay_o["dispatch_pos"], rows)
+        assert np.array_equal(got["recv_q"].cpu().numpy()[filled], qo[filled]), where
+        assert np.array_equal(got["recv_scale"].cpu().numpy()[filled].view(np.uint32),
+                              so[filled].view(np.uint32)), where
+    else:
+        want = oracle.dispatch_bf16(x_bits, lay_o["dispatch_pos"], rows)
+        assert np.array_equal(gpu_bits(got["recv_x"])[filled], want[filled]), where
+
+
+def test_fused_ex_on_shared_expert_workload(moe):
+    """The DeepSeek-V3-like workload with a shared expert replicated on every
+    rank: route (routed + shared slots, physical ids), layout over E_phys and
+    FP8 rows against the oracle, and bit-identical to the separate calls."""
+    wl = workload("dsv3_shared")
+    cfg = wl["cfg"]
+    fp8 = cfg.dispatch == "fp8"
+    offs, ids = wl["placement"]
+    ex = dict(n_shared=cfg.n_shared, shared_weight=1.0, offs=to_dev(offs), ids=to_dev(ids),
+              E_phys=cfg.E_phys)
+    logits, x = to_dev(wl["logits"]), to_dev(wl["x"])
+    st = _status()
+    got = _fused_ex(moe, logits, x, cfg.k, cfg.R, ex, wl["cap"], wl["rows"], fp8, st=st)
+    assert st.item() == 0
+    assert np.array_equal(got["topk_idx"].cpu().numpy(), wl["idx"])
+    w = got["topk_w"].cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(w - wl["w"]) <= route_w_tol(wl["w"]))
+    for key in LAYOUT_KEYS:
+        assert np.array_equal(got[key].cpu().numpy(),
+                              wl["layout"][key].reshape(got[key].shape)), key
+    filled = wl["layout"]["recv_src"] >= 0
+    qo, so = oracle.dispatch_fp8(wl["x_bits"], wl["layout"]["dispatch_pos"], wl["rows"])
+    assert np.array_equal(got["recv_q"].cpu().numpy()[filled], qo[filled])
+    assert np.array_equal(got["recv_scale"].cpu().numpy()[filled].view(np.uint32),
+                          so[filled].view(np.uint32))
+    _assert_unfilled_untouched(got, fp8)
+    sep = _separate_ex(moe, logits, x, cfg.k, cfg.R, ex, wl["cap"], wl["rows"], fp8)
+    _assert_same_as_separate(got, sep, fp8, "dsv3_shared")
+
+
+def _random_ex_cases(n, seed):
+    """Seeded random shapes with random replica tables: each logical expert
+    (routed and shared) gets 1-3 replicas drawn from E_phys physical ids (a
+    multiple of R, some ids unused, some shared between logical experts)."""
+    rng = np.random.default_rng(seed)
+    cases = []
+    while len(cases) < n:
+        E = int(rng.choice([4, 8, 16, 40, 64, 256, 384]))
+        n_shared = int(rng.integers(0, 3))
+        k = int(rng.integers(1, min(E, 32 - n_shared) + 1))
+        R = int(rng.choice([1, 2, 4, 8]))
+        n_log = E + n_shared
+        E_phys = min(1024, -(-(n_log + int(rng.integers(0, n_log + 1))) // R) * R)
+        if k + n_shared > E_phys or E_phys > 1024:
+            continue
+        Tr = int(rng.choice([1, 3, 16, 50, 256]))
+        T = Tr * R
+        reps = rng.integers(1, 4, size=n_log)
+        offs = np.concatenate([[0], np.cumsum(reps)]).astype(np.int32)
+        ids = rng.integers(0, E_phys, size=int(offs[-1])).astype(np.int32)
+        fp8 = bool(rng.integers(0, 2))
+        H = int(rng.choice([128, 256])) if fp8 else int(rng.choice([64, 136]))
+        cap = 0 if rng.random() < 0.6 else int(rng.integers(1, max(2, T * (k + n_shared) // E_phys + 3)))
+        sw = float(rng.choice([1.0, 0.5, 0.8125]))
+        renorm = bool(rng.integers(0, 2))
+        cases.append((T, H, E, k, R, n_shared, E_phys, offs, ids, cap, fp8, sw, renorm))
+    return cases
+
+
+_EX_CASES = _random_ex_cases(12, 77)
+
+
+@pytest.mark.parametrize("i", range(len(_EX_CASES)),
+                         ids=lambda i: "T{}_E{}_k{}+{}_Ep{}_R{}_cap{}_{}".format(
+                             _EX_CASES[i][0], _EX_CASES[i][2], _EX_CASES[i][3], _EX_CASES[i][5],
+                             _EX_CASES[i][6], _EX_CASES[i][4], _EX_CASES[i][9],
+                             "fp8" if _EX_CASES[i][10] else "bf16"))
+def test_fused_ex_random_replica_tables(moe, i):
+    T, H, E, k, R, n_shared, E_phys, offs, ids, cap, fp8, sw, renorm = _EX_CASES[i]
+    logits, x = inputs.make_random_case(T, H, E, k, seed=500 + i)
+    ex = dict(n_shared=n_shared, shared_weight=sw, offs=to_dev(torch.from_numpy(offs)),
+              ids=to_dev(torch.from_numpy(ids)), E_phys=E_phys)
+    idx_o, _, _ = oracle.route_ex(logits.numpy(), k, n_shared, sw, offs, ids, E_phys, T // R)
+    rows = oracle.layout(idx_o, E_phys, R, cap)["recv_src"].shape[0]
+    lg, xd = to_dev(logits), to_dev(x)
+    st = _status()
+    got = _fused_ex(moe, lg, xd, k, R, ex, cap, rows, fp8, renormalize=renorm, st=st)
+    _check_ex_against_oracle(got, logits, x, k, R, ex, cap, rows, fp8, renorm, st, moe,
+                             str(_EX_CASES[i][:7]))
+    _assert_unfilled_untouched(got, fp8)
+    sep = _separate_ex(moe, lg, xd, k, R, ex, cap, rows, fp8, renormalize=renorm)
+    _assert_same_as_separate(got, sep, fp8, str(_EX_CASES[i][:7]))
+
+
+def test_fused_ex_without_table_and_bad_table(moe):
+    """No replica table: logical ids are the physical ones.  Then a table
+    entry past E_phys: that slot gets -1 and no row, MOE_ERR_INVALID_ARG is
+    reported, and everything else matches the oracle."""
+    T, H, E, k, R = 96, 256, 16, 3, 4
+    logits, x = inputs.make_random_case(T, H, E, k, seed=41)
+    lg, xd = to_dev(logits), to_dev(x)
+    ex = dict(n_shared=2, shared_weight=0.75, offs=None, ids=None, E_phys=20)
+    st = _status()
+    got = _fused_ex(moe, lg, xd, k, R, ex, 0, T * 5, True, st=st)
+    _check_ex_against_oracle(got, logits, x, k, R, ex, 0, T * 5, True, False, st, moe, "no table")
+    sep = _separate_ex(moe, lg, xd, k, R, ex, 0, T * 5, True)
+    _assert_same_as_separate(got, sep, True, "no table")
+
+    offs, ids = [0], []
+    for l in range(E + 2):
+        ids += [l] if l != 5 else [5, 18, 19]
+        offs.append(len(ids))
+    offs, ids = np.array(offs, np.int32), np.array(ids, np.int32)
+    bad = ids.copy()
+    bad[offs[7]] = 24                                # expert 7's replica: one past E_phys
+    ex = dict(n_shared=2, shared_weight=0.75, offs=to_dev(torch.from_numpy(offs)),
+              ids=to_dev(torch.from_numpy(bad)), E_phys=24)
+    st = _status()
+    got = _fused_ex(moe, lg, xd, k, R, ex, 0, T * 5, False, st=st)
+    assert bool((got["topk_idx"] == -1).any())
+    _check_ex_against_oracle(got, logits, x, k, R, ex, 0, T * 5, False, False, st, moe,
+                             "bad table")
