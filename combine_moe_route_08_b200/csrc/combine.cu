@@ -140,7 +140,7 @@ __device__ __forceinline__ float2 fmul2_rn(float2 a, float2 b)
 // takes tpb consecutive tokens, their row indices and weights fetched in one
 // go (measured at H = 7168: one token per CTA 67 us, four 59 us for dsv3).
 template <int KREG>
-__global__ void __launch_bounds__(kFp8Threads, 2)
+__global__ void __launch_bounds__(kFp8Threads, KREG <= 9 ? 2 : 1)
     k_combine_fp8(const uint4 *__restrict__ yq, const float *__restrict__ ys,
                   const int32_t *__restrict__ dispatch_pos, const float *__restrict__ topk_w, int T,
                   int H, int k, int tpb, int64_t rows, uint4 *__restrict__ out,
@@ -254,7 +254,13 @@ cudaError_t combine_fp8(const uint8_t *yq, const float *ys, const int32_t *dispa
     if (k <= 4)
         return launch_pdl(k_combine_fp8<4>, grid, block, 0, s, q, ys, dispatch_pos, topk_w, T, H,
                           k, tpb, rows, ov, dev_status);
-    return launch_pdl(k_combine_fp8<8>, grid, block, 0, s, q, ys, dispatch_pos, topk_w, T, H, k,
+    if (k <= 8)
+        return launch_pdl(k_combine_fp8<8>, grid, block, 0, s, q, ys, dispatch_pos, topk_w, T, H,
+                          k, tpb, rows, ov, dev_status);
+    if (k == 9)
+        return launch_pdl(k_combine_fp8<9>, grid, block, 0, s, q, ys, dispatch_pos, topk_w, T, H,
+                          k, tpb, rows, ov, dev_status);
+    return launch_pdl(k_combine_fp8<16>, grid, block, 0, s, q, ys, dispatch_pos, topk_w, T, H, k,
                       tpb, rows, ov, dev_status);
 }
 
@@ -272,8 +278,14 @@ cudaError_t combine_bf16(const uint16_t *y, const int32_t *dispatch_pos, const f
     if (k <= 4)
         return launch_pdl(k_combine_bf16<4>, grid, block, 0, s, yv, dispatch_pos, topk_w, nvec, k,
                           rows, ov, dev_status);
-    return launch_pdl(k_combine_bf16<8>, grid, block, 0, s, yv, dispatch_pos, topk_w, nvec, k, rows,
-                      ov, dev_status);
+    if (k <= 8)
+        return launch_pdl(k_combine_bf16<8>, grid, block, 0, s, yv, dispatch_pos, topk_w, nvec, k,
+                          rows, ov, dev_status);
+    if (k == 9)  // eight routed experts and a shared one
+        return launch_pdl(k_combine_bf16<9>, grid, block, 0, s, yv, dispatch_pos, topk_w, nvec, k,
+                          rows, ov, dev_status);
+    return launch_pdl(k_combine_bf16<16>, grid, block, 0, s, yv, dispatch_pos, topk_w, nvec, k,
+                      rows, ov, dev_status);
 }
 
 }  // namespace moe

@@ -482,8 +482,32 @@ def test_combine_fp8_parity_prefill_sampled(moe):
     assert check_combine(gpu_bits(out)[tokens], acc, out_o, "prefill fp8") == 1.0
 
 
-@pytest.mark.parametrize("k,T,H", [(1, 37, 128), (3, 37, 128), (8, 37, 128), (11, 37, 128),
-                                   (32, 37, 128), (8, 4099, 128), (2, 9001, 128),
+@pytest.mark.parametrize("k,T,H", [(1, 37, 64), (2, 37, 7168), (4, 50, 136), (8, 37, 1024),
+                                   (9, 37, 7168), (9, 1000, 512), (12, 37, 256), (16, 37, 256),
+                                   (17, 37, 256), (32, 37, 264)])
+def test_combine_bf16_k_sweep(moe, k, T, H):
+    """Every register-held row count of the bf16 combine (k up to 2, 4, 8,
+    9, 16, and beyond 16 with the rest read in order), -1 slots, ragged H
+    (passes that do not fill the CTA), against the oracle within 1 bf16 ulp
+    and bit-identical to its bf16 rounding."""
+    rng = np.random.default_rng(90 + k + T + H)
+    rows = 300
+    y_bits = inputs.bf16_bits(torch.randn(rows, H, generator=torch.Generator().manual_seed(k))
+                              .to(torch.bfloat16))
+    pos = rng.integers(-1, rows, (T, k)).astype(np.int32)
+    w = rng.random((T, k)).astype(np.float32)
+    acc, out_o = oracle.combine(y_bits, pos, w)
+    st = _status()
+    y = to_dev(inputs.bits_to_bf16(y_bits))
+    out = moe.moe_combine_bf16(y, to_dev(pos), to_dev(w), dev_status=st)
+    torch.cuda.synchronize()
+    assert check_combine(gpu_bits(out), acc, out_o, f"k={k} T={T} H={H}") == 1.0
+    assert st.item() == 0
+
+
+@pytest.mark.parametrize("k,T,H", [(1, 37, 128), (3, 37, 128), (8, 37, 128), (9, 37, 128),
+                                   (11, 37, 128), (16, 37, 128), (17, 37, 128),
+                                   (32, 37, 128), (8, 4099, 128), (2, 9001, 128), (9, 2100, 1024),
                                    (1, 37, 512), (8, 300, 512), (11, 37, 512), (32, 37, 512),
                                    (8, 4099, 1024)])
 @pytest.mark.parametrize("scale_offset", [0, 1])
