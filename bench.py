@@ -611,8 +611,36 @@ def run_ours(args) -> None:
         dcev = timed_replays(g_dcG, g_dc1, K)
         s.synchronize()
     local_dc = ms_per(dcev, K)
-    ms = max_over_ranks([local_step, local_dc, *[float(v) for v in stage_ms]], world, dev)
-    ms_step, ms_dc, ms_route, ms_layout, ms_dispatch, ms_combine = ms
+
+    # eager: the same calls launched one by one from Python, no graph -- the
+    # cost a caller that does not capture graphs pays (launch latency included)
+    K3 = min(K, 200)
+    with torch.cuda.stream(s):
+        for i in range(3):
+            flush(i)
+            step()
+        s.synchronize()
+        eev = []
+        if flush_needed:
+            for i in range(K3):
+                flush(i)
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(s)
+                step()
+                b.record(s)
+                eev.append((a, b))
+        else:
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(s)
+            for i in range(K3):
+                step()
+            b.record(s)
+            eev.append((a, b))
+        s.synchronize()
+    local_eager = ms_per(eev, K3)
+    ms = max_over_ranks([local_step, local_dc, local_eager, *[float(v) for v in stage_ms]], world,
+                        dev)
+    ms_step, ms_dc, ms_eager, ms_route, ms_layout, ms_dispatch, ms_combine = ms
     del g_step1, g_stepG, g_dc1, g_dcG
 
     # ---- end to end through the public API, host buffers in and out ----
@@ -705,6 +733,9 @@ def run_ours(args) -> None:
                                   f"{G} consecutive step(s)")},
             "us_per_layer": ms_step * 1e3,
             "stages_us": stages,
+            "eager": {"us_per_step": ms_eager * 1e3, "steps": K3,
+                      "how": "the same C ABI calls launched one by one, no CUDA graph, "
+                             "events around the steps (L2 as for the headline)"},
             "dispatch_combine": {"us": dc_ms * 1e3, "bytes": dc_bytes,
                                  "how": dc_how,
                                  "gbs": dc_bytes / (dc_ms * 1e-3) / 1e9,
