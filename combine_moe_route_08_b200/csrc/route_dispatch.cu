@@ -51,6 +51,7 @@
 // and records MOE_ERR_TIMEOUT; the launch is cooperative, so the driver
 // guarantees that every CTA is resident.
 #include <algorithm>
+#include <type_traits>
 #include <mutex>
 #include <vector>
 
@@ -90,7 +91,8 @@ __host__ __device__ inline int kPosOffset(int E)
 {
     return (kWarps * E + 2 * E + 1 + kWarps + 1 + 31) / 32 * 32;
 }
-constexpr int kSumBatch = 12;                      // table loads in flight per thread
+constexpr int kSumBatch = 12;                      // 4-byte table loads in flight per thread
+constexpr int kSumBatch4 = 4;                      // 16-byte table loads in flight per thread
 
 constexpr int kMaxSteps = 8;                       // 32-slot steps per warp
 constexpr int kChunkSlots = kThreads * kMaxSteps;  // 4096 slots per chunk at most
@@ -270,42 +272,69 @@ __device__ void sum_rows(const int32_t *tab, int E, int r0, int r1, int P, int32
     __syncthreads();
 }
 
-// One pass of loads for the first chunk a CTA places: over the rank rows
-// rt[0..R) (every one adds to the expert total; those of ranks < rb also to
-// the chunk's base) and the hist rows [h0, h1) of the earlier chunks of its
-// rank (base only).  The R + (h1 - h0) rows are split into P contiguous
-// shares per expert column; each thread keeps kSumBatch loads in flight.
-// tot_out / bef_out: [P][E].  Every thread calls it; ends with
+// Column sums of the int32 tables for placing a chunk, in one pass of loads:
+// rows [0, R) of rt (each adds to the expert total; those of ranks < rb also
+// to the chunk's base) and rows [h0, h1) of hist (base only).  The
+// R + (h1 - h0) rows are split into Q contiguous shares per column, Q <= Qmax
+// as large as the CTA's threads allow.  V = 4: a thread reads four columns
+// per 16-byte load (needs E % 4 == 0; rows are then 16-byte aligned); V = 1:
+// one column per 4-byte load.  Each thread keeps B loads in flight.  Writes
+// tot_out / bef_out [Q][E] and returns Q.  Every thread calls it; ends with
 // __syncthreads().
-__device__ void sum_totals_and_base(const int32_t *rt, int R, int rb, const int32_t *hist, int h0,
-                                    int h1, int E, int P, int32_t *tot_out, int32_t *bef_out)
+template <int V, int B>
+__device__ int sum_totals_and_base(const int32_t *rt, int R, int rb, const int32_t *hist, int h0,
+                                   int h1, int E, int Qmax, int32_t *tot_out, int32_t *bef_out)
 {
+    using Vec = typename std::conditional<V == 4, int4, int>::type;
     const int n = R + (h1 - h0);
-    const int per = (n + P - 1) / P;
-    for (int idx = threadIdx.x; idx < P * E; idx += kThreads) {
-        const int x = idx % E, part = idx / E;
+    const int EV = E / V;
+    const int Q = max(1, min(min(kThreads / EV, Qmax), n));
+    const int per = (n + Q - 1) / Q;
+    for (int idx = threadIdx.x; idx < Q * EV; idx += kThreads) {
+        const int xv = idx % EV, part = idx / EV;
         const int b = part * per, e = min(n, b + per);
-        int total = 0, before = 0;
-        for (int j0 = b; j0 < e; j0 += kSumBatch) {
-            int val[kSumBatch];
+        int total[V], before[V];
 #pragma unroll
-            for (int u = 0; u < kSumBatch; ++u) {
+        for (int q = 0; q < V; ++q)
+            total[q] = before[q] = 0;
+        for (int j0 = b; j0 < e; j0 += B) {
+            Vec val[B];
+#pragma unroll
+            for (int u = 0; u < B; ++u) {
                 const int j = j0 + u;
-                const int32_t *src = (j < R) ? rt + static_cast<size_t>(j) * E
+                const int32_t *row = (j < R) ? rt + static_cast<size_t>(j) * E
                                              : hist + static_cast<size_t>(h0 + j - R) * E;
-                val[u] = (j < e) ? __ldcg(src + x) : 0;
+                val[u] = (j < e) ? __ldcg(reinterpret_cast<const Vec *>(row) + xv) : Vec{};
             }
 #pragma unroll
-            for (int u = 0; u < kSumBatch; ++u) {
+            for (int u = 0; u < B; ++u) {  // rows past e hold zeros
                 const int j = j0 + u;
-                total += (j < R) ? val[u] : 0;
-                before += (j < rb || j >= R) ? val[u] : 0;
+                const int *vv = reinterpret_cast<const int *>(&val[u]);
+#pragma unroll
+                for (int q = 0; q < V; ++q) {
+                    total[q] += (j < R) ? vv[q] : 0;
+                    before[q] += (j < rb || j >= R) ? vv[q] : 0;
+                }
             }
         }
-        tot_out[part * E + x] = total;
-        bef_out[part * E + x] = before;
+#pragma unroll
+        for (int q = 0; q < V; ++q) {
+            tot_out[part * E + V * xv + q] = total[q];
+            bef_out[part * E + V * xv + q] = before[q];
+        }
     }
     __syncthreads();
+    return Q;
+}
+
+__device__ __forceinline__ int sum_totals_and_base(const int32_t *rt, int R, int rb,
+                                                   const int32_t *hist, int h0, int h1, int E,
+                                                   int Qmax, int32_t *tot_out, int32_t *bef_out)
+{
+    if (E % 4 == 0)  // CTA-uniform
+        return sum_totals_and_base<4, kSumBatch4>(rt, R, rb, hist, h0, h1, E, Qmax, tot_out,
+                                                  bef_out);
+    return sum_totals_and_base<1, kSumBatch>(rt, R, rb, hist, h0, h1, E, Qmax, tot_out, bef_out);
 }
 
 template <int NPL, bool FP8>
@@ -425,13 +454,14 @@ __global__ void __launch_bounds__(kThreads, (NPL <= 12) ? 2 : 1)
             e_first[s] = (c_first < G.nchunks && i < w1) ? __ldcg(A.topk_idx + i) : -1;
         }
     }
-    const int P = max(1, min(kThreads / E, kWarps / 2));  // 2 * P rows of wh used below
-    sum_totals_and_base(rt, R, r_first, hist, h0_first, h1_first, E, P, wh, wh + P * E);
+    constexpr int kQ = kWarps / 2;  // shares per column: totals in wh rows [0, kQ), bases after
+    const int Q1 = sum_totals_and_base(rt, R, r_first, hist, h0_first, h1_first, E, kQ, wh,
+                                       wh + kQ * E);
     for (int x = tid; x < E; x += kThreads) {
         int total = 0, before = 0;
-        for (int part = 0; part < P; ++part) {
+        for (int part = 0; part < Q1; ++part) {
             total += wh[part * E + x];
-            before += wh[(P + part) * E + x];
+            before += wh[(kQ + part) * E + x];
         }
         off[x] = total;
         chb[x] = before;
@@ -489,6 +519,7 @@ __global__ void __launch_bounds__(kThreads, (NPL <= 12) ? 2 : 1)
             }
             // base of the chunk inside each expert: slots of earlier ranks
             // (rank rows 0..r-1), then of the earlier chunks of its rank
+            const int P = max(1, min(kThreads / E, kWarps / 2));
             sum_rows(rt, E, 0, r, P, wh);
             sum_rows(hist, E, cfirst, c, P, wh + P * E);
             for (int x = tid; x < E; x += kThreads) {
