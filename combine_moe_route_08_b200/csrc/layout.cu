@@ -37,6 +37,7 @@
 // The warp-level pieces (equality masks, per-warp histograms and bases, the
 // block scan) are in layout_dev.cuh.
 #include <algorithm>
+#include <type_traits>
 
 #include "common.cuh"
 #include "kernels.cuh"
@@ -50,7 +51,8 @@ constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
 constexpr int kMaxSteps = 8;                       // 32-slot steps per warp
 constexpr int kChunkSlots = kThreads * kMaxSteps;  // 8192
-constexpr int kColBatch = 16;                      // histogram loads in flight per thread
+constexpr int kColBatch = 16;                      // 4-byte histogram loads in flight per thread
+constexpr int kColBatch4 = 6;                      // 16-byte histogram loads in flight per thread
 
 __device__ __forceinline__ void chunk_tokens(const LayoutGeom &G, int c, int &t0, int &t1)
 {
@@ -121,6 +123,59 @@ __global__ void __launch_bounds__(kThreads)
     pdl_trigger();
 }
 
+// Histogram columns for chunk c of rank r (chunks [r0, r1) of that rank):
+// slots of each expert in earlier chunks (before), in all chunks (total), in
+// the rank's chunks (mine) and in chunks of earlier ranks (rstart).  P
+// threads per column group each sum a contiguous share of the n chunk rows;
+// V = 4 reads four experts per 16-byte load (E % 4 == 0, rows 16-byte
+// aligned), V = 1 one per 4-byte load; B loads in flight per thread.  Share
+// `part` writes rows 4*part .. 4*part+3 of wh (before, total, mine, rstart).
+template <int V, int B>
+__device__ __forceinline__ void column_sums(const int32_t *__restrict__ ws_hist, int n, int c, int r0,
+                                            int r1, int E, int P, int32_t *wh)
+{
+    using Vec = typename std::conditional<V == 4, int4, int>::type;
+    const int EV = E / V;
+    const int xv = threadIdx.x % EV, part = threadIdx.x / EV;
+    if (part >= P)
+        return;
+    const int per = ceil_div(n, P);
+    const int cb = part * per, ce = min(n, cb + per);
+    int before[V], total[V], mine[V], rstart[V];
+#pragma unroll
+    for (int q = 0; q < V; ++q)
+        before[q] = total[q] = mine[q] = rstart[q] = 0;
+    for (int c0 = cb; c0 < ce; c0 += B) {
+        Vec v[B];
+#pragma unroll
+        for (int u = 0; u < B; ++u)
+            v[u] = (c0 + u < ce)
+                       ? __ldg(reinterpret_cast<const Vec *>(ws_hist + static_cast<size_t>(c0 + u) * E) +
+                               xv)
+                       : Vec{};
+#pragma unroll
+        for (int u = 0; u < B; ++u) {
+            const int cc = c0 + u;
+            const int *vv = reinterpret_cast<const int *>(&v[u]);
+#pragma unroll
+            for (int q = 0; q < V; ++q) {
+                before[q] += (cc < c) ? vv[q] : 0;
+                rstart[q] += (cc < r0) ? vv[q] : 0;
+                total[q] += vv[q];
+                mine[q] += (cc >= r0 && cc < r1) ? vv[q] : 0;
+            }
+        }
+    }
+#pragma unroll
+    for (int q = 0; q < V; ++q) {
+        const int x = V * xv + q;
+        wh[(4 * part) * E + x] = before[q];
+        wh[(4 * part + 1) * E + x] = total[q];
+        wh[(4 * part + 2) * E + x] = mine[q];
+        wh[(4 * part + 3) * E + x] = rstart[q];
+    }
+}
+
 __global__ void __launch_bounds__(kThreads)
     k_layout_assign(const int32_t *__restrict__ topk_idx, LayoutGeom G, int capacity, int64_t rows,
                     const int32_t *__restrict__ ws_hist, int32_t *__restrict__ expert_counts,
@@ -145,8 +200,10 @@ __global__ void __launch_bounds__(kThreads)
     int e[kMaxSteps];
     load_run(topk_idx, w0, w1, e);  // in flight while the columns are summed
 
-    for (int x = threadIdx.x + 4 * max(1, min(kThreads / E, kWarps / 4)) * E; x < kWarps * E;
-         x += kThreads)
+    // shares per column: as many as the threads allow (rows 4 * P of wh)
+    const bool vec = (E % 4 == 0);
+    const int P = max(1, min(kThreads / (vec ? E / 4 : E), kWarps / 4));
+    for (int x = threadIdx.x + 4 * P * E; x < kWarps * E; x += kThreads)
         wh[x] = 0;
 
     // histogram columns: base of this chunk inside each expert (earlier
@@ -155,34 +212,11 @@ __global__ void __launch_bounds__(kThreads)
     // part of the chunks (coalesced over experts); the parts meet in shared
     // memory (the per-warp rows, not yet used).
     const int n = G.nchunks;
-    const int P = max(1, min(kThreads / E, kWarps / 4));
     const int r = c / G.cpr;
-    {
-        const int x = threadIdx.x % E, part = threadIdx.x / E;
-        if (part < P) {
-            const int per = ceil_div(n, P);
-            const int cb = part * per, ce = min(n, cb + per);
-            int before = 0, total = 0, mine = 0, rstart = 0;
-            for (int c0 = cb; c0 < ce; c0 += kColBatch) {
-                int v[kColBatch];
-#pragma unroll
-                for (int u = 0; u < kColBatch; ++u)
-                    v[u] = (c0 + u < ce) ? __ldg(ws_hist + static_cast<size_t>(c0 + u) * E + x) : 0;
-#pragma unroll
-                for (int u = 0; u < kColBatch; ++u) {
-                    const int cc = c0 + u;
-                    before += (cc < c) ? v[u] : 0;
-                    rstart += (cc < r * G.cpr) ? v[u] : 0;
-                    total += v[u];
-                    mine += (cc >= r * G.cpr && cc < (r + 1) * G.cpr) ? v[u] : 0;
-                }
-            }
-            wh[(4 * part) * E + x] = before;
-            wh[(4 * part + 1) * E + x] = total;
-            wh[(4 * part + 2) * E + x] = mine;
-            wh[(4 * part + 3) * E + x] = rstart;
-        }
-    }
+    if (vec)  // CTA-uniform
+        column_sums<4, kColBatch4>(ws_hist, n, c, r * G.cpr, (r + 1) * G.cpr, E, P, wh);
+    else
+        column_sums<1, kColBatch>(ws_hist, n, c, r * G.cpr, (r + 1) * G.cpr, E, P, wh);
     __syncthreads();
     for (int x = threadIdx.x; x < E; x += kThreads) {
         int before = 0, total = 0, mine = 0, rstart = 0;
