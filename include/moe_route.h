@@ -62,7 +62,7 @@ extern "C" {
 typedef enum moe_status {
     MOE_OK = 0,
     MOE_ERR_INVALID_ARG = 1, /* bad size, NULL or misaligned pointer, bad id/row */
-    MOE_ERR_UNSUPPORTED = 2, /* valid request this build does not support (fp8 with H % 128 != 0) */
+    MOE_ERR_UNSUPPORTED = 2, /* valid request the library does not support (fp8 with H % 128 != 0) */
     MOE_ERR_CAPACITY = 3,    /* padded layout: a slot beyond its expert's capacity was dropped */
     MOE_ERR_WORKSPACE = 4,   /* workspace too small or misaligned */
     MOE_ERR_TIMEOUT = 5,     /* a bounded wait inside a kernel gave up */
