@@ -99,6 +99,7 @@ __global__ void __launch_bounds__(kThreads)
     warp_run(G, c, w0, w1);
     for (int x = threadIdx.x; x < E; x += kThreads)
         h[x] = 0;
+    pdl_trigger();  // the next kernel may take idle SM slots now; it waits for this one
     pdl_wait();
     int e[kMaxSteps];
     load_run(topk_idx, w0, w1, e);
@@ -120,7 +121,6 @@ __global__ void __launch_bounds__(kThreads)
     __syncthreads();
     for (int x = threadIdx.x; x < E; x += kThreads)
         ws_hist[static_cast<size_t>(c) * E + x] = h[x];
-    pdl_trigger();
 }
 
 // Histogram columns for chunk c of rank r (chunks [r0, r1) of that rank):
@@ -196,6 +196,7 @@ __global__ void __launch_bounds__(kThreads)
 
     int64_t w0, w1;
     warp_run(G, c, w0, w1);
+    pdl_trigger();  // the next kernel may take idle SM slots now; it waits for this one
     pdl_wait();
     int e[kMaxSteps];
     load_run(topk_idx, w0, w1, e);  // in flight while the columns are summed
@@ -316,7 +317,6 @@ __global__ void __launch_bounds__(kThreads)
         for (int64_t r = static_cast<int64_t>(E) * capacity + first; r < rows; r += stride)
             recv_src[r] = -1;
     }
-    pdl_trigger();
 }
 
 size_t assign_smem_bytes(int E) { return (static_cast<size_t>(kWarps + 3) * E + 1 + kWarps + 1) * sizeof(int32_t); }

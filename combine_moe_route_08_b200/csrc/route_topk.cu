@@ -29,6 +29,9 @@ __global__ void __launch_bounds__(kRouteWarps * 32)
         return;  // warp-uniform
     }
     const float *row = logits + static_cast<size_t>(g) * E;
+    // release the next kernel at once: it still waits for this one to finish
+    // before reading, so its CTAs only take idle SM slots early
+    pdl_trigger();
     pdl_wait();
 
     int my_e;
@@ -62,7 +65,6 @@ __global__ void __launch_bounds__(kRouteWarps * 32)
             topk_w[static_cast<size_t>(g) * kk + lane] = wt;
         }
     }
-    pdl_trigger();
 }
 
 template <int NPL>
