@@ -51,8 +51,13 @@ def test_route_parity(moe, name, renormalize):
     assert np.array_equal(idx.cpu().numpy(), idx_o)
     w = w.cpu().numpy()
     err = np.abs(w.astype(np.float64) - w_o)
-    assert np.all(err <= route_w_tol(w_o))
-    print(f"{name}: max weight error {np.max(err / ulp_f32(w_o)):.2f} fp32 ulp")
+    assert np.all(err <= route_w_tol(w_o))      # the proven bound (7u of p, + the oracle's u)
+    # the acceptance rule stated for the weights, 4 fp32 ulps of the oracle's
+    # weight: not implied by the relative bound at the top of a binade, so
+    # checked as measured on these seeded inputs (the maximum is 3 ulps)
+    ulps = err / ulp_f32(w_o)
+    assert np.all(ulps <= 4.0), f"{name}: {np.max(ulps):.2f} ulp"
+    print(f"{name}: max weight error {np.max(ulps):.2f} fp32 ulp")
 
 
 # ----------------------------------------------------------------- layout
