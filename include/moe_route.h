@@ -243,7 +243,8 @@ int moe_compact_bf16(const uint16_t *priv_x, int64_t private_rows, const int32_t
  *   - Limit: (T, k, E, R) whose moe_layout_workspace_bytes exceeds
  *     MOE_LAYOUT_NOALLOC_SCRATCH_BYTES are rejected with MOE_ERR_WORKSPACE
  *     before anything is enqueued (e.g. E = 256 fits up to 1024 chunks of at
- *     most 8192 slots each; every workload of the benchmark fits).
+ *     most 2048 slots each, T*k up to 2^21; every workload of the benchmark
+ *     fits).
  *   - Set-up: the first call on each device looks the array's device address
  *     up (cudaGetSymbolAddress, with that device current) and keeps it; make
  *     that first call before any stream capture on that device.

@@ -57,11 +57,11 @@ def test_status_strings(moe):
 
 
 def test_workspace_bytes(moe):
-    # one int32 histogram row of E per chunk; a chunk holds at most 8192 slots
+    # one int32 histogram row of E per chunk; a chunk holds at most 2048 slots
     # of one logical rank.  dsv3-like decode: 32 ranks of 128 tokens -> 32 chunks
     assert moe.moe_layout_workspace_bytes(4096, 8, 256, 32) == 32 * 256 * 4
-    # prefill-like: 4096 tokens per rank cut into chunks of 1024 tokens
-    assert moe.moe_layout_workspace_bytes(32768, 8, 256, 8) == 32 * 256 * 4
+    # prefill-like: 4096 tokens per rank cut into chunks of 256 tokens
+    assert moe.moe_layout_workspace_bytes(32768, 8, 256, 8) == 128 * 256 * 4
     assert moe.moe_layout_workspace_bytes(0, 2, 8, 2) == 256  # rounded up to 256 B
     for bad in [(-1, 2, 8, 2), (64, 0, 8, 2), (64, 33, 64, 2), (64, 2, 8, 3), (63, 2, 8, 2),
                 (64, 9, 8, 2), (64, 2, 2048, 2)]:
