@@ -101,40 +101,54 @@ __device__ __forceinline__ void route_warp(const float *__restrict__ row, int E,
             key[i] = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
         }
     }
-    // Each lane keeps its best key and that key's slot (the lowest slot among
-    // equal keys); a round is one warp max of the lanes' bests, one warp min
-    // of the expert ids holding it, and a rescan by the winning lane alone.
-    // The chosen logit is read back from the winning key (the map is
-    // invertible; -0 comes back as +0, which gives the same softmax terms).
-    uint32_t bk = 0u;
-    int bi = 0;
+    // Each lane keeps its best key and slot and, while known, its second
+    // best (order: key descending, slot ascending; the lowest slot among
+    // equal keys first).  A round is one warp max of the lanes' bests and one
+    // warp min of the expert ids holding it; the winning lane then promotes
+    // its second best, and only a lane that wins again with no second left
+    // rescans its remaining keys (bit i of `gone`: slot i taken or past E).
+    // With k = 8 over 32 lanes most rounds need no rescan.  The chosen logit
+    // is read back from the winning key (the map is invertible; -0 comes back
+    // as +0, which gives the same softmax terms).
+    uint32_t b1 = 0u, b2 = 0u;  // best and second-best key (0: none)
+    int i1 = 0, i2 = 0;
+    auto top2 = [&]() {
+        b1 = 0u;
+        b2 = 0u;
+        i1 = 0;
+        i2 = 0;
 #pragma unroll
-    for (int i = 0; i < NPL; ++i)
-        if (key[i] > bk) {
-            bk = key[i];
-            bi = i;
+        for (int i = 0; i < NPL; ++i) {
+            const uint32_t kk = ((gone >> i) & 1u) ? 0u : key[i];
+            if (kk > b1) {
+                b2 = b1;
+                i2 = i1;
+                b1 = kk;
+                i1 = i;
+            } else if (kk > b2) {
+                b2 = kk;
+                i2 = i;
+            }
         }
+    };
+    top2();
     my_e = 0;
     float my_v = 0.0f;
     float vmax = 0.0f;
     for (int j = 0; j < k; ++j) {
-        const uint32_t m = __reduce_max_sync(kFullMask, bk);
-        const uint32_t cand = (bk == m) ? static_cast<uint32_t>(bi * 32 + lane) : 0xffffffffu;
+        const uint32_t m = __reduce_max_sync(kFullMask, b1);
+        const uint32_t cand = (b1 == m) ? static_cast<uint32_t>(i1 * 32 + lane) : 0xffffffffu;
         const uint32_t e = __reduce_min_sync(kFullMask, cand);
         const uint32_t u = (m & 0x80000000u) ? (m & 0x7fffffffu) : ~m;
         const float ve = __uint_as_float(u);
-        if ((e & 31u) == static_cast<uint32_t>(lane)) {  // the winner takes its next best
-            const int taken = bi;
-            bk = 0u;
-            bi = 0;
-#pragma unroll
-            for (int i = 0; i < NPL; ++i) {
-                if (i == taken)
-                    key[i] = 0u;
-                if (key[i] > bk) {
-                    bk = key[i];
-                    bi = i;
-                }
+        if ((e & 31u) == static_cast<uint32_t>(lane)) {  // the winner moves to its next best
+            gone |= 1u << i1;
+            if (b2 != 0u) {
+                b1 = b2;
+                i1 = i2;
+                b2 = 0u;  // unknown until needed
+            } else {
+                top2();  // taken keys are skipped
             }
         }
         if (lane == j) {
