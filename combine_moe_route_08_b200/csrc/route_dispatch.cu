@@ -249,7 +249,10 @@ __device__ __forceinline__ bool wait_placed(const unsigned *flags, int c, unsign
 // out[part * E + x] = sum of rows [r0, r1) of a [rows][E] int32 table at
 // column x, rows split into P contiguous shares (out holds P * E ints); loads
 // kSumBatch at a time, all in flight.  Every thread calls it; ends with
-// __syncthreads().
+// __syncthreads().  Used for a CTA's later chunks (only when chunks outnumber
+// CTAs); a second inlined copy of the 16-byte form below pushed the kernel
+// past its 64-register budget (spills), so that form serves the first chunk
+// only.
 __device__ void sum_rows(const int32_t *tab, int E, int r0, int r1, int P, int32_t *out)
 {
     for (int idx = threadIdx.x; idx < P * E; idx += kThreads) {
