@@ -95,6 +95,25 @@ def test_ties_in_logits(moe):
     _full_path_vs_oracle(moe, logits, x, 64, 8, 4)
 
 
+@pytest.mark.parametrize("E,k", [(1024, 32), (256, 8), (37, 5), (8, 8), (64, 1)])
+def test_route_all_equal_logits_and_signed_zeros(moe, E, k):
+    """Every logit +0.0 or -0.0 (equal keys everywhere): the top-k is experts
+    0..k-1 in order and every weight is 1/E (1/k renormalised), the case
+    where each lane's best and second-best keys tie and the selection order
+    rests entirely on the expert index."""
+    T = 70
+    rng = np.random.default_rng(E + k)
+    logits = np.where(rng.random((T, E)) < 0.5, np.float32(-0.0), np.float32(0.0)).astype(np.float32)
+    for renorm in (False, True):
+        idx_o, w_o = oracle.route(logits, k, renormalize=renorm)
+        assert np.array_equal(idx_o, np.tile(np.arange(k, dtype=np.int32), (T, 1)))
+        idx, w = moe.moe_route_topk(to_dev(torch.from_numpy(logits)), k, renormalize=renorm)
+        torch.cuda.synchronize()
+        assert np.array_equal(idx.cpu().numpy(), idx_o)
+        gw = w.cpu().numpy().astype(np.float64)
+        assert np.all(np.abs(gw - w_o) <= route_w_tol(w_o))
+
+
 def test_masked_and_invalid_ids(moe):
     T, E, k, R, H = 96, 16, 4, 4, 256
     logits, x = inputs.make_random_case(T, H, E, k, seed=21)

@@ -213,6 +213,7 @@ EDGE = [
     (640, 128, 320, 6, 320, 0, False, 0),     # more ranks than resident CTAs may hold
     (512, 256, 64, 4, 8, 24, True, 0),        # padded with drops
     (256, 128, 24, 3, 4, 0, True, 3),         # heavy logit ties
+    (512, 128, 256, 8, 8, 0, True, 1),        # every logit equal: order by expert id alone
 ]
 
 
