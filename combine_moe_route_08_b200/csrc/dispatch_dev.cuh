@@ -45,4 +45,29 @@ __device__ __forceinline__ uint4 quant_e4m3_x16(uint4 a, uint4 b, float &s)
     return make_uint4(c[0], c[1], c[2], c[3]);
 }
 
+constexpr int kPrefetchPiece = 32768;  // bytes per L2 prefetch (a multiple of 16)
+
+// Share `share` of `shares` of the bulk L2 prefetches covering
+// [p, p + bytes): the pieces of kPrefetchPiece bytes whose index is congruent
+// to `share`, issued by the CTA's threads in turn.  p 16-byte aligned, bytes
+// a multiple of 16 and below 2^46.  TMA's untiled prefetch is fire-and-forget: no register,
+// no shared memory, nothing to wait for.  It only warms L2, the point of
+// coherence, so it can never expose stale data; lines evicted again are read
+// from HBM as usual.
+__device__ __forceinline__ void l2_prefetch_share(const void *p, int64_t bytes, int share,
+                                                  int shares)
+{
+    // at most L2-sized ranges: piece indices fit in 32 bits
+    const int n = static_cast<int>((bytes + kPrefetchPiece - 1) / kPrefetchPiece);
+    const uint8_t *base = static_cast<const uint8_t *>(p);
+    for (int i = static_cast<int>(threadIdx.x) * shares + share; i < n;
+         i += static_cast<int>(blockDim.x) * shares) {
+        const int64_t off = static_cast<int64_t>(i) * kPrefetchPiece;
+        const uint32_t size =
+            (i == n - 1) ? static_cast<uint32_t>(bytes - off) : static_cast<uint32_t>(kPrefetchPiece);
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(base + off), "r"(size)
+                     : "memory");
+    }
+}
+
 }  // namespace moe

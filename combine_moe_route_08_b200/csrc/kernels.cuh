@@ -93,4 +93,8 @@ cudaError_t combine_fp8(const uint8_t *yq, const float *ys, const int32_t *dispa
 
 cudaError_t quantize_e4m3(const float *v, int64_t n, uint8_t *q, cudaStream_t s);
 
+// How many bytes of x (x_bytes = T*H*2) a dispatch prefetches into L2 ahead of
+// its wait, and from how many CTAs (0 bytes when x would not fit in L2).
+void prefetch_plan(int64_t x_bytes, int64_t &pf_bytes, int &pf_ctas);
+
 }  // namespace moe

@@ -275,7 +275,9 @@ int moe_dispatch_layout_noalloc(const int32_t *topk_idx, int T, int k, int E, in
  *                 (MOE_ERR_INVALID_ARG via dev_status).
  *   recv_x        [rows][H] bf16 bits out; rows no slot targets are not
  *                 written.
- * T == 0 enqueues nothing.
+ * T == 0 enqueues nothing.  When x fits in three quarters of L2, the kernel's
+ * first CTAs issue L2 prefetches of x before they wait for the kernel ahead
+ * of them on the stream (a scheduling hint: no effect on any result).
  */
 int moe_dispatch_bf16(const uint16_t *x, int T, int H, int k,
                       const int32_t *dispatch_pos, uint16_t *recv_x,
@@ -295,7 +297,8 @@ int moe_dispatch_bf16(const uint16_t *x, int T, int H, int k,
  *     saturating at +-448).
  *   recv_q      [rows][H] uint8 e4m3 codes out.
  *   recv_scale  [rows][H/128] fp32 scales out (dequantised value = e4m3(q)*s).
- *   dispatch_pos, rows, dev_status: as for moe_dispatch_bf16.
+ *   dispatch_pos, rows, dev_status: as for moe_dispatch_bf16 (L2 prefetch of
+ *   x included).
  * H % 128 != 0 returns MOE_ERR_UNSUPPORTED.  T == 0 enqueues nothing.
  */
 int moe_dispatch_fp8(const uint16_t *x, int T, int H, int k,
