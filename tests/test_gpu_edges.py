@@ -30,7 +30,8 @@ def _status():
 
 
 def _full_path_vs_oracle(moe, logits, x, E, k, R, cap=0, fp8=True, idx_override=None):
-    """Every stage on the GPU against the oracle on the same inputs."""
+    """Every stage on the GPU against the oracle on the same inputs (with FP8
+    dispatch, also the FP8-payload combine of the dispatched rows)."""
     T, H = x.shape
     idx_o, w_o = oracle.route(logits.numpy(), k)
     if T:
@@ -60,6 +61,11 @@ def _full_path_vs_oracle(moe, logits, x, E, k, R, cap=0, fp8=True, idx_override=
         torch.cuda.synchronize()
         assert np.array_equal(q.cpu().numpy()[filled], qo[filled])
         assert np.array_equal(s.cpu().numpy()[filled].view(np.uint32), so[filled].view(np.uint32))
+        if T:  # the FP8-payload combine on the dispatched rows themselves
+            acc8, out8_o = oracle.combine_fp8(qo, so, pos_o, w_o)
+            out8 = moe.moe_combine_fp8(q, s, lay["dispatch_pos"], to_dev(w_o))
+            torch.cuda.synchronize()
+            assert check_combine(gpu_bits(out8), acc8, out8_o, "edge fp8") == 1.0
     else:
         r = moe.moe_dispatch_bf16(to_dev(x), lay["dispatch_pos"], rows)
         ro = oracle.dispatch_bf16(xb, pos_o, rows)
@@ -83,6 +89,8 @@ def _full_path_vs_oracle(moe, logits, x, E, k, R, cap=0, fp8=True, idx_override=
     (520, 1024, 32, 8, 128, 0),      # maximum E and k
     (4096 + 44, 32, 4, 4, 256, 0),   # several chunks per rank, ragged
     (1200, 24, 6, 3, 512, 120),      # padded with drops
+    (96, 16, 4, 2, 16384, 0),        # wide rows: several passes per CTA in every kernel
+    (64, 32, 8, 4, 12416, 0),        # wide and not a multiple of the CTA's span
 ])
 def test_random_shapes_all_stages(moe, T, E, k, R, H, cap):
     logits, x = inputs.make_random_case(T, H, E, k, seed=T + E + k + H)

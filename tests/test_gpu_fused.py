@@ -214,6 +214,8 @@ EDGE = [
     (512, 256, 64, 4, 8, 24, True, 0),        # padded with drops
     (256, 128, 24, 3, 4, 0, True, 3),         # heavy logit ties
     (512, 128, 256, 8, 8, 0, True, 1),        # every logit equal: order by expert id alone
+    (64, 16384, 16, 4, 2, 0, True, 0),        # wide rows, FP8
+    (64, 10248, 16, 4, 2, 0, False, 0),       # wide rows, bf16, H not a multiple of 128
 ]
 
 
