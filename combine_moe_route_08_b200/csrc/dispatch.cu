@@ -10,7 +10,9 @@
 //
 // One CTA per token: the row of x is read once (16-byte loads that skip L1),
 // quantised once, and written k times with 16-byte streaming stores, each
-// destination row by the whole CTA in one coalesced sweep.
+// destination row by the whole CTA in one coalesced sweep.  Before waiting
+// for the layout, the first CTAs prefetch x into L2 (prefetch_x) so that its
+// HBM read overlaps the latency-bound route and layout.
 #include <algorithm>
 #include <atomic>
 
