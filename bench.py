@@ -772,12 +772,16 @@ def run_ours(args) -> None:
 
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", choices=sorted(inputs.CONFIGS), default="dsv3")
-    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--gpus", type=int, default=1,
+                    help="ranks (one per GPU, launched by torch.distributed.run): independent replicas")
+    ap.add_argument("--steps", type=int, default=2000, help="timed steps")
+    ap.add_argument("--warmup", type=int, default=20, help="untimed warm-up steps")
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours",
+                    help="reference: time the CPU oracle on samples of the same workload")
+    ap.add_argument("--config", choices=sorted(inputs.CONFIGS), default="dsv3",
+                    help="seeded synthetic workload")
+    ap.add_argument("--no-cpu-baseline", action="store_true",
+                    help="skip timing the oracle on the host (cpu_baseline)")
     ap.add_argument("--two-phase", action="store_true",
                     help="dispatch as the pages' two-phase form (private regions + compaction)")
     ap.add_argument("--fused", action="store_true",
