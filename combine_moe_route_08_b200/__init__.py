@@ -18,7 +18,7 @@ import torch
 
 __all__ = [
     "MoeError", "lib", "moe_status_string", "moe_route_topk", "moe_route_topk_ex",
-    "moe_layout_workspace_bytes",
+    "moe_layout_workspace_bytes", "moe_dispatch_layout_launches", "kernels_per_step",
     "moe_dispatch_layout", "moe_dispatch_bf16", "moe_dispatch_fp8", "moe_combine_bf16",
     "moe_quantize_e4m3", "moe_dispatch_layout_noalloc", "moe_dispatch_fp8_ex", "Workspace",
     "LIB_PATH", "MOE_SCALE_ROW_MAJOR", "MOE_SCALE_COL_MAJOR", "moe_dispatch_layout_private",
@@ -48,6 +48,8 @@ lib.moe_route_topk_ex.argtypes = [_P, _i32, _i32, _i32, _i32, _i32, ctypes.c_flo
 lib.moe_route_topk_ex.restype = _i32
 lib.moe_layout_workspace_bytes.argtypes = [_i32, _i32, _i32, _i32]
 lib.moe_layout_workspace_bytes.restype = _sz
+lib.moe_dispatch_layout_launches.argtypes = [_i32, _i32, _i32, _i32]
+lib.moe_dispatch_layout_launches.restype = _i32
 lib.moe_dispatch_layout.argtypes = [_P, _i32, _i32, _i32, _i32, _i32, _i64, _P, _P, _P, _P, _P, _P,
                                     _P, _sz, _P, _P]
 lib.moe_dispatch_layout.restype = _i32
@@ -100,6 +102,7 @@ MOE_ERR_TIMEOUT = 5
 MOE_ERR_CUDA = 6
 MOE_SCALE_ROW_MAJOR = 0
 MOE_SCALE_COL_MAJOR = 1
+MOE_LAYOUT_NOALLOC_SCRATCH_BYTES = 1 << 20   # the fixed scratch of moe_dispatch_layout_noalloc
 
 
 class MoeError(RuntimeError):
@@ -189,6 +192,16 @@ def moe_route_topk_ex(logits: torch.Tensor, k: int, n_shared: int = 0, shared_we
 
 def moe_layout_workspace_bytes(T: int, k: int, E: int, R: int) -> int:
     return int(lib.moe_layout_workspace_bytes(T, k, E, R))
+
+
+def moe_dispatch_layout_launches(T: int, k: int, E: int, R: int) -> int:
+    return int(lib.moe_dispatch_layout_launches(T, k, E, R))
+
+
+def kernels_per_step(T: int, k: int, E: int, R: int, two_phase: bool = False) -> int:
+    """Library kernels of one route -> layout -> dispatch -> combine pass
+    (with two_phase, the receiver's compaction too)."""
+    return 1 + moe_dispatch_layout_launches(T, k, E, R) + 1 + (1 if two_phase else 0) + 1
 
 
 class Workspace:

@@ -103,6 +103,13 @@ size_t moe_layout_workspace_bytes(int T, int k, int E, int R)
     return moe::layout_workspace_bytes(moe::layout_geom(T, k, E, R));
 }
 
+int moe_dispatch_layout_launches(int T, int k, int E, int R)
+{
+    if (!valid_layout_sizes(T, k, E, R))
+        return 0;
+    return moe::layout_launches(moe::layout_geom(T, k, E, R));
+}
+
 int moe_dispatch_layout(const int32_t *topk_idx, int T, int k, int E, int R, int capacity,
                         int64_t rows, int32_t *expert_counts, int32_t *expert_src_counts,
                         int32_t *rank_counts, int32_t *expert_offsets, int32_t *dispatch_pos,

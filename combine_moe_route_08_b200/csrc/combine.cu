@@ -90,7 +90,8 @@ __global__ void __launch_bounds__(kMaxThreads)
                 }
             }
         }
-        // k > KREG: the remaining terms, in order, from shared memory
+        // k > KREG: the remaining terms, in order, each row index and weight
+        // broadcast from its lane by a shuffle
         for (int j = KREG; j < k; ++j) {
             const int r = __shfl_sync(kFullMask, myr, j);
             const float wj = __shfl_sync(kFullMask, myw, j);

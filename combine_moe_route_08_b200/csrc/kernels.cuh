@@ -22,6 +22,8 @@ struct LayoutGeom {
 
 LayoutGeom layout_geom(int T, int k, int E, int R);
 size_t layout_workspace_bytes(const LayoutGeom &g);
+// Kernels dispatch_layout launches for g on the current device (1 or 2).
+int layout_launches(const LayoutGeom &g);
 
 // Extension of the route: shared experts and expert replicas.
 struct RouteEx {

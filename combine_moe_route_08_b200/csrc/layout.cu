@@ -34,9 +34,20 @@
 // The kernel boundary between the two is the only grid-wide ordering; nothing
 // waits on another CTA.
 //
+// Decode-sized layouts (one chunk per logical rank, at most 8 steps of 32
+// slots per warp) take a single launch instead: k_layout_cluster, one
+// thread-block cluster of at most 8 CTAs.  Each CTA owns a run of whole ranks,
+// counts them per warp, and publishes its per-expert totals in its own shared
+// memory; one cluster barrier later every CTA reads the others' totals over
+// distributed shared memory, scans, and ranks its slots exactly as
+// k_layout_assign does.  The grid-wide ordering is then the hardware cluster
+// barrier (all CTAs of a cluster are co-scheduled), not a kernel boundary
+// plus a global round trip through the workspace.
+//
 // The warp-level pieces (equality masks, per-warp histograms and bases, the
 // block scan) are in layout_dev.cuh.
 #include <algorithm>
+#include <atomic>
 #include <type_traits>
 
 #include "common.cuh"
@@ -323,6 +334,199 @@ __global__ void __launch_bounds__(kThreads)
     }
 }
 
+// ---------------------------------------------------------------------------
+// Single-launch layout for one chunk per rank (decode sizes): one cluster.
+
+constexpr int kClusterMax = 8;        // CTAs of the cluster (portable cluster size)
+constexpr int kClusterSteps = 8;      // 32-slot steps per warp, at most
+constexpr int kClusterMaxE = 1024;
+
+__device__ __forceinline__ unsigned cluster_ctarank()
+{
+    unsigned r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
+
+// p (this CTA's shared memory) as seen in CTA `rank` of the cluster, loaded.
+__device__ __forceinline__ int32_t ld_peer_smem(const int32_t *p, unsigned rank)
+{
+    const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(p));
+    uint32_t ra;
+    int32_t v;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(a), "r"(rank));
+    asm volatile("ld.shared::cluster.b32 %0, [%1];" : "=r"(v) : "r"(ra) : "memory");
+    return v;
+}
+
+// CTA b of the cluster owns chunks (= ranks) [b*cpb, b*cpb + cpb); warp w
+// serves chunk b*cpb + w / wpc, the (w % wpc)-th run of seg slots of it.
+// Shared memory: wh[32][E] per-warp counts, then in-CTA bases; tot[E] this
+// CTA's totals (read by the other CTAs); off[E+1] totals over the cluster,
+// then their exclusive scan; bef[E] slots of each expert in earlier CTAs;
+// cst[cpb][E] in-CTA base at each chunk's first warp (private mode);
+// scan scratch [33].
+__global__ void __launch_bounds__(kThreads)
+    k_layout_cluster(const int32_t *__restrict__ topk_idx, LayoutGeom G, int cpb, int wpc, int seg,
+                     int capacity, int64_t rows, int32_t *__restrict__ expert_counts,
+                     int32_t *__restrict__ expert_src_counts, int32_t *__restrict__ rank_counts,
+                     int32_t *__restrict__ expert_offsets, int32_t *__restrict__ dispatch_pos,
+                     int32_t *__restrict__ recv_src, int32_t *__restrict__ private_pos,
+                     int32_t *__restrict__ dev_status)
+{
+    extern __shared__ int32_t sm[];
+    const int E = G.E, lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const int nb = key_bits(E);
+    int32_t *wh = sm;
+    int32_t *tot = wh + kWarps * E;
+    int32_t *off = tot + E;
+    int32_t *bef = off + E + 1;
+    int32_t *cst = bef + E;
+    int32_t *scr = cst + cpb * E;
+    const unsigned b = cluster_ctarank();
+    const unsigned C = gridDim.x;
+
+    // this warp's run [w0, w1) of the slots of chunk c (empty for spare warps)
+    const int lc = w / wpc;
+    const int c = static_cast<int>(b) * cpb + lc;
+    const bool has_chunk = lc < cpb && c < G.nchunks;
+    int64_t w0 = 0, w1 = 0;
+    if (has_chunk) {
+        const int64_t i0 = static_cast<int64_t>(c) * G.Tr * G.k;
+        const int64_t i1 = i0 + static_cast<int64_t>(G.Tr) * G.k;
+        w0 = min(i0 + static_cast<int64_t>(w % wpc) * seg, i1);
+        w1 = min(w0 + seg, i1);
+    }
+    for (int x = threadIdx.x; x < kWarps * E; x += kThreads)
+        wh[x] = 0;
+    pdl_trigger();  // the next kernel may take idle SM slots now; it waits for this one
+    pdl_wait();
+    int e[kClusterSteps];
+    bool bad = false;
+#pragma unroll
+    for (int s = 0; s < kClusterSteps; ++s) {
+        const int64_t i = w0 + 32 * s + lane;
+        e[s] = (i < w1) ? __ldg(topk_idx + i) : -1;
+        bad |= (i < w1) && e[s] != -1 && static_cast<unsigned>(e[s]) >= static_cast<unsigned>(E);
+    }
+    if (bad)
+        report(dev_status, MOE_ERR_INVALID_ARG);
+    __syncthreads();
+    warp_histogram(e, w0, w1, E, nb, wh + w * E);
+    __syncthreads();
+
+    // per expert: in-CTA exclusive prefix over the warps (slot order), each
+    // chunk's count (its rank's source-count column) and the CTA total
+    for (int x = threadIdx.x; x < E; x += kThreads) {
+        int run = 0;
+        for (int q = 0; q < cpb; ++q) {
+            const int start = run;
+            if (G.max_m > 0)
+                cst[q * E + x] = start;
+            for (int ww = q * wpc; ww < (q + 1) * wpc; ++ww) {
+                const int t = wh[ww * E + x];
+                wh[ww * E + x] = run;
+                run += t;
+            }
+            const int cq = static_cast<int>(b) * cpb + q;
+            if (cq < G.nchunks)
+                expert_src_counts[static_cast<size_t>(x) * G.R + cq] = run - start;
+        }
+        tot[x] = run;
+    }
+    cluster_arrive();  // publishes tot (release) ...
+    cluster_wait();    // ... and sees every CTA's (acquire)
+    for (int x = threadIdx.x; x < E; x += kThreads) {
+        int before = 0, total = 0;
+        for (unsigned bb = 0; bb < C; ++bb) {
+            const int v = ld_peer_smem(tot + x, bb);
+            total += v;
+            before += (bb < b) ? v : 0;
+        }
+        off[x] = total;
+        bef[x] = before;
+        if (b == 0)
+            expert_counts[x] = total;
+    }
+    cluster_arrive();  // done reading the other CTAs' tot; waited for before exit
+    __syncthreads();
+    block_exclusive_scan<kWarps>(off, E, scr);  // off[e] = slots of experts < e; off[E] = total
+    if (b == 0) {
+        for (int x = threadIdx.x; x <= E; x += kThreads)
+            expert_offsets[x] = (capacity == 0) ? off[x] : x * capacity;
+        const int L = E / G.R;
+        for (int rr = threadIdx.x; rr < G.R; rr += kThreads)
+            rank_counts[rr] = off[(rr + 1) * L] - off[rr * L];
+    }
+
+    // rank every slot among equal experts, in slot order
+    int32_t *mywh = wh + w * E;
+    bool dropped = false, bad_row = false;
+#pragma unroll
+    for (int s = 0; s < kClusterSteps; ++s) {
+        if (w0 + 32 * s >= w1)
+            break;  // warp-uniform
+        const int64_t i = w0 + 32 * s + lane;
+        const bool valid = static_cast<unsigned>(e[s]) < static_cast<unsigned>(E);
+        const int p = rank_step(e[s], E, nb, mywh);  // in-CTA position among equal experts
+        if (i < w1) {
+            int64_t row = -1, prow = -1;
+            bool hole = false;  // private mode: packed row left empty by a dropped slot
+            if (valid) {
+                const int pe = bef[e[s]] + p;  // position inside the expert
+                if (capacity == 0)
+                    row = off[e[s]] + pe;
+                else if (pe < capacity)
+                    row = static_cast<int64_t>(e[s]) * capacity + pe;
+                else
+                    dropped = true;
+                if (G.max_m > 0 && row >= 0) {
+                    const int pr = p - cst[lc * E + e[s]];  // among this rank's slots of e
+                    if (pr < G.max_m) {
+                        prow = (static_cast<int64_t>(e[s]) * G.R + c) * G.max_m + pr;
+                    } else {
+                        dropped = true;
+                        hole = true;
+                    }
+                }
+            }
+            if (row >= rows) {  // cannot happen for a consistent layout; never write past rows
+                bad_row = true;
+                row = -1;
+            }
+            dispatch_pos[i] = hole ? -1 : static_cast<int32_t>(row);
+            if (row >= 0)
+                recv_src[row] = hole ? -1 : static_cast<int32_t>(i);
+            if (G.max_m > 0)
+                private_pos[i] = static_cast<int32_t>(prow);
+        }
+    }
+    if (dropped)
+        report(dev_status, MOE_ERR_CAPACITY);
+    if (bad_row)
+        report(dev_status, MOE_ERR_INVALID_ARG);
+
+    // rows that no slot fills -> -1
+    const int64_t stride = static_cast<int64_t>(C) * kThreads;
+    const int64_t first = static_cast<int64_t>(b) * kThreads + threadIdx.x;
+    if (capacity == 0) {
+        for (int64_t r = off[E] + first; r < rows; r += stride)
+            recv_src[r] = -1;
+    } else {
+        for (int x = static_cast<int>(b); x < E; x += static_cast<int>(C)) {
+            const int filled = min(off[x + 1] - off[x], capacity);
+            for (int p = filled + threadIdx.x; p < capacity; p += kThreads)
+                recv_src[static_cast<int64_t>(x) * capacity + p] = -1;
+        }
+        for (int64_t r = static_cast<int64_t>(E) * capacity + first; r < rows; r += stride)
+            recv_src[r] = -1;
+    }
+    cluster_wait();  // no CTA exits while another may still read its tot
+}
+
 size_t assign_smem_bytes(int E) { return (static_cast<size_t>(kWarps + 3) * E + 1 + kWarps + 1) * sizeof(int32_t); }
 
 }  // namespace
@@ -348,12 +552,129 @@ size_t layout_workspace_bytes(const LayoutGeom &g)
     return std::max<size_t>(256, (hist + 255) / 256 * 256);
 }
 
+namespace {
+
+// The single-launch plan for a geometry, or ok = false when it does not fit:
+// more than one chunk per rank, E beyond the kernel's limit, runs longer than
+// kClusterSteps steps per warp, shared memory beyond the device's opt-in
+// limit, or a device that cannot schedule such a cluster.
+struct ClusterPlan {
+    bool ok = false;
+    int C = 0, cpb = 0, wpc = 0, seg = 0;
+    size_t smem = 0;
+};
+
+size_t cluster_smem_bytes(int E, int cpb)
+{
+    return (static_cast<size_t>(kWarps + 3 + cpb) * E + 1 + kWarps + 1) * sizeof(int32_t);
+}
+
+// Whether this device can run one cluster of kClusterMax CTAs of kThreads
+// threads with `smem` bytes each (queried once per device for the largest
+// shared-memory size the plan allows).
+bool cluster_schedulable(size_t smem)
+{
+    constexpr int kMaxDev = 64;
+    static std::atomic<int> state[kMaxDev];  // 0 unknown, 1 yes, 2 no
+    static std::atomic<int> optin[kMaxDev];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) {
+        cudaGetLastError();
+        return false;
+    }
+    int st = state[dev].load(std::memory_order_acquire);
+    if (st == 0) {
+        int limit = 0;
+        bool ok = cudaDeviceGetAttribute(&limit, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) == cudaSuccess;
+        const size_t probe = std::min<size_t>(static_cast<size_t>(limit), cluster_smem_bytes(kClusterMaxE, 8));
+        ok = ok && cudaFuncSetAttribute(k_layout_cluster, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        static_cast<int>(probe)) == cudaSuccess;
+        int n = 0;
+        if (ok) {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(kClusterMax);
+            cfg.blockDim = dim3(kThreads);
+            cfg.dynamicSmemBytes = probe;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = kClusterMax;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            ok = cudaOccupancyMaxActiveClusters(&n, k_layout_cluster, &cfg) == cudaSuccess && n >= 1;
+        }
+        if (!ok)
+            cudaGetLastError();
+        optin[dev].store(ok ? static_cast<int>(probe) : 0, std::memory_order_relaxed);
+        st = ok ? 1 : 2;
+        state[dev].store(st, std::memory_order_release);
+    }
+    return st == 1 && smem <= static_cast<size_t>(optin[dev].load(std::memory_order_relaxed));
+}
+
+ClusterPlan cluster_plan(const LayoutGeom &g)
+{
+    ClusterPlan p;
+    if (g.cpr != 1 || g.E > kClusterMaxE)
+        return p;
+    const int n = g.nchunks;  // one chunk per rank
+    int C = std::min(kClusterMax, n);
+    const int cpb = ceil_div(n, C);
+    if (cpb > kWarps)
+        return p;
+    const int wpc = kWarps / cpb;
+    const int slots = g.Tr * g.k;
+    const int seg = round_up(ceil_div(slots, wpc), 32);
+    if (seg > 32 * kClusterSteps)
+        return p;
+    C = ceil_div(n, cpb);
+    const size_t smem = cluster_smem_bytes(g.E, cpb);
+    if (!cluster_schedulable(smem))
+        return p;
+    p.ok = true;
+    p.C = C;
+    p.cpb = cpb;
+    p.wpc = wpc;
+    p.seg = seg;
+    p.smem = smem;
+    return p;
+}
+
+}  // namespace
+
+int layout_launches(const LayoutGeom &g) { return cluster_plan(g).ok ? 1 : 2; }
+
 cudaError_t dispatch_layout(const int32_t *topk_idx, const LayoutGeom &g, int capacity, int64_t rows,
                             int32_t *expert_counts, int32_t *expert_src_counts,
                             int32_t *rank_counts, int32_t *expert_offsets, int32_t *dispatch_pos,
                             int32_t *recv_src, int32_t *private_pos, void *workspace,
                             int32_t *dev_status, cudaStream_t s)
 {
+    const ClusterPlan cp = cluster_plan(g);
+    if (cp.ok) {
+        cudaError_t err = cudaFuncSetAttribute(k_layout_cluster, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               static_cast<int>(cp.smem));
+        if (err != cudaSuccess)
+            return err;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(cp.C);
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = cp.smem;
+        cfg.stream = s;
+        cudaLaunchAttribute attr[2];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = cp.C;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 2;
+        return cudaLaunchKernelEx(&cfg, k_layout_cluster, topk_idx, g, cp.cpb, cp.wpc, cp.seg,
+                                  capacity, rows, expert_counts, expert_src_counts, rank_counts,
+                                  expert_offsets, dispatch_pos, recv_src, private_pos, dev_status);
+    }
     int32_t *hist = static_cast<int32_t *>(workspace);
     cudaError_t err = launch_pdl(k_layout_hist, dim3(g.nchunks), dim3(kThreads), g.E * sizeof(int32_t),
                                  s, topk_idx, g, hist, dev_status);

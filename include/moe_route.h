@@ -133,6 +133,17 @@ int moe_route_topk_ex(const float *logits, int T, int E, int k, int renormalize,
 size_t moe_layout_workspace_bytes(int T, int k, int E, int R);
 
 /*
+ * How many kernels moe_dispatch_layout (and moe_dispatch_layout_private)
+ * launch for (T, k, E, R) on the current device: 1 when every logical rank
+ * fits one chunk of at most 2048 slots (T/R * k <= 2048; the decode sizes)
+ * and the device can schedule the single-launch form (one thread-block
+ * cluster of at most 8 CTAs), else 2 (a per-chunk histogram, then the
+ * placement).  0 on invalid sizes.  Both forms give identical outputs; the
+ * count serves callers that account for launches (graph sizing, profiling).
+ */
+int moe_dispatch_layout_launches(int T, int k, int E, int R);
+
+/*
  * moe_dispatch_layout -- counts, offsets and index maps for dispatch/combine.
  * Follows "Enabling trillion-parameter models on AWS EFA", "Gönderme ve Alma
  * Arabellekleri" (per-expert token counts first; then every sender knows
@@ -240,14 +251,24 @@ int moe_compact_bf16(const uint16_t *priv_x, int64_t private_rows, const int32_t
  * array of MOE_LAYOUT_NOALLOC_SCRATCH_BYTES (1 MiB) inside this library:
  * every GPU that loads the library holds it until the process exits.
  *
- *   - Limit: (T, k, E, R) whose moe_layout_workspace_bytes exceeds
- *     MOE_LAYOUT_NOALLOC_SCRATCH_BYTES are rejected with MOE_ERR_WORKSPACE
- *     before anything is enqueued (e.g. E = 256 fits up to 1024 chunks of at
- *     most 2048 slots each, T*k up to 2^21; every workload of the benchmark
- *     fits).
+ *   - Limit: a call fits exactly when moe_layout_workspace_bytes(T, k, E, R)
+ *     <= MOE_LAYOUT_NOALLOC_SCRATCH_BYTES; larger sizes are rejected with
+ *     MOE_ERR_WORKSPACE before anything is enqueued.  That size is
+ *     max(256, round_up(R * ceil((T/R) / max(1, floor(2048/k))) * E * 4, 256))
+ *     bytes: one E-wide int32 histogram row per chunk, where a chunk is at
+ *     most floor(2048/k) tokens of one logical rank, so a partly filled chunk
+ *     still takes a whole row.  (E = 256, k = 8: up to 1024 chunks, e.g.
+ *     T/R = 256 tokens per rank and R <= 1024; every workload of the
+ *     benchmark fits.)
  *   - Set-up: the first call on each device looks the array's device address
- *     up (cudaGetSymbolAddress, with that device current) and keeps it; make
- *     that first call before any stream capture on that device.
+ *     up (cudaGetSymbolAddress, with that device current); every later call
+ *     made outside stream capture looks it up again (a host query, no
+ *     allocation), so a device reset or a re-created context never leaves a
+ *     stale address.  Calls during stream capture reuse the last address
+ *     found outside capture: make the first call on each device before any
+ *     stream capture on it, else the call returns MOE_ERR_UNSUPPORTED.  Any
+ *     number of devices is served (the table is sized from
+ *     cudaGetDeviceCount).
  *   - Sharing: all calls share the one array and it keeps the last call's
  *     contents.  Each call rewrites every scratch word it reads, so nothing
  *     needs clearing, but two calls whose kernels overlap on the GPU (other

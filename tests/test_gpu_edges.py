@@ -91,6 +91,9 @@ def _full_path_vs_oracle(moe, logits, x, E, k, R, cap=0, fp8=True, idx_override=
     (1200, 24, 6, 3, 512, 120),      # padded with drops
     (96, 16, 4, 2, 16384, 0),        # wide rows: several passes per CTA in every kernel
     (64, 32, 8, 4, 12416, 0),        # wide and not a multiple of the CTA's span
+    (1024, 1024, 32, 64, 128, 0),    # single-launch layout: 8 ranks per CTA, E and k at maximum
+    (2048, 64, 4, 16, 128, 100),     # single-launch layout, padded with drops
+    (6144, 384, 8, 48, 128, 0),      # single-launch layout: 6 ranks per CTA, 5 warps each
 ])
 def test_random_shapes_all_stages(moe, T, E, k, R, H, cap):
     logits, x = inputs.make_random_case(T, H, E, k, seed=T + E + k + H)
@@ -284,6 +287,17 @@ def test_layout_large_token_count_many_chunks(moe):
     for key in LAYOUT_KEYS:
         assert np.array_equal(lay_p[key].cpu().numpy(), want_p[key].reshape(lay_p[key].shape)), key
     assert st.item() == moe.MOE_ERR_CAPACITY
+
+
+def test_layout_launch_count(moe):
+    """Decode sizes (one chunk of at most 2048 slots per rank) take the
+    single-launch cluster layout; prefill (16 chunks per rank) the
+    histogram + placement pair."""
+    assert moe.moe_dispatch_layout_launches(4096, 8, 256, 32) == 1      # dsv3
+    assert moe.moe_dispatch_layout_launches(6144, 8, 384, 48) == 1      # kimi
+    assert moe.moe_dispatch_layout_launches(4096, 9, 288, 32) == 1      # dsv3 + shared expert
+    assert moe.moe_dispatch_layout_launches(32768, 8, 256, 8) == 2      # prefill
+    assert moe.moe_dispatch_layout_launches(4096, 8, 256, 3) == 0       # R does not divide E
 
 
 def test_all_slots_masked(moe):

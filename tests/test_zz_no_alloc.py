@@ -5,8 +5,10 @@ fixed 1 MiB device scratch instead of a caller workspace.
 
 Called through the C ABI (ctypes, raw device pointers) twice in a row on
 different routings, each time compared with moe_dispatch_layout given its
-own workspace: the outputs are integer maps, so they must be identical.  The
-file is collected last so that a failure here leaves every other test run.
+own workspace and with the oracle's layout: the outputs are integer maps, so
+they must be identical.  The size limit is checked at its exact boundary.
+The file is collected last so that a failure here leaves every other test
+run.
 """
 import ctypes
 
@@ -73,9 +75,54 @@ def test_noalloc_layout_matches_workspace_layout_twice_in_a_row():
                                              st_b.data_ptr(), stream)
         assert rc == moe.MOE_OK
         torch.cuda.synchronize()
+        ref = oracle.layout(idx.cpu().numpy(), E, R, cap, rows)
         for key in KEYS:
             assert torch.equal(got[key], want[key]), f"{name}: {key}"
+            assert np.array_equal(got[key].cpu().numpy(), ref[key].reshape(got[key].shape)), \
+                f"{name}: {key} vs the oracle"
         assert st_a.item() == st_b.item() == 0
+
+
+def _noalloc_bytes(T, k, E, R):
+    """The documented size of the scratch a (T, k, E, R) needs: one E-wide
+    int32 histogram row per chunk of at most floor(2048 / k) tokens of one
+    logical rank, rounded up to 256 bytes (at least 256)."""
+    per_chunk = max(1, 2048 // k)
+    chunks = R * max(1, -(-(T // R) // per_chunk))
+    return max(256, -(-chunks * E * 4 // 256) * 256)
+
+
+def test_noalloc_limit_at_its_exact_boundary():
+    """E = 1024, k = 8, R = 256: 256 tokens per rank fill one chunk per rank,
+    256 rows of 4 KiB = exactly the 1 MiB scratch, and run (compared with
+    the oracle); 257 tokens per rank need a second, almost empty chunk per
+    rank and are rejected although T * k is far below 2^21."""
+    import combine_moe_route_08_b200 as moe
+    lib = moe.lib
+    limit = moe.MOE_LAYOUT_NOALLOC_SCRATCH_BYTES
+    E, k, R = 1024, 8, 256
+    T_fit, T_over = 256 * R, 257 * R
+    assert lib.moe_layout_workspace_bytes(T_fit, k, E, R) == _noalloc_bytes(T_fit, k, E, R) == limit
+    assert lib.moe_layout_workspace_bytes(T_over, k, E, R) == _noalloc_bytes(T_over, k, E, R) > limit
+    fake = ctypes.c_void_p(0x10000)
+    rc = lib.moe_dispatch_layout_noalloc(fake, T_over, k, E, R, 0, T_over * k, fake, fake, fake,
+                                         fake, fake, fake, None, None)
+    assert rc == moe.MOE_ERR_WORKSPACE
+    dev = torch.device("cuda", 0)
+    rng = np.random.default_rng(5)
+    idx_np = np.argsort(rng.random((T_fit, E), dtype=np.float32), axis=1)[:, :k].astype(np.int32)
+    idx = torch.from_numpy(idx_np).cuda()
+    rows = T_fit * k
+    got = _alloc(T_fit, k, E, R, rows, dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    rc = lib.moe_dispatch_layout_noalloc(idx.data_ptr(), T_fit, k, E, R, 0, rows, *_ptrs(got),
+                                         st.data_ptr(), torch.cuda.current_stream().cuda_stream or None)
+    assert rc == moe.MOE_OK
+    torch.cuda.synchronize()
+    ref = oracle.layout(idx_np, E, R)
+    for key in KEYS:
+        assert np.array_equal(got[key].cpu().numpy(), ref[key].reshape(got[key].shape)), key
+    assert st.item() == 0
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
