@@ -1,7 +1,7 @@
 #!/usr/bin/env python
 """Benchmark of the MoE route -> layout -> dispatch -> combine path on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config dsv3]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config dsv3,kimi,prefill]
                     [--impl ours|reference]
 
 One step = one pass of the whole path over one batch of seeded synthetic
@@ -10,23 +10,32 @@ moe_combine_bf16.  The stand-in expert between dispatch and combine is not
 part of the path (it needs trained weights): its outputs are prepared once,
 before timing, and stay resident, as a grouped GEMM would leave them.
 
-Timing: W untimed warm-up steps, then exactly K timed steps between a
-barrier + device synchronise on both sides.  When a step moves more than
-twice the L2 size (126 MB) its inputs cannot stay in L2 from one step to the
-next ("inputs larger than L2"); smaller workloads write a 512 MiB buffer
-before every step to flush L2, outside the timed events.  Each step and each
-stage is timed with CUDA events on the stream the kernels run on; the timed
-loop calls the C ABI directly with pre-marshalled arguments.
-Clocks and throttle reasons are sampled with nvidia-smi during the timed
-region.  With N > 1 (torchrun) every rank runs an independent replica (the
-path does not shard: no data-path collective); the reported time is the
-maximum over ranks and `value` the bytes of all ranks over that time.
+By default one run measures the decode workloads dsv3 and kimi and the
+prefill workload, one after the other, and prints ONE JSON line: the
+headline fields (value, roofline, e2e, cpu_baseline) belong to the largest
+workload, prefill; every workload's step and dispatch+combine figures are in
+its `configs` entry.
+
+Timing: W untimed warm-up steps, then timed regions of exactly K steps, each
+between a barrier + device synchronise on both sides.  The K-step region is
+repeated until about a second of timed work has run (at least 5 times), and
+the median region gives the reported time; the spread is reported beside it.
+When a step moves more than twice the L2 size (126 MB) its inputs cannot
+stay in L2 from one step to the next ("inputs larger than L2"); smaller
+workloads write a 512 MiB buffer before every step to flush L2, outside the
+timed events.  Each step and each stage is timed with CUDA events on the
+stream the kernels run on; the timed loop calls the C ABI directly with
+pre-marshalled arguments.  Clocks and throttle reasons are sampled with
+nvidia-smi across the repeated regions.  With N > 1 (torchrun) every rank
+runs an independent replica (the path does not shard: no data-path
+collective); the reported time is the maximum over ranks and `value` the
+bytes of all ranks over that time.
 
 `value` is the effective HBM bandwidth of a step: the algorithmic bytes the
 path must move (each token read once, each row written once, see
 algorithmic_bytes) divided by the step time.  The reference arm
 (--impl reference) times the oracle, a plain single-threaded CPU program,
-on the same workload and metric.
+on samples of the same headline workload, with the same metric and config.
 """
 from __future__ import annotations
 
@@ -34,6 +43,7 @@ import argparse
 import datetime as _dt
 import hashlib
 import json
+import math
 import os
 import subprocess
 import sys
@@ -51,8 +61,15 @@ METRIC = "dispatch+combine µs/layer and effective HBM GB/s (% of B200 roofline)
 SPEC_HBM_GBS = 8000.0          # B200 HBM3e bandwidth the roofline target is quoted against
 FALLBACK_HBM_GBS = 6650.0      # earlier measured copy bandwidth on this machine
 L2_FLUSH_BYTES = 512 << 20
-KERNELS_PER_STEP = 5           # route, layout (2 kernels), dispatch, combine (+1 compaction, two-phase)
 STEPS_PER_GRAPH = 10           # consecutive steps captured in one CUDA graph (no-flush workloads)
+DEFAULT_CONFIGS = "dsv3,kimi,prefill"
+REGION_TARGET_S = 1.0          # timed work per workload for the step (repeated K-step regions)
+DC_TARGET_S = 0.5              # the same for the dispatch+combine graphs
+MIN_REPS, MAX_REPS = 5, 4000
+DTYPES = {"route": "f32 logits -> f32 weights, int32 ids",
+          "layout": "int32",
+          "dispatch": "bf16 rows -> e4m3 codes + f32 1x128 scales (bf16 copy for bf16 workloads)",
+          "combine": "bf16 rows, f32 multiply and add, bf16 out"}
 
 
 # --------------------------------------------------------------------------
@@ -108,6 +125,45 @@ def combine_traffic(cfg_name: str, fp8: bool = False):
     return rec.get("dram_bytes_per_launch")
 
 
+def config_names(arg: str) -> list[str]:
+    names = [n.strip() for n in arg.split(",") if n.strip()]
+    bad = [n for n in names if n not in inputs.CONFIGS]
+    if not names or bad:
+        raise SystemExit(f"unknown workload(s) {bad}; choose from {sorted(inputs.CONFIGS)}")
+    return list(dict.fromkeys(names))
+
+
+def headline_name(names: list[str]) -> str:
+    """The largest workload of the run (tokens x hidden size): its figures
+    are the line's headline."""
+    return max(names, key=lambda n: (inputs.CONFIGS[n].T * inputs.CONFIGS[n].H, names.index(n)))
+
+
+def pipeline_text(args) -> str:
+    if args.fused:
+        return "fused: route + layout + dispatch in one cooperative launch (moe_route_dispatch), then combine"
+    if args.two_phase:
+        return ("two-phase: private-region layout, send into E*R private regions of T_r rows, "
+                "receiver compaction")
+    return "direct scatter into the packed (or padded) rows"
+
+
+def line_config(args, names: list[str], n_gpus: int) -> dict:
+    """The workload description shared by both arms (no measured value in it)."""
+    head = inputs.CONFIGS[headline_name(names)]
+    return {
+        "workload": head.describe(),
+        "workloads": {n: inputs.CONFIGS[n].describe() for n in names},
+        "parallelism": f"replicas x{n_gpus}",
+        "pipeline": pipeline_text(args),
+        "combine_payload": ("fp8 e4m3 + 1x128 fp32 scales (the dispatched rows)"
+                            if args.combine_fp8 else "bf16 (stand-in expert output)"),
+        "l2": ("inputs larger than L2 (no flush) for workloads that move more than 2 x L2 per "
+               f"step; a {L2_FLUSH_BYTES >> 20} MiB write before every step outside the timed "
+               "events otherwise"),
+    }
+
+
 # --------------------------------------------------------------------------
 # clocks during the timed region
 # --------------------------------------------------------------------------
@@ -119,7 +175,7 @@ class ClockSampler:
 
     def __init__(self, device_index: int):
         self.proc = None
-        self.t0 = self.t1 = None
+        self.windows: list[list] = []
         uuid = None
         try:
             uuid = str(torch.cuda.get_device_properties(device_index).uuid)
@@ -140,14 +196,16 @@ class ClockSampler:
         time.sleep(0.3)
 
     def mark_start(self):
-        self.t0 = _dt.datetime.now()
+        self.windows.append([_dt.datetime.now(), None])
 
     def mark_end(self):
-        self.t1 = _dt.datetime.now()
+        if self.windows:
+            self.windows[-1][1] = _dt.datetime.now()
 
     def stop(self) -> dict:
         if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"],
+                    "samples": 0, "samples_in_timed_region": 0}
         time.sleep(0.1)
         self.proc.terminate()
         out, _ = self.proc.communicate(timeout=10)
@@ -161,7 +219,8 @@ class ClockSampler:
             except ValueError:
                 continue
             rows.append((ts, parts))
-        inside = [p for ts, p in rows if self.t0 and self.t1 and self.t0 <= ts <= self.t1]
+        inside = [p for ts, p in rows
+                  if any(a is not None and b is not None and a <= ts <= b for a, b in self.windows)]
         use = inside or [p for _, p in rows]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({n for p in use for n, v in zip(names, p[5:9]) if v.lower() == "active"})
@@ -169,7 +228,10 @@ class ClockSampler:
         smax = [float(p[2]) for p in use if p[2].replace(".", "").isdigit()]
         return {"sm_mhz": float(np.median(sm)) if sm else None,
                 "sm_max_mhz": max(smax) if smax else None,
-                "reasons": reasons, "samples": len(use), "samples_in_timed_region": len(inside)}
+                "sm_mhz_min": min(sm) if sm else None,
+                "reasons": reasons, "samples": len(rows), "samples_in_timed_region": len(inside),
+                "from": "samples inside the timed regions" if inside else
+                        "no sample fell inside the timed regions: samples around them"}
 
 
 # --------------------------------------------------------------------------
@@ -208,6 +270,13 @@ def max_over_ranks(values: list[float], world: int, device) -> list[float]:
     t = torch.tensor(values, dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return t.cpu().tolist()
+
+
+def repetitions(region_s: float, target_s: float) -> int:
+    """How many K-step regions make about target_s seconds of timed work."""
+    if not region_s > 0:
+        return MIN_REPS
+    return int(min(MAX_REPS, max(MIN_REPS, math.ceil(target_s / region_s))))
 
 
 # --------------------------------------------------------------------------
@@ -260,7 +329,7 @@ def cpu_inputs(cfg: inputs.Config) -> dict:
                 placement=inputs.expert_placement(cfg) if cfg.n_shared else None)
 
 
-def cpu_baseline(cfg: inputs.Config, budget_s: float = 12.0) -> dict:
+def cpu_baseline(cfg: inputs.Config, budget_s: float = 10.0) -> dict:
     """The oracle as it stands, single-threaded, on whole-workload steps
     repeated until about `budget_s` seconds of CPU work."""
     wl = cpu_inputs(cfg)
@@ -271,7 +340,7 @@ def cpu_baseline(cfg: inputs.Config, budget_s: float = 12.0) -> dict:
         total_b += b
         n += 1
     return {"value": total_b / total_t / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "host_cores": os.cpu_count(),
+            "host_cores": os.cpu_count(), "workload": cfg.name,
             "sample": f"{n} full {cfg.name} step(s) (T={cfg.T}), {total_t:.1f} s of CPU work, "
                       f"1 thread of {os.cpu_count()} host cores",
             "s_per_step": total_t / n}
@@ -281,7 +350,8 @@ def run_reference(args) -> None:
     world, rank, _ = dist_env()
     if rank != 0:
         return  # the oracle runs on rank 0 only; other ranks exit without work
-    cfg = inputs.CONFIGS[args.config]
+    names = config_names(args.config)
+    cfg = inputs.CONFIGS[headline_name(names)]
     wl = cpu_inputs(cfg)
     # size each step so that warm-up + timed steps fit in about two minutes
     dt1, _ = oracle_step_on_sample(cfg, wl, cfg.R)           # one token per rank
@@ -301,10 +371,11 @@ def run_reference(args) -> None:
         "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * tt / args.steps, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": cfg.describe(), "sample_tokens_per_step": tokens},
+        "vs_baseline": None, "dtype": "bf16+e4m3", "dtypes": DTYPES, "data": "synthetic",
+        "config": line_config(args, names, args.gpus),
         "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
-                         "sample": f"{tokens} of {cfg.T} tokens per step "
+                         "workload": cfg.name,
+                         "sample": f"{tokens} of {cfg.T} {cfg.name} tokens per step "
                                    f"({ranks} per logical rank), 1 thread of {os.cpu_count()}"},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -315,14 +386,10 @@ def run_reference(args) -> None:
 # our arm
 # --------------------------------------------------------------------------
 
-def run_ours(args) -> None:
-    world, rank, local = dist_env()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    init_dist(world, "nccl")
+def measure(cfg: inputs.Config, args, dev, world: int, local: int) -> dict:
+    """Set up one workload on the device and time it (all ranks call this)."""
     import combine_moe_route_08_b200 as moe
 
-    cfg = inputs.CONFIGS[args.config]
     T, H, E, R = cfg.T, cfg.H, cfg.E, cfg.R
     k = cfg.k_total                         # slots per token (routed + shared)
     E_lay = cfg.E_phys if cfg.n_shared else E   # experts the layout sees
@@ -351,12 +418,12 @@ def run_ours(args) -> None:
         rows = T * k if cap == 0 else E_lay * cap
         lay = moe.moe_dispatch_layout(idx, E_lay, R, capacity=cap, rows=rows, workspace=ws)
         if args.combine_fp8 and cfg.dispatch != "fp8":
-            raise SystemExit("--combine-fp8 needs an FP8-dispatch workload")
+            raise SystemExit("--combine-fp8 needs FP8-dispatch workloads")
         if args.fused and args.two_phase:
             raise SystemExit("--fused runs the direct layout")
         if args.two_phase:
             if cap:
-                raise SystemExit("--two-phase needs a packed-layout workload")
+                raise SystemExit("--two-phase needs packed-layout workloads")
             max_m = cfg.T_r                      # a rank sends at most T_r tokens to an expert
             lay["private_pos"] = torch.empty(T, k, dtype=torch.int32, device=dev)
             moe.moe_dispatch_layout_private(idx, E_lay, R, max_m, out=lay, workspace=ws)
@@ -377,7 +444,7 @@ def run_ours(args) -> None:
         flush_buf = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
     s.synchronize()
 
-    # the four C ABI calls of a step with their arguments marshalled once
+    # the C ABI calls of a step with their arguments marshalled once
     lib, sp = moe.lib, s.cuda_stream
     ws_buf = ws.get(moe.moe_layout_workspace_bytes(T, k, E_lay, R))
     pos = lay["dispatch_pos"]
@@ -478,7 +545,7 @@ def run_ours(args) -> None:
             flush.buf.fill_(i)
     flush.buf = flush_buf
 
-    # Steps run as replays of CUDA graphs of the four C ABI calls (the library
+    # Steps run as replays of CUDA graphs of the C ABI calls (the library
     # launches its kernels with programmatic dependent launch).  Workloads
     # timed without an L2 flush put STEPS_PER_GRAPH consecutive steps in one
     # graph, as a model forward puts many layers in one graph, so the graph
@@ -521,23 +588,56 @@ def run_ours(args) -> None:
     def ms_per(evs, n_steps):
         return float(sum(a.elapsed_time(b) for a, b in evs)) / n_steps
 
+    def region(g_many, g_one, sampler=None):
+        """One timed region of exactly K steps between a barrier and a device
+        synchronise on both sides; ms per step."""
+        barrier(world, dev)
+        torch.cuda.synchronize(dev)
+        if sampler is not None:
+            sampler.mark_start()
+        evs = timed_replays(g_many, g_one, K)
+        s.synchronize()
+        torch.cuda.synchronize(dev)
+        if sampler is not None:
+            sampler.mark_end()
+        barrier(world, dev)
+        return ms_per(evs, K)
+
+    def repeated_regions(g_many, g_one, target_s, sampler):
+        """Calibrate with one untimed-for-the-record region, then run the same
+        number of K-step regions on every rank; per-rank median ms per step."""
+        with torch.cuda.stream(s):
+            t0 = time.perf_counter()
+            region(g_many, g_one)
+            region_s = time.perf_counter() - t0
+            reps = int(max_over_ranks([float(repetitions(region_s, target_s))], world, dev)[0])
+            got = [region(g_many, g_one, sampler) for _ in range(reps)]
+        return float(np.median(got)), float(min(got)), float(max(got)), reps
+
     g_step1 = capture(step, 1)
     g_stepG = capture(step, G) if G > 1 else g_step1
+    # dispatch+combine as the pages count it (layout + dispatch + combine,
+    # route excluded): its own graphs, timed the same way
+    dc_calls = calls if args.fused else calls[1:]   # fused: the route cannot be left out
+
+    def dc_step():
+        for fn, a in dc_calls:
+            rc = fn(*a)
+            if rc != 0:
+                raise moe.MoeError(rc, fn.__name__)
+    g_dc1 = capture(dc_step, 1)
+    g_dcG = capture(dc_step, G) if G > 1 else g_dc1
+
     with torch.cuda.stream(s):
         timed_replays(g_stepG, g_step1, W)          # warm-up
+        timed_replays(g_dcG, g_dc1, W)
         s.synchronize()
-        sampler = ClockSampler(local)
-        sampler.start()
-        barrier(world, dev)
-        torch.cuda.synchronize(dev)
-        sampler.mark_start()
-        evs = timed_replays(g_stepG, g_step1, K)
-        s.synchronize()
-        torch.cuda.synchronize(dev)
-        barrier(world, dev)
-        sampler.mark_end()
-        clocks = sampler.stop()
-    local_step = ms_per(evs, K)
+    sampler = ClockSampler(local)
+    sampler.start()
+    local_step, step_min, step_max, reps = repeated_regions(g_stepG, g_step1, REGION_TARGET_S,
+                                                            sampler)
+    local_dc, dc_min, dc_max, dc_reps = repeated_regions(g_dcG, g_dc1, DC_TARGET_S, sampler)
+    clocks = sampler.stop()
 
     # per-stage breakdown: G consecutive steps captured with timing events
     # between the stages (event record nodes inside the graph); each replay is
@@ -595,22 +695,6 @@ def run_ours(args) -> None:
         stage_ms = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(4)] for e in rows_ms]).mean(0)
         stage_how = "one graph per stage, events between the replays"
         del gs
-    # dispatch+combine as the pages count it (layout + dispatch + combine,
-    # route excluded): its own graphs, timed the same way
-    dc_calls = calls if args.fused else calls[1:]   # fused: the route cannot be left out
-
-    def dc_step():
-        for fn, a in dc_calls:
-            rc = fn(*a)
-            if rc != 0:
-                raise moe.MoeError(rc, fn.__name__)
-    g_dc1 = capture(dc_step, 1)
-    g_dcG = capture(dc_step, G) if G > 1 else g_dc1
-    with torch.cuda.stream(s):
-        timed_replays(g_dcG, g_dc1, W)
-        dcev = timed_replays(g_dcG, g_dc1, K)
-        s.synchronize()
-    local_dc = ms_per(dcev, K)
 
     # eager: the same calls launched one by one from Python, no graph -- the
     # cost a caller that does not capture graphs pays (launch latency included)
@@ -698,71 +782,121 @@ def run_ours(args) -> None:
 
     peak, peak_kind = load_peak()
     n_gpus = world
-    value = n_gpus * nb["step"] / (ms_step * 1e-3) / 1e9
     comb_gbs = nb["combine"] / (ms_combine * 1e-3) / 1e9
-    dc_ms = ms_dc
     dc_bytes = nb["layout"] + nb["dispatch"] + nb["combine"]
-
+    dc_gbs = dc_bytes / (ms_dc * 1e-3) / 1e9
     if args.fused:
-        pipeline = ("fused: route + layout + dispatch in one cooperative launch "
-                    "(moe_route_dispatch), then combine")
         stages = {"route+layout+dispatch": (ms_route + ms_layout + ms_dispatch) * 1e3,
                   "combine": ms_combine * 1e3}
         dc_how = ("CUDA graphs of the fused route+layout+dispatch launch + combine (the route "
-                  "is inside the fused launch, so it is included), K steps timed like the step")
-        launches = 2 * K
+                  "is inside the fused launch, so it is included), K-step regions timed like the step")
+        kernels_per_step = 2
     else:
-        pipeline = ("two-phase: private-region layout, send into E*R private regions of T_r "
-                    "rows, receiver compaction" if args.two_phase
-                    else "direct scatter into the packed rows")
         stages = {"route": ms_route * 1e3, "layout": ms_layout * 1e3,
                   "dispatch": ms_dispatch * 1e3, "combine": ms_combine * 1e3}
-        dc_how = "CUDA graphs of layout + dispatch + combine, K steps timed like the step"
-        launches = (KERNELS_PER_STEP + (1 if args.two_phase else 0)) * K
+        dc_how = "CUDA graphs of layout + dispatch + combine, K-step regions timed like the step"
+        kernels_per_step = moe.kernels_per_step(T, k, E_lay, R, two_phase=args.two_phase)
+    res = {
+        "workload": cfg.describe(), "capacity": cap, "rows": rows, "l2": l2_mode,
+        "value": n_gpus * nb["step"] / (ms_step * 1e-3) / 1e9,
+        "ms_per_step": ms_step,
+        "us_per_layer": ms_step * 1e3,
+        "regions": {"steps_per_region": K, "repeats": reps, "median_us": ms_step * 1e3,
+                    "min_us": step_min * 1e3, "max_us": step_max * 1e3,
+                    "how": (f"{reps} regions of exactly K = {K} steps (replays of CUDA graphs of "
+                            f"{G} consecutive step(s)), each between a barrier and a device "
+                            "synchronise; the median region per rank, the maximum over ranks")},
+        "stages_us": stages,
+        "stage_timing": stage_how,
+        "eager": {"us_per_step": ms_eager * 1e3, "steps": K3,
+                  "how": "the same C ABI calls launched one by one, no CUDA graph, "
+                         "events around the steps (L2 as for the headline)"},
+        "dispatch_combine": {"us": ms_dc * 1e3, "bytes": dc_bytes, "how": dc_how,
+                             "repeats": dc_reps, "min_us": dc_min * 1e3, "max_us": dc_max * 1e3,
+                             "gbs": dc_gbs, "frac_of_8tbs": dc_gbs / SPEC_HBM_GBS,
+                             "frac_of_measured": dc_gbs / peak},
+        "bytes_per_step": nb,
+        "roofline": {"bound": "hbm",
+                     "kernel": "k_combine_fp8" if args.combine_fp8 else "k_combine_bf16",
+                     "achieved": comb_gbs,
+                     "peak": peak, "unit": "GB/s", "frac": comb_gbs / peak,
+                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
+                     if peak_kind == "measured" else "fallback 6650 GB/s",
+                     "traffic": combine_traffic(cfg.name, args.combine_fp8),
+                     "algorithmic_bytes_per_launch": nb["combine"],
+                     "how": "algorithmic bytes of one launch over the combine stage's mean "
+                            "CUDA-event time inside the step graph"},
+        "e2e": {"value": n_gpus * nb["step"] / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                "us_per_step": e2e_ms * 1e3, "h2d_bytes_per_step": h2d,
+                "how": ("C ABI calls launched per step; every step's inputs copied in from "
+                        "pinned host memory and its output copied out, on two copy "
+                        "streams overlapping the neighbouring steps' compute; inputs and "
+                        "output double-buffered; no L2 flush"),
+                "d2h_bytes_per_step": d2h},
+        "kernels_per_step": kernels_per_step,
+        "clocks": clocks,
+    }
+    sm = clocks.get("sm_mhz")
+    if sm:
+        res["clocks"]["us_x_mhz"] = ms_step * 1e3 * sm
+        res["clocks"]["dispatch_combine_us_x_mhz"] = ms_dc * 1e3 * sm
+    del calls, calls2, sets
+    return res
+
+
+def summary(res: dict) -> dict:
+    """A workload's entry in the line's `configs`."""
+    dc = res["dispatch_combine"]
+    return {"workload": res["workload"], "us_per_layer": res["us_per_layer"], "value": res["value"],
+            "unit": "GB/s", "regions": res["regions"], "stages_us": res["stages_us"],
+            "eager_us": res["eager"]["us_per_step"],
+            "dispatch_combine": {k: dc[k] for k in ["us", "gbs", "frac_of_8tbs", "frac_of_measured",
+                                                    "bytes", "repeats", "min_us", "max_us"]},
+            "roofline": {k: res["roofline"][k] for k in ["kernel", "achieved", "peak", "frac",
+                                                         "traffic"]},
+            "e2e_us": res["e2e"]["us_per_step"], "clocks": res["clocks"],
+            "capacity": res["capacity"], "rows": res["rows"], "l2": res["l2"]}
+
+
+def run_ours(args) -> None:
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_dist(world, "nccl")
+    names = config_names(args.config)
+    head = headline_name(names)
+    results = {}
+    for name in names:
+        results[name] = measure(inputs.CONFIGS[name], args, dev, world, local)
+        torch.cuda.synchronize(dev)
+        torch.cuda.empty_cache()
+    hr = results[head]
+    K, W = args.steps, args.warmup
     if rank == 0:
         line = {
-            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": n_gpus, "steps": K,
-            "warmup": W, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": cfg.describe(), "parallelism": f"replicas x{n_gpus}",
-                       "l2": l2_mode,
-                       "capacity": cap, "rows": rows,
-                       "pipeline": pipeline,
-                       "combine_payload": ("fp8 e4m3 + 1x128 fp32 scales (the dispatched rows)"
-                                           if args.combine_fp8 else "bf16 (stand-in expert output)"), "timing": (f"CUDA events around K steps run as replays of CUDA graphs of "
-                                  f"{G} consecutive step(s)")},
-            "us_per_layer": ms_step * 1e3,
-            "stages_us": stages,
-            "eager": {"us_per_step": ms_eager * 1e3, "steps": K3,
-                      "how": "the same C ABI calls launched one by one, no CUDA graph, "
-                             "events around the steps (L2 as for the headline)"},
-            "dispatch_combine": {"us": dc_ms * 1e3, "bytes": dc_bytes,
-                                 "how": dc_how,
-                                 "gbs": dc_bytes / (dc_ms * 1e-3) / 1e9,
-                                 "frac_of_8tbs": dc_bytes / (dc_ms * 1e-3) / 1e9 / SPEC_HBM_GBS,
-                                 "frac_of_measured": dc_bytes / (dc_ms * 1e-3) / 1e9 / peak},
-            "stage_timing": stage_how,
-            "bytes_per_step": nb,
-            "roofline": {"bound": "hbm",
-                         "kernel": "k_combine_fp8" if args.combine_fp8 else "k_combine_bf16",
-                         "achieved": comb_gbs,
-                         "peak": peak, "unit": "GB/s", "frac": comb_gbs / peak,
-                         "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
-                         else "fallback 6650 GB/s",
-                         "traffic": combine_traffic(cfg.name, args.combine_fp8),
-                         "algorithmic_bytes_per_launch": nb["combine"]},
-            "e2e": {"value": n_gpus * nb["step"] / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
-                    "us_per_step": e2e_ms * 1e3, "h2d_bytes_per_step": h2d,
-                    "how": ("C ABI calls launched per step; every step's inputs copied in from "
-                            "pinned host memory and its output copied out, on two copy "
-                            "streams overlapping the neighbouring steps' compute; inputs and "
-                            "output double-buffered; no L2 flush"),
-                    "d2h_bytes_per_step": d2h},
-            "gpu_launches": launches,
-            "clocks": clocks,
+            "metric": METRIC, "value": hr["value"], "unit": "GB/s", "n_gpus": world, "steps": K,
+            "warmup": W, "ms_per_step": hr["ms_per_step"], "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16+e4m3", "dtypes": DTYPES,
+            "data": "synthetic",
+            "config": line_config(args, names, world),
+            "headline": head,
+            "us_per_layer": hr["us_per_layer"],
+            "timing": hr["regions"]["how"],
+            "stages_us": hr["stages_us"],
+            "stage_timing": hr["stage_timing"],
+            "eager": hr["eager"],
+            "dispatch_combine": hr["dispatch_combine"],
+            "bytes_per_step": hr["bytes_per_step"],
+            "roofline": hr["roofline"],
+            "e2e": hr["e2e"],
+            "gpu_launches": hr["kernels_per_step"] * K,
+            "gpu_launches_how": (f"{hr['kernels_per_step']} library kernels per step x K = {K} "
+                                 "steps per timed region (each region repeated, see timing)"),
+            "clocks": hr["clocks"],
+            "configs": {n: summary(r) for n, r in results.items()},
         }
         if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(cfg)
+            line["cpu_baseline"] = cpu_baseline(inputs.CONFIGS[head])
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
@@ -774,12 +908,13 @@ def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1,
                     help="ranks (one per GPU, launched by torch.distributed.run): independent replicas")
-    ap.add_argument("--steps", type=int, default=2000, help="timed steps")
-    ap.add_argument("--warmup", type=int, default=20, help="untimed warm-up steps")
+    ap.add_argument("--steps", type=int, default=20, help="steps per timed region")
+    ap.add_argument("--warmup", type=int, default=5, help="untimed warm-up steps")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours",
-                    help="reference: time the CPU oracle on samples of the same workload")
-    ap.add_argument("--config", choices=sorted(inputs.CONFIGS), default="dsv3",
-                    help="seeded synthetic workload")
+                    help="reference: time the CPU oracle on samples of the headline workload")
+    ap.add_argument("--config", default=DEFAULT_CONFIGS,
+                    help="comma-separated seeded synthetic workloads, measured in turn; the "
+                         f"largest is the headline (choices: {', '.join(sorted(inputs.CONFIGS))})")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip timing the oracle on the host (cpu_baseline)")
     ap.add_argument("--two-phase", action="store_true",
@@ -791,6 +926,9 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.steps < 1:
+        ap.error("--steps must be at least 1")
+    config_names(args.config)
     if args.impl == "reference":
         run_reference(args)
     else:
