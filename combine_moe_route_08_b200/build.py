@@ -51,17 +51,36 @@ def nvcc() -> str:
     return "nvcc"
 
 
-def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None) -> str:
-    """Compile every .cu under csrc/ into one shared library (static cudart)."""
-    if not force and not _stale():
-        return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc(), *NVCC_FLAGS, *(extra or []), "-I", INCLUDE, "-I", CSRC, "-o", tmp, *sources()]
-    if verbose:
-        print(" ".join(cmd), flush=True)
-    subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None,
+          csrc: str = CSRC, out: str = LIB) -> str:
+    """Compile every .cu under csrc/ into one shared library (static cudart):
+    one nvcc process per source file, in parallel, then one link."""
+    if not force and out == LIB and not _stale():
+        return out
+    import concurrent.futures as cf
+    srcs = sorted(glob.glob(os.path.join(csrc, "*.cu")))
+    objdir = os.path.join(os.path.dirname(out), "_build", f"obj{os.getpid()}")
+    os.makedirs(objdir, exist_ok=True)
+    compile_flags = [f for f in NVCC_FLAGS if f != "-shared"]
+
+    def one(src):
+        obj = os.path.join(objdir, os.path.basename(src) + ".o")
+        cmd = [nvcc(), *compile_flags, *(extra or []), "-I", INCLUDE, "-I", csrc, "-c", "-o", obj, src]
+        if verbose:
+            print(" ".join(cmd), flush=True)
+        subprocess.run(cmd, check=True)
+        return obj
+
+    with cf.ThreadPoolExecutor(max_workers=min(len(srcs), os.cpu_count() or 4)) as pool:
+        objs = list(pool.map(one, srcs))
+    tmp = out + f".tmp{os.getpid()}"
+    subprocess.run([nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", tmp, *objs],
+                   check=True)
+    os.replace(tmp, out)
+    for o in objs:
+        os.remove(o)
+    os.rmdir(objdir)
+    return out
 
 
 if __name__ == "__main__":

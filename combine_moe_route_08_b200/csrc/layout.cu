@@ -19,8 +19,8 @@
 // 32 warps a contiguous run of at most 2 x 32 slots, which every lane keeps in
 // registers (one load round trip per kernel).
 //
-//   k_layout_hist    chunk histogram (per-warp aggregation of equal experts,
-//                    shared-memory atomics) -> workspace hist[chunk][E].
+//   k_layout_hist    chunk histogram (shared-memory atomics; small CTAs)
+//                    -> workspace hist[chunk][E].
 //   k_layout_assign  every CTA sums the histogram columns it needs (the base
 //                    of its chunk inside each expert, the expert totals, its
 //                    rank's source counts) with all its threads -- redundant
@@ -34,15 +34,20 @@
 // The kernel boundary between the two is the only grid-wide ordering; nothing
 // waits on another CTA.
 //
-// Decode-sized layouts (one chunk per logical rank, at most 8 steps of 32
-// slots per warp) take a single launch instead: k_layout_cluster, one
-// thread-block cluster of at most 8 CTAs.  Each CTA owns a run of whole ranks,
+// Small layouts (one chunk per logical rank and at most one slot per thread
+// of an 8-CTA cluster: T*k <= 8192, e.g. the Mixtral-like workload) take a
+// single launch instead: k_layout_cluster, one thread-block cluster of at
+// most 8 CTAs.  Each CTA owns a run of whole ranks,
 // counts them per warp, and publishes its per-expert totals in its own shared
 // memory; one cluster barrier later every CTA reads the others' totals over
 // distributed shared memory, scans, and ranks its slots exactly as
 // k_layout_assign does.  The grid-wide ordering is then the hardware cluster
 // barrier (all CTAs of a cluster are co-scheduled), not a kernel boundary
-// plus a global round trip through the workspace.
+// plus a global round trip through the workspace.  Larger layouts keep the
+// pair: with 4096 slots per SM (T = 4096, k = 8) the single cluster measured
+// 11.9 against 9.0 us per layout, its per-warp equality masks and ranking
+// steps then costing about 0.7 us each on eight SMs; at 1024 slots it saves
+// about 0.9 us (5.1 against 5.9 us).
 //
 // The warp-level pieces (equality masks, per-warp histograms and bases, the
 // block scan) are in layout_dev.cuh.
@@ -102,39 +107,47 @@ __device__ __forceinline__ void load_run(const int32_t *__restrict__ topk_idx, i
     }
 }
 
-__global__ void __launch_bounds__(kThreads)
+// The histogram needs no order, so it runs in small CTAs: kHistThreads
+// threads take the chunk's slots in strides, one shared-memory atomic per
+// slot.  Small CTAs fit beside the route kernel's resident CTAs, so they are
+// in place (waiting) when the route finishes, where a 1024-thread CTA must
+// wait for a whole SM to drain first.
+constexpr int kHistThreads = 256;
+constexpr int kHistSlots = kChunkSlots / kHistThreads;  // slots per thread, at most
+
+__global__ void __launch_bounds__(kHistThreads)
     k_layout_hist(const int32_t *__restrict__ topk_idx, LayoutGeom G,
                   int32_t *__restrict__ ws_hist, int32_t *__restrict__ dev_status)
 {
     extern __shared__ int32_t h[];  // [E]
-    const int E = G.E, lane = threadIdx.x & 31;
+    const int E = G.E;
     const int c = blockIdx.x;
-    const int nb = key_bits(E);
-    int64_t w0, w1;
-    warp_run(G, c, w0, w1);
-    for (int x = threadIdx.x; x < E; x += kThreads)
+    int t0, t1;
+    chunk_tokens(G, c, t0, t1);
+    const int64_t i0 = static_cast<int64_t>(t0) * G.k, i1 = static_cast<int64_t>(t1) * G.k;
+    for (int x = threadIdx.x; x < E; x += kHistThreads)
         h[x] = 0;
     pdl_trigger();  // the next kernel may take idle SM slots now; it waits for this one
     pdl_wait();
-    int e[kMaxSteps];
-    load_run(topk_idx, w0, w1, e);
+    int e[kHistSlots];
+#pragma unroll
+    for (int s = 0; s < kHistSlots; ++s) {
+        const int64_t i = i0 + s * kHistThreads + threadIdx.x;
+        e[s] = (i < i1) ? __ldg(topk_idx + i) : -1;
+    }
     __syncthreads();
-
     bool bad = false;
 #pragma unroll
-    for (int s = 0; s < kMaxSteps; ++s) {
-        if (w0 + 32 * s >= w1)
-            break;  // warp-uniform
+    for (int s = 0; s < kHistSlots; ++s) {
         const bool valid = static_cast<unsigned>(e[s]) < static_cast<unsigned>(E);
-        bad |= !valid && e[s] != -1 && (w0 + 32 * s + lane < w1);
-        const unsigned mask = match_mask(match_key(e[s], E, lane, nb), nb);
-        if (valid && lane == __ffs(mask) - 1)
-            atomicAdd(&h[e[s]], __popc(mask));
+        bad |= !valid && e[s] != -1;  // -1 past the chunk's end too
+        if (valid)  // counts are order-free: one shared-memory atomic per slot
+            atomicAdd(&h[e[s]], 1);
     }
     if (bad)
         report(dev_status, MOE_ERR_INVALID_ARG);
     __syncthreads();
-    for (int x = threadIdx.x; x < E; x += kThreads)
+    for (int x = threadIdx.x; x < E; x += kHistThreads)
         ws_hist[static_cast<size_t>(c) * E + x] = h[x];
 }
 
@@ -144,10 +157,10 @@ __global__ void __launch_bounds__(kThreads)
 // threads per column group each sum a contiguous share of the n chunk rows;
 // V = 4 reads four experts per 16-byte load (E % 4 == 0, rows 16-byte
 // aligned), V = 1 one per 4-byte load; B loads in flight per thread.  Share
-// `part` writes rows 4*part .. 4*part+3 of wh (before, total, mine, rstart).
+// `part` writes rows 4*part .. 4*part+3 of out (before, total, mine, rstart).
 template <int V, int B>
 __device__ __forceinline__ void column_sums(const int32_t *__restrict__ ws_hist, int n, int c, int r0,
-                                            int r1, int E, int P, int32_t *wh)
+                                            int r1, int E, int P, int32_t *out)
 {
     using Vec = typename std::conditional<V == 4, int4, int>::type;
     const int EV = E / V;
@@ -184,13 +197,24 @@ __device__ __forceinline__ void column_sums(const int32_t *__restrict__ ws_hist,
 #pragma unroll
     for (int q = 0; q < V; ++q) {
         const int x = V * xv + q;
-        wh[(4 * part) * E + x] = before[q];
-        wh[(4 * part + 1) * E + x] = total[q];
-        wh[(4 * part + 2) * E + x] = mine[q];
-        wh[(4 * part + 3) * E + x] = rstart[q];
+        out[(4 * part) * E + x] = before[q];
+        out[(4 * part + 1) * E + x] = total[q];
+        out[(4 * part + 2) * E + x] = mine[q];
+        out[(4 * part + 3) * E + x] = rstart[q];
     }
 }
 
+// Shares per histogram column: as many as the threads allow, at most
+// kWarps / 4 (kColBatch4 or kColBatch rows in flight per thread).
+__host__ __device__ inline int column_shares(int E)
+{
+    const int per_share = (E % 4 == 0) ? E / 4 : E;
+    const int p = kThreads / per_share;
+    return p < 1 ? 1 : (p > kWarps / 4 ? kWarps / 4 : p);
+}
+
+// Shared memory: wh[kWarps][E] per-warp counts, then bases; parts[4P][E]
+// column-sum shares; off[E + 1]; chb[E]; rbs[E]; tot[kWarps + 1].
 __global__ void __launch_bounds__(kThreads)
     k_layout_assign(const int32_t *__restrict__ topk_idx, LayoutGeom G, int capacity, int64_t rows,
                     const int32_t *__restrict__ ws_hist, int32_t *__restrict__ expert_counts,
@@ -202,8 +226,10 @@ __global__ void __launch_bounds__(kThreads)
     extern __shared__ int32_t sm[];
     const int E = G.E, lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     const int nb = key_bits(E);
+    const int P = column_shares(E);
     int32_t *wh = sm;                   // [kWarps][E] per-warp counts, then bases
-    int32_t *off = wh + kWarps * E;     // [E + 1] expert totals, then their scan
+    int32_t *parts = wh + kWarps * E;   // [4P][E] column-sum shares
+    int32_t *off = parts + 4 * P * E;   // [E + 1] expert totals, then their scan
     int32_t *chb = off + E + 1;         // [E] slots of e in earlier chunks
     int32_t *rbs = chb + E;             // [E] slots of e in chunks of earlier ranks
     int32_t *tot = rbs + E;             // [kWarps + 1]
@@ -211,36 +237,33 @@ __global__ void __launch_bounds__(kThreads)
 
     int64_t w0, w1;
     warp_run(G, c, w0, w1);
+    for (int x = threadIdx.x; x < kWarps * E; x += kThreads)
+        wh[x] = 0;  // before the wait: nothing upstream is read
     pdl_trigger();  // the next kernel may take idle SM slots now; it waits for this one
     pdl_wait();
     int e[kMaxSteps];
     load_run(topk_idx, w0, w1, e);  // in flight while the columns are summed
 
-    // shares per column: as many as the threads allow (rows 4 * P of wh)
-    const bool vec = (E % 4 == 0);
-    const int P = max(1, min(kThreads / (vec ? E / 4 : E), kWarps / 4));
-    for (int x = threadIdx.x + 4 * P * E; x < kWarps * E; x += kThreads)
-        wh[x] = 0;
-
     // histogram columns: base of this chunk inside each expert (earlier
     // chunks), expert totals, and this chunk's rank column of the
     // per-source-rank counts.  P threads per expert each sum a contiguous
-    // part of the chunks (coalesced over experts); the parts meet in shared
-    // memory (the per-warp rows, not yet used).
+    // part of the chunks (coalesced over experts); the parts meet below.
     const int n = G.nchunks;
     const int r = c / G.cpr;
-    if (vec)  // CTA-uniform
-        column_sums<4, kColBatch4>(ws_hist, n, c, r * G.cpr, (r + 1) * G.cpr, E, P, wh);
+    if (E % 4 == 0)  // CTA-uniform
+        column_sums<4, kColBatch4>(ws_hist, n, c, r * G.cpr, (r + 1) * G.cpr, E, P, parts);
     else
-        column_sums<1, kColBatch>(ws_hist, n, c, r * G.cpr, (r + 1) * G.cpr, E, P, wh);
-    __syncthreads();
+        column_sums<1, kColBatch>(ws_hist, n, c, r * G.cpr, (r + 1) * G.cpr, E, P, parts);
+    __syncthreads();  // wh zeroed by every thread before any warp counts into it
+    // per-warp counts of this CTA's slots (order-free: shared-memory atomics)
+    warp_count(e, w0, w1, E, wh + w * E);
     for (int x = threadIdx.x; x < E; x += kThreads) {
         int before = 0, total = 0, mine = 0, rstart = 0;
         for (int part = 0; part < P; ++part) {
-            before += wh[(4 * part) * E + x];
-            total += wh[(4 * part + 1) * E + x];
-            mine += wh[(4 * part + 2) * E + x];
-            rstart += wh[(4 * part + 3) * E + x];
+            before += parts[(4 * part) * E + x];
+            total += parts[(4 * part + 1) * E + x];
+            mine += parts[(4 * part + 2) * E + x];
+            rstart += parts[(4 * part + 3) * E + x];
         }
         off[x] = total;
         chb[x] = before;
@@ -251,15 +274,7 @@ __global__ void __launch_bounds__(kThreads)
             expert_src_counts[static_cast<size_t>(x) * G.R + r] = mine;
     }
     __syncthreads();
-    for (int x = threadIdx.x; x < 4 * P * E; x += kThreads)
-        wh[x] = 0;
-    __syncthreads();
-
-    // per-warp histogram of this CTA's slots (warp-private rows: no atomics)
-    int32_t *mywh = wh + w * E;
-    warp_histogram(e, w0, w1, E, nb, mywh);
     block_exclusive_scan<kWarps>(off, E, tot);  // off[e] = slots of experts < e; off[E] = total
-
     if (c == 0) {
         for (int x = threadIdx.x; x <= E; x += kThreads)
             expert_offsets[x] = (capacity == 0) ? off[x] : x * capacity;
@@ -268,8 +283,9 @@ __global__ void __launch_bounds__(kThreads)
             rank_counts[rr] = off[(rr + 1) * L] - off[rr * L];
     }
     // per-warp base of each expert's positions: earlier chunks + earlier warps
-    warp_bases<kWarps>(wh, chb, E);
+    warp_bases_par<kWarps>(wh, chb, E);
     __syncthreads();
+    int32_t *mywh = wh + w * E;
 
     // rank every slot among equal experts, in slot order
     bool dropped = false, bad_row = false;
@@ -338,7 +354,7 @@ __global__ void __launch_bounds__(kThreads)
 // Single-launch layout for one chunk per rank (decode sizes): one cluster.
 
 constexpr int kClusterMax = 8;        // CTAs of the cluster (portable cluster size)
-constexpr int kClusterSteps = 8;      // 32-slot steps per warp, at most
+constexpr int kClusterSteps = 2;      // 32-slot steps per warp, at most
 constexpr int kClusterMaxE = 1024;
 
 __device__ __forceinline__ unsigned cluster_ctarank()
@@ -415,7 +431,7 @@ __global__ void __launch_bounds__(kThreads)
     if (bad)
         report(dev_status, MOE_ERR_INVALID_ARG);
     __syncthreads();
-    warp_histogram(e, w0, w1, E, nb, wh + w * E);
+    warp_count(e, w0, w1, E, wh + w * E);
     __syncthreads();
 
     // per expert: in-CTA exclusive prefix over the warps (slot order), each
@@ -527,7 +543,10 @@ __global__ void __launch_bounds__(kThreads)
     cluster_wait();  // no CTA exits while another may still read its tot
 }
 
-size_t assign_smem_bytes(int E) { return (static_cast<size_t>(kWarps + 3) * E + 1 + kWarps + 1) * sizeof(int32_t); }
+size_t assign_smem_bytes(int E)
+{
+    return (static_cast<size_t>(kWarps + 4 * column_shares(E) + 3) * E + 1 + kWarps + 1) * sizeof(int32_t);
+}
 
 }  // namespace
 
@@ -554,10 +573,10 @@ size_t layout_workspace_bytes(const LayoutGeom &g)
 
 namespace {
 
-// The single-launch plan for a geometry, or ok = false when it does not fit:
-// more than one chunk per rank, E beyond the kernel's limit, runs longer than
-// kClusterSteps steps per warp, shared memory beyond the device's opt-in
-// limit, or a device that cannot schedule such a cluster.
+// The single-launch plan for a geometry, or ok = false when it does not pay
+// or fit: more than one chunk per rank, more slots than one per thread of
+// the CTAs, E beyond the kernel's limit, shared memory beyond the device's
+// opt-in limit, or a device that cannot schedule such a cluster.
 struct ClusterPlan {
     bool ok = false;
     int C = 0, cpb = 0, wpc = 0, seg = 0;
@@ -625,6 +644,8 @@ ClusterPlan cluster_plan(const LayoutGeom &g)
         return p;
     const int wpc = kWarps / cpb;
     const int slots = g.Tr * g.k;
+    if (static_cast<int64_t>(cpb) * slots > kThreads)
+        return p;  // more work per SM than the two-kernel form spreads over more SMs
     const int seg = round_up(ceil_div(slots, wpc), 32);
     if (seg > 32 * kClusterSteps)
         return p;
@@ -676,8 +697,8 @@ cudaError_t dispatch_layout(const int32_t *topk_idx, const LayoutGeom &g, int ca
                                   expert_offsets, dispatch_pos, recv_src, private_pos, dev_status);
     }
     int32_t *hist = static_cast<int32_t *>(workspace);
-    cudaError_t err = launch_pdl(k_layout_hist, dim3(g.nchunks), dim3(kThreads), g.E * sizeof(int32_t),
-                                 s, topk_idx, g, hist, dev_status);
+    cudaError_t err = launch_pdl(k_layout_hist, dim3(g.nchunks), dim3(kHistThreads),
+                                 g.E * sizeof(int32_t), s, topk_idx, g, hist, dev_status);
     if (err != cudaSuccess)
         return err;
     const size_t smem = assign_smem_bytes(g.E);

@@ -51,7 +51,9 @@ __device__ __forceinline__ int match_key(int e, int E, int lane, int nbits)
 }
 
 // Count the warp run's slots per expert into the warp's private row `mywh`
-// (one add per distinct expert of a step, by its lowest lane; no atomics).
+// with one add per distinct expert of a step, by its lowest lane (no
+// atomics; the equality masks cost more instructions than warp_count's
+// atomics but fewer registers, which the fused kernel's budget needs).
 template <int MAXS>
 __device__ __forceinline__ void warp_histogram(const int (&e)[MAXS], int64_t w0, int64_t w1, int E,
                                                int nb, int32_t *mywh)
@@ -69,18 +71,57 @@ __device__ __forceinline__ void warp_histogram(const int (&e)[MAXS], int64_t w0,
     }
 }
 
-// Turn the per-warp rows wh[NW][E] into per-warp bases: chb[x] (slots of x
-// in earlier chunks) plus the counts of the earlier warps.
-template <int NW>
-__device__ __forceinline__ void warp_bases(int32_t *wh, const int32_t *chb, int E)
+// Count the warp run's slots per expert into the warp's private row `mywh`
+// with one shared-memory atomic per slot: counts do not depend on the order
+// in which they are added, so atomics are safe here (unlike positions).
+template <int MAXS>
+__device__ __forceinline__ void warp_count(const int (&e)[MAXS], int64_t w0, int64_t w1, int E,
+                                           int32_t *mywh)
 {
-    for (int x = threadIdx.x; x < E; x += NW * 32) {
-        int run = chb[x];
-#pragma unroll 8
-        for (int ww = 0; ww < NW; ++ww) {
-            const int t = wh[ww * E + x];
-            wh[ww * E + x] = run;
-            run += t;
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int s = 0; s < MAXS; ++s)
+        if (w0 + 32 * s + lane < w1 && static_cast<unsigned>(e[s]) < static_cast<unsigned>(E))
+            atomicAdd(mywh + e[s], 1);
+}
+
+// Turn the per-warp rows wh[NW][E] into per-warp bases: chb[x] (slots of x
+// in earlier chunks) plus the counts of the earlier warps.  The whole CTA of
+// NW warps takes part: G adjacent lanes per expert (G a power of two, G * E
+// <= NW * 32 when it can be above 1) each sum the counts of NW / G
+// consecutive warps, scan their G partial sums by shuffles, then rewrite
+// their warps' rows as running bases (chains G times shorter than one thread
+// per expert walking all NW rows).  Called by every thread.
+template <int NW>
+__device__ __forceinline__ void warp_bases_par(int32_t *wh, const int32_t *chb, int E)
+{
+    int G = 1;
+    while (2 * G <= NW && 2 * G * E <= NW * 32)
+        G *= 2;
+    const int per = NW / G;
+    // whole warps (every lane takes part in the shuffles); more than one pass
+    // only when E exceeds the CTA's threads (then G = 1)
+    const int span = (E * G + 31) / 32 * 32;
+    for (int idx = threadIdx.x; idx < span; idx += NW * 32) {
+        const int x = idx / G, part = idx % G;
+        const bool valid = x < E;
+        int sum = 0;
+        if (valid)
+            for (int ww = part * per; ww < (part + 1) * per; ++ww)
+                sum += wh[ww * E + x];
+        int incl = sum;
+        for (int o = 1; o < G; o <<= 1) {
+            const int t = __shfl_up_sync(kFullMask, incl, o, G);
+            if (part >= o)
+                incl += t;
+        }
+        if (valid) {
+            int run = chb[x] + incl - sum;
+            for (int ww = part * per; ww < (part + 1) * per; ++ww) {
+                const int t = wh[ww * E + x];
+                wh[ww * E + x] = run;
+                run += t;
+            }
         }
     }
 }

@@ -66,51 +66,63 @@ __device__ __forceinline__ float warp_total_f64(double sum)
     return __shfl_sync(kFullMask, __double2float_rn(sum), 0);
 }
 
+// Order-preserving 32-bit key of a logit: larger logit -> larger key, -0 and
+// +0 the same key (x + 0.0f turns -0 into +0); key 0 is never produced for a
+// finite or infinite logit and marks a taken or absent slot.
+__device__ __forceinline__ uint32_t logit_key(float x)
+{
+    const uint32_t u = __float_as_uint(__fadd_rn(x, 0.0f));
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// The logit a key came from (the map is invertible; -0 comes back as +0,
+// which gives the same softmax terms).
+__device__ __forceinline__ float key_logit(uint32_t m)
+{
+    return __uint_as_float((m & 0x80000000u) ? (m & 0x7fffffffu) : ~m);
+}
+
 // Route one token with the whole warp: on return lane j < k holds the j-th
 // chosen expert (logit descending, index ascending among equal logits) in
 // `my_e` and its weight in `my_w` (the softmax probability over all E, or
 // over the k chosen ones with `renormalize`).  Other lanes' outputs are 0.
-// NPL = logits per lane, NPL * 32 >= E.  Called by all 32 lanes.
-template <int NPL>
+// NPL = logits per lane, NPL * 32 >= E.  KT > 0: k == KT known at compile
+// time (the rounds unroll); KT == 0: k at run time.  Called by all 32 lanes.
+//
+// Lane l holds experts l, l + 32, ...: hot experts of a skewed router (a
+// Zipf-like bias on the lowest ids) fall on different lanes, so a lane
+// rarely wins more rounds than its two best keys cover.  (Holding eight
+// consecutive experts per lane, loaded as two 16-byte vectors, measured the
+// same at dsv3 and prefill but 12.3 against 8.4 us at the skewed kimi
+// workload: lane 0 won most rounds and rescanned.)
+template <int NPL, int KT = 0>
 __device__ __forceinline__ void route_warp(const float *__restrict__ row, int E, int k,
                                            int renormalize, int &my_e, float &my_w)
 {
     const int lane = threadIdx.x & 31;
     float v[NPL];
-    uint32_t gone = 0;  // bit i: element i past E
+    uint32_t key[NPL];
+    uint32_t gone = 0;  // bit i: slot i taken or past E
 #pragma unroll
     for (int i = 0; i < NPL; ++i) {
         const int e = i * 32 + lane;
         if (e < E) {
             v[i] = __ldg(row + e);
+            key[i] = logit_key(v[i]);
         } else {
             v[i] = -FLT_MAX;
+            key[i] = 0u;
             gone |= 1u << i;
         }
     }
 
-    // selection on order-preserving 32-bit keys: larger logit -> larger key,
-    // -0 and +0 the same key (x + 0.0f turns -0 into +0); key 0 = taken/absent
-    uint32_t key[NPL];
-#pragma unroll
-    for (int i = 0; i < NPL; ++i) {
-        if ((gone >> i) & 1u) {
-            key[i] = 0u;
-        } else {
-            const uint32_t u = __float_as_uint(__fadd_rn(v[i], 0.0f));
-            key[i] = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-        }
-    }
-    // Each lane keeps its best key and slot and, while known, its second
-    // best (order: key descending, slot ascending; the lowest slot among
-    // equal keys first).  A round is one warp max of the lanes' bests and one
-    // warp min of the expert ids holding it; the winning lane then promotes
-    // its second best, and only a lane that wins again with no second left
-    // rescans its remaining keys (bit i of `gone`: slot i taken or past E).
-    // With k = 8 over 32 lanes most rounds need no rescan.  The chosen logit
-    // is read back from the winning key (the map is invertible; -0 comes back
-    // as +0, which gives the same softmax terms).
-    uint32_t b1 = 0u, b2 = 0u;  // best and second-best key (0: none)
+    // Each lane keeps its best key b1 (slot i1) and, while known, its second
+    // best b2 (order: key descending, slot ascending, so the lower expert
+    // first among equal keys).  A round is one warp max of the lanes' bests
+    // and one warp min of the expert ids holding it (redux.sync); the lane
+    // whose expert won promotes its second best, and only a lane that wins
+    // again with no second left rescans its remaining keys.
+    uint32_t b1 = 0u, b2 = 0u;
     int i1 = 0, i2 = 0;
     auto top2 = [&]() {
         b1 = 0u;
@@ -133,15 +145,20 @@ __device__ __forceinline__ void route_warp(const float *__restrict__ row, int E,
     };
     top2();
     my_e = 0;
-    float my_v = 0.0f;
-    float vmax = 0.0f;
-    for (int j = 0; j < k; ++j) {
+    uint32_t my_key = 0u, m0 = 0u;
+    const int nk = (KT > 0) ? KT : k;
+#pragma unroll(KT > 0 ? KT : 1)
+    for (int j = 0; j < nk; ++j) {
         const uint32_t m = __reduce_max_sync(kFullMask, b1);
         const uint32_t cand = (b1 == m) ? static_cast<uint32_t>(i1 * 32 + lane) : 0xffffffffu;
         const uint32_t e = __reduce_min_sync(kFullMask, cand);
-        const uint32_t u = (m & 0x80000000u) ? (m & 0x7fffffffu) : ~m;
-        const float ve = __uint_as_float(u);
-        if ((e & 31u) == static_cast<uint32_t>(lane)) {  // the winner moves to its next best
+        if (lane == j) {
+            my_key = m;
+            my_e = static_cast<int>(e);
+        }
+        if (j == 0)
+            m0 = m;
+        if (e == cand) {  // this lane's best was chosen: move to its next best
             gone |= 1u << i1;
             if (b2 != 0u) {
                 b1 = b2;
@@ -151,13 +168,9 @@ __device__ __forceinline__ void route_warp(const float *__restrict__ row, int E,
                 top2();  // taken keys are skipped
             }
         }
-        if (lane == j) {
-            my_e = static_cast<int>(e);
-            my_v = ve;
-        }
-        if (j == 0)
-            vmax = ve;
     }
+    const float vmax = key_logit(m0);
+    const float my_v = key_logit(my_key);
 
     // softmax over all E logits: fp32 terms, binary64 sum
     double sum = 0.0;

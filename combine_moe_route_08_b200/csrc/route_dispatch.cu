@@ -543,7 +543,7 @@ __global__ void __launch_bounds__(kThreads, (NPL <= 12) ? 2 : 1)
         int32_t *mywh = wh + w * E;
         warp_histogram(e, w0, w1, E, nb, mywh);
         __syncthreads();
-        warp_bases<kWarps>(wh, chb, E);
+        warp_bases_par<kWarps>(wh, chb, E);
         __syncthreads();
 #pragma unroll
         for (int s = 0; s < kMaxSteps; ++s) {

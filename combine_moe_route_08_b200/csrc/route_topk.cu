@@ -16,8 +16,11 @@ namespace {
 
 constexpr int kRouteWarps = 8;  // tokens per CTA
 
-template <int NPL, bool EX>
-__global__ void __launch_bounds__(kRouteWarps * 32)
+// At most 1024 experts (NPL = 32) a lane holds 32 logits and their keys: the
+// register budget is left open there (one CTA per SM suffices to fill the
+// grid's few warps per token) so nothing spills.
+template <int NPL, bool EX, int KT>
+__global__ void __launch_bounds__(kRouteWarps * 32, NPL >= 24 ? 1 : 4)
     k_route_topk(const float *__restrict__ logits, int T, int E, int k, int renormalize,
                  int32_t *__restrict__ topk_idx, float *__restrict__ topk_w, RouteEx ex)
 {
@@ -36,7 +39,7 @@ __global__ void __launch_bounds__(kRouteWarps * 32)
 
     int my_e;
     float my_w;
-    route_warp<NPL>(row, E, k, renormalize, my_e, my_w);
+    route_warp<NPL, KT>(row, E, k, renormalize, my_e, my_w);
     if (!EX) {
         if (lane < k) {
             topk_idx[static_cast<size_t>(g) * k + lane] = my_e;
@@ -67,16 +70,28 @@ __global__ void __launch_bounds__(kRouteWarps * 32)
     }
 }
 
+template <int NPL, int KT>
+cudaError_t launch_kt(const float *logits, int T, int E, int k, int renormalize, int32_t *idx,
+                      float *w, const RouteEx *ex, cudaStream_t s)
+{
+    const int grid = ceil_div(T, kRouteWarps);
+    if (ex == nullptr)
+        return launch_pdl(k_route_topk<NPL, false, KT>, dim3(grid), dim3(kRouteWarps * 32), 0, s,
+                          logits, T, E, k, renormalize, idx, w, RouteEx{});
+    return launch_pdl(k_route_topk<NPL, true, KT>, dim3(grid), dim3(kRouteWarps * 32), 0, s, logits,
+                      T, E, k, renormalize, idx, w, *ex);
+}
+
+// k = 8 (the decode and prefill routers) unrolls its rounds: 7.4 -> 6.2 us
+// for 4096 tokens at E = 256 (with the other changes of route_warp,
+// 8.2 -> 6.2 us; prefill 32.8 -> 24.3 us, kimi 12.1 -> 8.4 us).
 template <int NPL>
 cudaError_t launch(const float *logits, int T, int E, int k, int renormalize, int32_t *idx,
                    float *w, const RouteEx *ex, cudaStream_t s)
 {
-    const int grid = ceil_div(T, kRouteWarps);
-    if (ex == nullptr)
-        return launch_pdl(k_route_topk<NPL, false>, dim3(grid), dim3(kRouteWarps * 32), 0, s,
-                          logits, T, E, k, renormalize, idx, w, RouteEx{});
-    return launch_pdl(k_route_topk<NPL, true>, dim3(grid), dim3(kRouteWarps * 32), 0, s, logits,
-                      T, E, k, renormalize, idx, w, *ex);
+    if (NPL >= 4 && k == 8)
+        return launch_kt<NPL, (NPL >= 4 ? 8 : 0)>(logits, T, E, k, renormalize, idx, w, ex, s);
+    return launch_kt<NPL, 0>(logits, T, E, k, renormalize, idx, w, ex, s);
 }
 
 }  // namespace

@@ -134,11 +134,11 @@ size_t moe_layout_workspace_bytes(int T, int k, int E, int R);
 
 /*
  * How many kernels moe_dispatch_layout (and moe_dispatch_layout_private)
- * launch for (T, k, E, R) on the current device: 1 when every logical rank
- * fits one chunk of at most 2048 slots (T/R * k <= 2048; the decode sizes)
- * and the device can schedule the single-launch form (one thread-block
- * cluster of at most 8 CTAs), else 2 (a per-chunk histogram, then the
- * placement).  0 on invalid sizes.  Both forms give identical outputs; the
+ * launch for (T, k, E, R) on the current device: 1 for small layouts, when
+ * every logical rank fits one chunk of at most 2048 slots, the slots come to
+ * at most one per thread of an 8-CTA cluster of 1024 threads each (T*k <=
+ * 8192) and the device can schedule that cluster; else 2 (a per-chunk
+ * histogram, then the placement).  0 on invalid sizes.  Both forms give identical outputs; the
  * count serves callers that account for launches (graph sizing, profiling).
  */
 int moe_dispatch_layout_launches(int T, int k, int E, int R);

@@ -91,9 +91,10 @@ def _full_path_vs_oracle(moe, logits, x, E, k, R, cap=0, fp8=True, idx_override=
     (1200, 24, 6, 3, 512, 120),      # padded with drops
     (96, 16, 4, 2, 16384, 0),        # wide rows: several passes per CTA in every kernel
     (64, 32, 8, 4, 12416, 0),        # wide and not a multiple of the CTA's span
-    (1024, 1024, 32, 64, 128, 0),    # single-launch layout: 8 ranks per CTA, E and k at maximum
+    (512, 1024, 16, 64, 128, 0),     # single-launch layout: 8 ranks per CTA, E at maximum
     (2048, 64, 4, 16, 128, 100),     # single-launch layout, padded with drops
-    (6144, 384, 8, 48, 128, 0),      # single-launch layout: 6 ranks per CTA, 5 warps each
+    (960, 96, 8, 24, 128, 0),        # single-launch layout: 3 ranks per CTA, 10 warps each
+    (1024, 64, 8, 8, 128, 0),        # single-launch layout: one 1024-slot rank per CTA
 ])
 def test_random_shapes_all_stages(moe, T, E, k, R, H, cap):
     logits, x = inputs.make_random_case(T, H, E, k, seed=T + E + k + H)
@@ -290,12 +291,15 @@ def test_layout_large_token_count_many_chunks(moe):
 
 
 def test_layout_launch_count(moe):
-    """Decode sizes (one chunk of at most 2048 slots per rank) take the
-    single-launch cluster layout; prefill (16 chunks per rank) the
+    """Small layouts (T * k <= 8192, one chunk per rank) take the
+    single-launch cluster layout; the decode and prefill workloads the
     histogram + placement pair."""
-    assert moe.moe_dispatch_layout_launches(4096, 8, 256, 32) == 1      # dsv3
-    assert moe.moe_dispatch_layout_launches(6144, 8, 384, 48) == 1      # kimi
-    assert moe.moe_dispatch_layout_launches(4096, 9, 288, 32) == 1      # dsv3 + shared expert
+    assert moe.moe_dispatch_layout_launches(512, 2, 8, 8) == 1          # mixtral
+    assert moe.moe_dispatch_layout_launches(64, 2, 8, 2) == 1           # tiny
+    assert moe.moe_dispatch_layout_launches(1024, 8, 64, 8) == 1        # 8192 slots
+    assert moe.moe_dispatch_layout_launches(1032, 8, 64, 8) == 2        # 8256 slots
+    assert moe.moe_dispatch_layout_launches(4096, 8, 256, 32) == 2      # dsv3
+    assert moe.moe_dispatch_layout_launches(6144, 8, 384, 48) == 2      # kimi
     assert moe.moe_dispatch_layout_launches(32768, 8, 256, 8) == 2      # prefill
     assert moe.moe_dispatch_layout_launches(4096, 8, 256, 3) == 0       # R does not divide E
 
