@@ -64,7 +64,6 @@ L2_FLUSH_BYTES = 512 << 20
 STEPS_PER_GRAPH = 10           # consecutive steps captured in one CUDA graph (no-flush workloads)
 DEFAULT_CONFIGS = "dsv3,kimi,prefill"
 REGION_TARGET_S = 1.0          # timed work per workload for the step (repeated K-step regions)
-DC_TARGET_S = 0.5              # the same for the dispatch+combine graphs
 MIN_REPS, MAX_REPS = 5, 4000
 DTYPES = {"route": "f32 logits -> f32 weights, int32 ids",
           "layout": "int32",
@@ -634,9 +633,10 @@ def measure(cfg: inputs.Config, args, dev, world: int, local: int) -> dict:
         s.synchronize()
     sampler = ClockSampler(local)
     sampler.start()
-    local_step, step_min, step_max, reps = repeated_regions(g_stepG, g_step1, REGION_TARGET_S,
+    local_step, step_min, step_max, reps = repeated_regions(g_stepG, g_step1, args.region_seconds,
                                                             sampler)
-    local_dc, dc_min, dc_max, dc_reps = repeated_regions(g_dcG, g_dc1, DC_TARGET_S, sampler)
+    local_dc, dc_min, dc_max, dc_reps = repeated_regions(g_dcG, g_dc1, args.region_seconds / 2,
+                                                         sampler)
     clocks = sampler.stop()
 
     # per-stage breakdown: G consecutive steps captured with timing events
@@ -923,11 +923,16 @@ def main(argv=None):
                     help="route + layout + dispatch as one cooperative launch, then combine")
     ap.add_argument("--combine-fp8", action="store_true",
                     help="expert rows come back as E4M3 + 1x128 scales (moe_combine_fp8)")
+    ap.add_argument("--region-seconds", type=float, default=REGION_TARGET_S,
+                    help="timed work per workload: the K-step region repeats (at least 5 times) "
+                         "until about this many seconds (dispatch+combine: half of it)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     if args.steps < 1:
         ap.error("--steps must be at least 1")
+    if args.region_seconds < 0:
+        ap.error("--region-seconds must be >= 0")
     config_names(args.config)
     if args.impl == "reference":
         run_reference(args)

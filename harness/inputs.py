@@ -20,6 +20,10 @@ kimi        128   48   7168   384  8  fp8       packed   dequantise
 prefill     4096  8    7168   256  8  fp8       padded   dequantise
 ==========  ====  ===  =====  ===  =  ========  =======  ===============
 
+Two more: dsv3_shared (dsv3 with one shared expert routed as a ninth slot,
+seed 1005) and prefill_r2 (prefill on 2 of its logical ranks, seed 1006, for
+profiler captures that must stay small).
+
 Recipe: config i (0..4 in the order above) uses seed_i = 1000 + i and three
 independent CPU generators seeded seed_i*10 + s: s = 0 router logits
 N(0, 1) fp32 [T][E]; s = 1 hidden states N(0, 1) drawn in fp32 and rounded
@@ -92,6 +96,10 @@ CONFIGS = {
         # beyond the five: DeepSeek-V3-like decode where the shared expert is
         # routed too (9 experts per token, 8 routed + 1 shared per rank)
         Config("dsv3_shared", 5, 128, 32, 7168, 256, 8, "fp8", "packed", "dequant", n_shared=1),
+        # the prefill workload on 2 of its 8 logical ranks (same per-rank
+        # shape, a quarter of the tokens): small enough for full per-kernel
+        # profiler captures (about 2 GB on the device), still larger than L2
+        Config("prefill_r2", 6, 4096, 2, 7168, 256, 8, "fp8", "padded", "dequant"),
     ]
 }
 
