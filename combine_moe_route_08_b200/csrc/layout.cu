@@ -37,11 +37,10 @@
 // Small layouts (one chunk per logical rank and at most one slot per thread
 // of an 8-CTA cluster: T*k <= 8192, e.g. the Mixtral-like workload) take a
 // single launch instead: k_layout_cluster, one thread-block cluster of at
-// most 8 CTAs.  Each CTA owns a run of whole ranks,
-// counts them per warp, and publishes its per-expert totals in its own shared
-// memory; one cluster barrier later every CTA reads the others' totals over
-// distributed shared memory, scans, and ranks its slots exactly as
-// k_layout_assign does.  The grid-wide ordering is then the hardware cluster
+// most 8 CTAs.  Each CTA owns a run of whole ranks, counts them per warp, and
+// publishes its per-expert totals in its own shared memory; one cluster
+// barrier later every CTA reads the others' totals over distributed shared
+// memory, scans, and ranks its slots exactly as k_layout_assign does.  The grid-wide ordering is then the hardware cluster
 // barrier (all CTAs of a cluster are co-scheduled), not a kernel boundary
 // plus a global round trip through the workspace.  Larger layouts keep the
 // pair: with 4096 slots per SM (T = 4096, k = 8) the single cluster measured
@@ -140,7 +139,7 @@ __global__ void __launch_bounds__(kHistThreads)
 #pragma unroll
     for (int s = 0; s < kHistSlots; ++s) {
         const bool valid = static_cast<unsigned>(e[s]) < static_cast<unsigned>(E);
-        bad |= !valid && e[s] != -1;  // -1 past the chunk's end too
+        bad |= !valid && e[s] != -1;  // -1: an empty slot, or past the chunk's end
         if (valid)  // counts are order-free: one shared-memory atomic per slot
             atomicAdd(&h[e[s]], 1);
     }
@@ -351,7 +350,7 @@ __global__ void __launch_bounds__(kThreads)
 }
 
 // ---------------------------------------------------------------------------
-// Single-launch layout for one chunk per rank (decode sizes): one cluster.
+// Single-launch layout for small layouts (one chunk per rank): one cluster.
 
 constexpr int kClusterMax = 8;        // CTAs of the cluster (portable cluster size)
 constexpr int kClusterSteps = 2;      // 32-slot steps per warp, at most

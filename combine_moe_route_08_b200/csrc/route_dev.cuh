@@ -9,11 +9,11 @@
 //
 // Each lane holds the logits e = i*32 + lane (a warp-wide load per i is one
 // coalesced 128-byte line), as order-preserving 32-bit keys, and tracks its
-// own best key.  k rounds of warp arg-max under the order (logit descending,
-// index ascending) pick the experts: one warp-wide max of the lanes' best
-// keys and one warp-wide min of the expert ids holding it (redux.sync, a
-// single instruction each); only the winning lane then clears that key and
-// rescans for its next best.
+// own best and second-best key.  k rounds of warp arg-max under the order
+// (logit descending, index ascending) pick the experts: one warp-wide max of
+// the lanes' best keys and one warp-wide min of the expert ids holding it
+// (redux.sync, a single instruction each); the winning lane promotes its
+// second best, and rescans only when it has none left.
 //
 // The softmax is evaluated with its error bounded (u = 2^-24):
 //   d = l - m is split exactly into d_hi + d_lo (Knuth's TwoSum), so the
