@@ -218,3 +218,15 @@ def test_combine_fp8_rejects_bad_arguments(moe):
     assert f(A16 + 4, A4, A4, A4, 4, 128, 2, 8, A16, None, None) == moe.MOE_ERR_INVALID_ARG
     assert f(A16, None, A4, A4, 4, 128, 2, 8, A16, None, None) == moe.MOE_ERR_INVALID_ARG
     assert f(None, None, None, None, 0, 128, 2, 0, None, None, None) == moe.MOE_OK  # T = 0
+
+
+def test_layout_launch_count_on_the_host(moe):
+    """The launch count is a host query: 0 for invalid sizes, 2 (histogram +
+    placement) for layouts beyond the single-launch limit, 1 or 2 for small
+    ones (1 only where a device can schedule the cluster)."""
+    assert moe.moe_dispatch_layout_launches(64, 2, 8, 3) == 0          # R does not divide E
+    assert moe.moe_dispatch_layout_launches(-1, 2, 8, 2) == 0
+    assert moe.moe_dispatch_layout_launches(4096, 8, 256, 32) == 2     # 32768 slots
+    assert moe.moe_dispatch_layout_launches(32768, 8, 256, 8) == 2     # 16 chunks per rank
+    assert moe.moe_dispatch_layout_launches(64, 2, 8, 2) in (1, 2)
+    assert moe.kernels_per_step(4096, 8, 256, 32) == 5
