@@ -270,13 +270,13 @@ namespace {
 template <int KREG>
 int fp8_grid(int threads)
 {
-    constexpr int kMaxDev = 64;
+    constexpr int kMaxDev = 64;  // devices whose answer is remembered; others ask each time
     static std::atomic<int> cache[kMaxDev][kFp8Threads / 32 + 1];
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev)
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0)
         return 0;
-    std::atomic<int> &slot = cache[dev][threads / 32];
-    int v = slot.load(std::memory_order_relaxed);
+    std::atomic<int> *slot = (dev < kMaxDev) ? &cache[dev][threads / 32] : nullptr;
+    int v = slot ? slot->load(std::memory_order_relaxed) : 0;
     if (v > 0)
         return v;
     int nsm = 0, per = 0;
@@ -287,7 +287,8 @@ int fp8_grid(int threads)
         return 0;
     }
     v = std::max(1, nsm * per);
-    slot.store(v, std::memory_order_relaxed);
+    if (slot)
+        slot->store(v, std::memory_order_relaxed);
     return v;
 }
 

@@ -70,6 +70,11 @@ constexpr int kWarps = kThreads / 32;
 // have one chunk per rank either way.
 constexpr int kMaxSteps = 2;
 constexpr int kChunkSlots = kThreads * kMaxSteps;  // 2048
+// The placement kernel: kAssignThreads threads per chunk, each warp owning a
+// run of at most kAssignSteps 32-slot steps.
+constexpr int kAssignThreads = 1024;
+constexpr int kAssignWarps = kAssignThreads / 32;
+constexpr int kAssignSteps = kChunkSlots / kAssignThreads;
 constexpr int kColBatch = 16;                      // 4-byte histogram loads in flight per thread
 constexpr int kColBatch4 = 6;                      // 16-byte histogram loads in flight per thread
 
@@ -88,7 +93,7 @@ __device__ __forceinline__ void warp_run(const LayoutGeom &G, int c, int64_t &w0
     int t0, t1;
     chunk_tokens(G, c, t0, t1);
     const int64_t i0 = static_cast<int64_t>(t0) * G.k, i1 = static_cast<int64_t>(t1) * G.k;
-    const int64_t seg = static_cast<int64_t>(ceil_div(static_cast<int>(i1 - i0), kWarps * 32)) * 32;
+    const int64_t seg = static_cast<int64_t>(ceil_div(static_cast<int>(i1 - i0), kAssignWarps * 32)) * 32;
     const int w = threadIdx.x >> 5;
     w0 = min(i0 + w * seg, i1);
     w1 = min(w0 + seg, i1);
@@ -96,11 +101,11 @@ __device__ __forceinline__ void warp_run(const LayoutGeom &G, int c, int64_t &w0
 
 // The lane's slots of its warp run, loaded in one go (-1 past the end).
 __device__ __forceinline__ void load_run(const int32_t *__restrict__ topk_idx, int64_t w0,
-                                         int64_t w1, int (&e)[kMaxSteps])
+                                         int64_t w1, int (&e)[kAssignSteps])
 {
     const int lane = threadIdx.x & 31;
 #pragma unroll
-    for (int s = 0; s < kMaxSteps; ++s) {
+    for (int s = 0; s < kAssignSteps; ++s) {
         const int64_t i = w0 + 32 * s + lane;
         e[s] = (i < w1) ? __ldg(topk_idx + i) : -1;
     }
@@ -204,17 +209,17 @@ __device__ __forceinline__ void column_sums(const int32_t *__restrict__ ws_hist,
 }
 
 // Shares per histogram column: as many as the threads allow, at most
-// kWarps / 4 (kColBatch4 or kColBatch rows in flight per thread).
+// kAssignWarps / 4 (kColBatch4 or kColBatch rows in flight per thread).
 __host__ __device__ inline int column_shares(int E)
 {
     const int per_share = (E % 4 == 0) ? E / 4 : E;
-    const int p = kThreads / per_share;
-    return p < 1 ? 1 : (p > kWarps / 4 ? kWarps / 4 : p);
+    const int p = kAssignThreads / per_share;
+    return p < 1 ? 1 : (p > kAssignWarps / 4 ? kAssignWarps / 4 : p);
 }
 
-// Shared memory: wh[kWarps][E] per-warp counts, then bases; parts[4P][E]
-// column-sum shares; off[E + 1]; chb[E]; rbs[E]; tot[kWarps + 1].
-__global__ void __launch_bounds__(kThreads)
+// Shared memory: wh[kAssignWarps][E] per-warp counts, then bases; parts[4P][E]
+// column-sum shares; off[E + 1]; chb[E]; rbs[E]; tot[kAssignWarps + 1].
+__global__ void __launch_bounds__(kAssignThreads)
     k_layout_assign(const int32_t *__restrict__ topk_idx, LayoutGeom G, int capacity, int64_t rows,
                     const int32_t *__restrict__ ws_hist, int32_t *__restrict__ expert_counts,
                     int32_t *__restrict__ expert_src_counts, int32_t *__restrict__ rank_counts,
@@ -226,21 +231,21 @@ __global__ void __launch_bounds__(kThreads)
     const int E = G.E, lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     const int nb = key_bits(E);
     const int P = column_shares(E);
-    int32_t *wh = sm;                   // [kWarps][E] per-warp counts, then bases
-    int32_t *parts = wh + kWarps * E;   // [4P][E] column-sum shares
+    int32_t *wh = sm;                   // [kAssignWarps][E] per-warp counts, then bases
+    int32_t *parts = wh + kAssignWarps * E;   // [4P][E] column-sum shares
     int32_t *off = parts + 4 * P * E;   // [E + 1] expert totals, then their scan
     int32_t *chb = off + E + 1;         // [E] slots of e in earlier chunks
     int32_t *rbs = chb + E;             // [E] slots of e in chunks of earlier ranks
-    int32_t *tot = rbs + E;             // [kWarps + 1]
+    int32_t *tot = rbs + E;             // [kAssignWarps + 1]
     const int c = blockIdx.x;
 
     int64_t w0, w1;
     warp_run(G, c, w0, w1);
-    for (int x = threadIdx.x; x < kWarps * E; x += kThreads)
+    for (int x = threadIdx.x; x < kAssignWarps * E; x += kAssignThreads)
         wh[x] = 0;  // before the wait: nothing upstream is read
     pdl_trigger();  // the next kernel may take idle SM slots now; it waits for this one
     pdl_wait();
-    int e[kMaxSteps];
+    int e[kAssignSteps];
     load_run(topk_idx, w0, w1, e);  // in flight while the columns are summed
 
     // histogram columns: base of this chunk inside each expert (earlier
@@ -256,7 +261,7 @@ __global__ void __launch_bounds__(kThreads)
     __syncthreads();  // wh zeroed by every thread before any warp counts into it
     // per-warp counts of this CTA's slots (order-free: shared-memory atomics)
     warp_count(e, w0, w1, E, wh + w * E);
-    for (int x = threadIdx.x; x < E; x += kThreads) {
+    for (int x = threadIdx.x; x < E; x += kAssignThreads) {
         int before = 0, total = 0, mine = 0, rstart = 0;
         for (int part = 0; part < P; ++part) {
             before += parts[(4 * part) * E + x];
@@ -273,23 +278,23 @@ __global__ void __launch_bounds__(kThreads)
             expert_src_counts[static_cast<size_t>(x) * G.R + r] = mine;
     }
     __syncthreads();
-    block_exclusive_scan<kWarps>(off, E, tot);  // off[e] = slots of experts < e; off[E] = total
+    block_exclusive_scan<kAssignWarps>(off, E, tot);  // off[e] = slots of experts < e; off[E] = total
     if (c == 0) {
-        for (int x = threadIdx.x; x <= E; x += kThreads)
+        for (int x = threadIdx.x; x <= E; x += kAssignThreads)
             expert_offsets[x] = (capacity == 0) ? off[x] : x * capacity;
         const int L = E / G.R;
-        for (int rr = threadIdx.x; rr < G.R; rr += kThreads)
+        for (int rr = threadIdx.x; rr < G.R; rr += kAssignThreads)
             rank_counts[rr] = off[(rr + 1) * L] - off[rr * L];
     }
     // per-warp base of each expert's positions: earlier chunks + earlier warps
-    warp_bases_par<kWarps>(wh, chb, E);
+    warp_bases_par<kAssignWarps>(wh, chb, E);
     __syncthreads();
     int32_t *mywh = wh + w * E;
 
     // rank every slot among equal experts, in slot order
     bool dropped = false, bad_row = false;
 #pragma unroll
-    for (int s = 0; s < kMaxSteps; ++s) {
+    for (int s = 0; s < kAssignSteps; ++s) {
         if (w0 + 32 * s >= w1)
             break;
         const int64_t i = w0 + 32 * s + lane;
@@ -333,15 +338,15 @@ __global__ void __launch_bounds__(kThreads)
         report(dev_status, MOE_ERR_INVALID_ARG);
 
     // rows that no slot fills -> -1
-    const int64_t stride = static_cast<int64_t>(gridDim.x) * kThreads;
-    const int64_t first = static_cast<int64_t>(c) * kThreads + threadIdx.x;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * kAssignThreads;
+    const int64_t first = static_cast<int64_t>(c) * kAssignThreads + threadIdx.x;
     if (capacity == 0) {
         for (int64_t r = off[E] + first; r < rows; r += stride)
             recv_src[r] = -1;
     } else {
         for (int x = c; x < E; x += gridDim.x) {
             const int filled = min(off[x + 1] - off[x], capacity);
-            for (int p = filled + threadIdx.x; p < capacity; p += kThreads)
+            for (int p = filled + threadIdx.x; p < capacity; p += kAssignThreads)
                 recv_src[static_cast<int64_t>(x) * capacity + p] = -1;
         }
         for (int64_t r = static_cast<int64_t>(E) * capacity + first; r < rows; r += stride)
@@ -544,7 +549,8 @@ __global__ void __launch_bounds__(kThreads)
 
 size_t assign_smem_bytes(int E)
 {
-    return (static_cast<size_t>(kWarps + 4 * column_shares(E) + 3) * E + 1 + kWarps + 1) * sizeof(int32_t);
+    return (static_cast<size_t>(kAssignWarps + 4 * column_shares(E) + 3) * E + 1 + kAssignWarps + 1) *
+           sizeof(int32_t);
 }
 
 }  // namespace
@@ -707,7 +713,7 @@ cudaError_t dispatch_layout(const int32_t *topk_idx, const LayoutGeom &g, int ca
         if (err != cudaSuccess)
             return err;
     }
-    return launch_pdl(k_layout_assign, dim3(g.nchunks), dim3(kThreads), smem, s, topk_idx, g, capacity,
+    return launch_pdl(k_layout_assign, dim3(g.nchunks), dim3(kAssignThreads), smem, s, topk_idx, g, capacity,
                       rows, hist, expert_counts, expert_src_counts, rank_counts, expert_offsets,
                       dispatch_pos, recv_src, private_pos, dev_status);
 }
