@@ -1,6 +1,7 @@
 """Host-side pieces of bench.py, on the CPU: the algorithmic byte counts, the
 max-over-ranks reduction with two gloo ranks, and the reference arm's
 rank-0-only output under a two-rank launch."""
+import argparse
 import json
 import os
 import socket
@@ -77,3 +78,34 @@ def test_reference_arm_prints_one_line_from_rank0(world, tmp_path):
     assert line["impl"] == "reference" and line["unit"] == "GB/s" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle"
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_default_workloads_and_headline():
+    """The default run measures the decode and prefill targets; the largest
+    workload (prefill) carries the headline; unknown names are refused."""
+    names = bench.config_names(bench.DEFAULT_CONFIGS)
+    assert names == ["dsv3", "kimi", "prefill"]
+    assert bench.headline_name(names) == "prefill"
+    assert bench.headline_name(["tiny", "mixtral"]) == "mixtral"
+    assert bench.config_names("dsv3, dsv3,kimi") == ["dsv3", "kimi"]
+    with pytest.raises(SystemExit):
+        bench.config_names("dsv3,nope")
+
+
+def test_both_arms_print_the_same_config():
+    """The reference arm and ours build `config` from the same function, so
+    the driver can match the two lines."""
+    args = argparse.Namespace(fused=False, two_phase=False, combine_fp8=False)
+    a = bench.line_config(args, ["dsv3", "kimi", "prefill"], 1)
+    b = bench.line_config(args, bench.config_names(bench.DEFAULT_CONFIGS), 1)
+    assert a == b
+    assert a["workload"].startswith("prefill:") and set(a["workloads"]) == {"dsv3", "kimi", "prefill"}
+
+
+def test_repeated_region_count():
+    """About target seconds of K-step regions, never fewer than the minimum
+    nor more than the maximum."""
+    assert bench.repetitions(0.003, 1.0) == 334
+    assert bench.repetitions(0.5, 1.0) == bench.MIN_REPS
+    assert bench.repetitions(1e-7, 1.0) == bench.MAX_REPS
+    assert bench.repetitions(0.0, 1.0) == bench.MIN_REPS
