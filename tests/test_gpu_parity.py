@@ -536,12 +536,14 @@ def test_combine_bf16_k_sweep(moe, k, T, H):
                                    (11, 37, 128), (16, 37, 128), (17, 37, 128),
                                    (32, 37, 128), (8, 4099, 128), (2, 9001, 128), (9, 2100, 1024),
                                    (1, 37, 512), (8, 300, 512), (11, 37, 512), (32, 37, 512),
-                                   (8, 4099, 1024)])
+                                   (8, 4099, 1024), (8, 37, 640), (8, 37, 7680), (8, 37, 2560)])
 @pytest.mark.parametrize("scale_offset", [0, 1])
 def test_combine_fp8_edges(moe, k, T, H, scale_offset):
     """k beyond the register-held rows, -1 slots, ragged token counts (several
     tokens per CTA with a short last CTA), several hidden sizes, and a scale
-    plane that is only 4-byte aligned."""
+    plane that is only 4-byte aligned.  k = 8 runs the guard-free one-pass
+    form when H / 16 is a multiple of 32 up to 448 (H = 512, 1024, 2560,
+    7168) and the general form otherwise (H = 128, 640, 7680)."""
     rng = np.random.default_rng(40 + k + T + H + scale_offset)
     rows = 200
     q, s, _ = _fp8_payload(H, 64, seed=50 + k + H, bank=64)
