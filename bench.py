@@ -728,54 +728,140 @@ def measure(cfg: inputs.Config, args, dev, world: int, local: int) -> dict:
     del g_step1, g_stepG, g_dc1, g_dcG
 
     # ---- end to end through the public API, host buffers in and out ----
-    # Every step copies its inputs (logits, x) in from pinned host memory and
-    # its output out to pinned host memory, inside the timed region.  The
-    # copies run on their own streams (H2D and D2H have separate copy
-    # engines): step i+1's inputs arrive while step i computes and step
-    # i-1's output leaves, as a serving loop would overlap them.  Inputs and
-    # output are double-buffered; the step's intermediates are reused.
+    # Every step copies its inputs (logits, x) in from page-locked host memory
+    # and its result out to page-locked host memory, inside the timed region.
+    # Direct and fused pipelines go through the library's host-buffer entry
+    # points (moe_route_dispatch_*_host, moe_combine_*_host), which enqueue
+    # the copies and the kernels on one stream; consecutive steps alternate
+    # between two streams with a device buffer set each, so one step's
+    # copies overlap the other's kernels and copies in the other direction.
+    # The two-phase and shared-expert pipelines have no host-buffer entry
+    # point: their steps are the device-pointer calls between torch copies on
+    # two copy streams, double-buffered the same way.
     logits_pin = logits_h.pin_memory()
     x_pin = x_h.pin_memory()
     out_pins = [torch.empty(T, H, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
-    logits2, x2, out2 = torch.empty_like(logits), torch.empty_like(x), torch.empty_like(out)
-    swap = {logits.data_ptr(): logits2.data_ptr(), x.data_ptr(): x2.data_ptr(),
-            out.data_ptr(): out2.data_ptr()}
-    calls2 = [(fn, tuple(swap.get(v, v) if isinstance(v, int) else v for v in a))
-              for fn, a in calls]
-    sets = [(logits, x, out, calls), (logits2, x2, out2, calls2)]
-    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-    ev_in = [torch.cuda.Event() for _ in range(2)]
-    ev_done = [torch.cuda.Event() for _ in range(2)]
-    ev_out = [torch.cuda.Event() for _ in range(2)]
     n_e2e = min(K, 100)
     first, last = max(W, 3), max(W, 3) + n_e2e
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize(dev)
-    for i in range(last):
-        lg, xx, oo, cl = sets[i % 2]
-        with torch.cuda.stream(s_in):
-            if i >= 2:
-                s_in.wait_event(ev_done[i % 2])   # step i-2 has finished reading this set
+    host_api = not args.two_phase and not cfg.n_shared
+    if host_api:
+        e2e_how = ("host-buffer C ABI entry points per step (moe_route_dispatch_"
+                   f"{'fp8' if cfg.dispatch == 'fp8' else 'bf16'}_host"
+                   f"{' with MOE_HOST_FUSED' if args.fused else ''}, moe_combine_"
+                   f"{'fp8' if args.combine_fp8 else 'bf16'}_host): every step's inputs copied "
+                   "in from page-locked host memory and its result copied out, inside the "
+                   "timed region; steps alternate between two streams and two device buffer "
+                   "sets; no L2 flush")
+        streams = [torch.cuda.Stream(dev) for _ in range(2)]
+        step_calls = []
+        for q in range(2):
+            with torch.cuda.stream(streams[q]):
+                b = dict(logits=torch.empty_like(logits), x=torch.empty_like(x),
+                         topk_idx=torch.empty_like(idx), topk_w=torch.empty_like(w),
+                         out=torch.empty_like(out))
+                for key in ("expert_counts", "expert_src_counts", "rank_counts",
+                            "expert_offsets", "dispatch_pos", "recv_src"):
+                    b[key] = torch.empty_like(lay[key])
+                if cfg.dispatch == "fp8":
+                    b["recv_q"], b["recv_scale"] = torch.empty_like(recv_q), torch.empty_like(recv_scale)
+                else:
+                    b["recv_x"] = torch.empty_like(recv_x)
+                nbytes = (moe.moe_route_dispatch_workspace_bytes(T, k, E_lay, R) if args.fused
+                          else moe.moe_layout_workspace_bytes(T, k, E_lay, R))
+                b["ws"] = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=dev)
+                b["status"] = torch.zeros(1, dtype=torch.int32, device=dev)
+            sq = streams[q].cuda_stream
+            stp = b["status"].data_ptr()
+            head = (logits_pin.data_ptr(), x_pin.data_ptr(), T, E, k, 0, R, cap, H,
+                    moe.MOE_HOST_FUSED if args.fused else 0,
+                    *[b[key].data_ptr() for key in ("logits", "x", "topk_idx", "topk_w",
+                                                    "expert_counts", "expert_src_counts",
+                                                    "rank_counts", "expert_offsets",
+                                                    "dispatch_pos", "recv_src")])
+            tail = (rows, b["ws"].data_ptr(), b["ws"].numel(), stp, sq)
+            if cfg.dispatch == "fp8":
+                rd = (lib.moe_route_dispatch_fp8_host,
+                      head + (b["recv_q"].data_ptr(), b["recv_scale"].data_ptr()) + tail)
+            else:
+                rd = (lib.moe_route_dispatch_bf16_host, head + (b["recv_x"].data_ptr(),) + tail)
+            pw = (b["dispatch_pos"].data_ptr(), b["topk_w"].data_ptr(), T, H, k, rows,
+                  b["out"].data_ptr(), out_pins[q].data_ptr(), stp, sq)
+            cb = ((lib.moe_combine_fp8_host, (b["recv_q"].data_ptr(), b["recv_scale"].data_ptr())
+                   + pw) if args.combine_fp8 else (lib.moe_combine_bf16_host, (y.data_ptr(),) + pw))
+            step_calls.append(([rd, cb], b))
+        ev_start = torch.cuda.Event()
+        ev_end = [torch.cuda.Event() for _ in range(2)]
+        torch.cuda.synchronize(dev)
+        for i in range(last):
+            q = i % 2
             if i == first:
-                t0.record(s_in)
-            lg.copy_(logits_pin, non_blocking=True)
-            xx.copy_(x_pin, non_blocking=True)
-            ev_in[i % 2].record(s_in)
-        s.wait_event(ev_in[i % 2])
-        if i >= 2:
-            s.wait_event(ev_out[i % 2])           # step i-2's output has left this buffer
-        for fn, a in cl:
-            rc = fn(*a)
-            if rc != 0:
-                raise moe.MoeError(rc, fn.__name__)
-        ev_done[i % 2].record(s)
-        with torch.cuda.stream(s_out):
-            s_out.wait_event(ev_done[i % 2])
-            out_pins[i % 2].copy_(oo, non_blocking=True)
-            ev_out[i % 2].record(s_out)
-            if i == last - 1:
-                t1.record(s_out)
-    torch.cuda.synchronize(dev)
+                torch.cuda.synchronize(dev)      # warm-up steps done on both streams
+                t0.record(streams[0])
+                ev_start.record(streams[0])
+                streams[1].wait_event(ev_start)
+            for fn, a in step_calls[q][0]:
+                rc = fn(*a)
+                if rc != 0:
+                    raise moe.MoeError(rc, fn.__name__)
+        for q in range(2):
+            ev_end[q].record(streams[q])
+            streams[0].wait_event(ev_end[q])
+        t1.record(streams[0])
+        torch.cuda.synchronize(dev)
+        # no kernel reported an error (a capacity drop, a wait that gave up), and
+        # the last step's result reached the host: the bits of the device buffer
+        for _, b in step_calls:
+            if int(b["status"].item()) not in (moe.MOE_OK, moe.MOE_ERR_CAPACITY):
+                raise moe.MoeError(int(b["status"].item()), "host-buffer step")
+        last_set = step_calls[(last - 1) % 2][1]
+        if not torch.equal(out_pins[(last - 1) % 2].view(torch.int16),
+                           last_set["out"].cpu().view(torch.int16)):
+            raise RuntimeError("host result differs from the device buffer it was copied from")
+        del step_calls, last_set, b
+    else:
+        e2e_how = ("device-pointer C ABI calls per step between torch copies: every step's "
+                   "inputs copied in from page-locked host memory and its output copied out, on "
+                   "two copy streams overlapping the neighbouring steps' compute; inputs and "
+                   "output double-buffered; no L2 flush (this pipeline has no host-buffer "
+                   "entry point)")
+        logits2, x2, out2 = torch.empty_like(logits), torch.empty_like(x), torch.empty_like(out)
+        swap = {logits.data_ptr(): logits2.data_ptr(), x.data_ptr(): x2.data_ptr(),
+                out.data_ptr(): out2.data_ptr()}
+        calls2 = [(fn, tuple(swap.get(v, v) if isinstance(v, int) else v for v in a))
+                  for fn, a in calls]
+        sets = [(logits, x, out, calls), (logits2, x2, out2, calls2)]
+        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_done = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
+        torch.cuda.synchronize(dev)
+        for i in range(last):
+            lg, xx, oo, cl = sets[i % 2]
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(ev_done[i % 2])   # step i-2 has finished reading this set
+                if i == first:
+                    t0.record(s_in)
+                lg.copy_(logits_pin, non_blocking=True)
+                xx.copy_(x_pin, non_blocking=True)
+                ev_in[i % 2].record(s_in)
+            s.wait_event(ev_in[i % 2])
+            if i >= 2:
+                s.wait_event(ev_out[i % 2])           # step i-2's output has left this buffer
+            for fn, a in cl:
+                rc = fn(*a)
+                if rc != 0:
+                    raise moe.MoeError(rc, fn.__name__)
+            ev_done[i % 2].record(s)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_done[i % 2])
+                out_pins[i % 2].copy_(oo, non_blocking=True)
+                ev_out[i % 2].record(s_out)
+                if i == last - 1:
+                    t1.record(s_out)
+        torch.cuda.synchronize(dev)
+        del calls2, sets
     e2e_ms = max_over_ranks([t0.elapsed_time(t1) / n_e2e], world, dev)[0]
     h2d = logits_h.numel() * 4 + x_h.numel() * 2
     d2h = out.numel() * 2
@@ -828,10 +914,7 @@ def measure(cfg: inputs.Config, args, dev, world: int, local: int) -> dict:
                             "CUDA-event time inside the step graph"},
         "e2e": {"value": n_gpus * nb["step"] / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
                 "us_per_step": e2e_ms * 1e3, "h2d_bytes_per_step": h2d,
-                "how": ("C ABI calls launched per step; every step's inputs copied in from "
-                        "pinned host memory and its output copied out, on two copy "
-                        "streams overlapping the neighbouring steps' compute; inputs and "
-                        "output double-buffered; no L2 flush"),
+                "how": e2e_how,
                 "d2h_bytes_per_step": d2h},
         "kernels_per_step": kernels_per_step,
         "clocks": clocks,
@@ -840,7 +923,7 @@ def measure(cfg: inputs.Config, args, dev, world: int, local: int) -> dict:
     if sm:
         res["clocks"]["us_x_mhz"] = ms_step * 1e3 * sm
         res["clocks"]["dispatch_combine_us_x_mhz"] = ms_dc * 1e3 * sm
-    del calls, calls2, sets
+    del calls
     return res
 
 

@@ -24,7 +24,9 @@ __all__ = [
     "LIB_PATH", "MOE_SCALE_ROW_MAJOR", "MOE_SCALE_COL_MAJOR", "moe_dispatch_layout_private",
     "moe_compact_fp8", "moe_compact_bf16", "moe_route_dispatch_workspace_bytes",
     "moe_route_dispatch_fp8", "moe_route_dispatch_bf16", "moe_route_dispatch_ex_fp8",
-    "moe_route_dispatch_ex_bf16", "moe_combine_fp8",
+    "moe_route_dispatch_ex_bf16", "moe_combine_fp8", "MOE_HOST_FUSED",
+    "moe_route_dispatch_fp8_host", "moe_route_dispatch_bf16_host", "moe_combine_bf16_host",
+    "moe_combine_fp8_host",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_route.so")
@@ -92,6 +94,15 @@ lib.moe_combine_fp8.argtypes = [_P, _P, _P, _P, _i32, _i32, _i32, _i64, _P, _P, 
 lib.moe_combine_fp8.restype = _i32
 lib.moe_quantize_e4m3.argtypes = [_P, _i64, _P, _P]
 lib.moe_quantize_e4m3.restype = _i32
+_HOST_HEAD = [_P, _P] + [_i32] * 8 + [_P] * 10       # host inputs .. recv_src
+lib.moe_route_dispatch_fp8_host.argtypes = _HOST_HEAD + [_P, _P, _i64, _P, _sz, _P, _P]
+lib.moe_route_dispatch_fp8_host.restype = _i32
+lib.moe_route_dispatch_bf16_host.argtypes = _HOST_HEAD + [_P, _i64, _P, _sz, _P, _P]
+lib.moe_route_dispatch_bf16_host.restype = _i32
+lib.moe_combine_bf16_host.argtypes = [_P, _P, _P, _i32, _i32, _i32, _i64, _P, _P, _P, _P]
+lib.moe_combine_bf16_host.restype = _i32
+lib.moe_combine_fp8_host.argtypes = [_P, _P, _P, _P, _i32, _i32, _i32, _i64, _P, _P, _P, _P]
+lib.moe_combine_fp8_host.restype = _i32
 
 MOE_OK = 0
 MOE_ERR_INVALID_ARG = 1
@@ -103,6 +114,7 @@ MOE_ERR_CUDA = 6
 MOE_SCALE_ROW_MAJOR = 0
 MOE_SCALE_COL_MAJOR = 1
 MOE_LAYOUT_NOALLOC_SCRATCH_BYTES = 1 << 20   # the fixed scratch of moe_dispatch_layout_noalloc
+MOE_HOST_FUSED = 1                           # host-buffer route+dispatch: the single launch
 
 
 class MoeError(RuntimeError):
@@ -125,6 +137,16 @@ def _ptr(t: torch.Tensor | None):
         return None
     if not t.is_cuda:
         raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return t.data_ptr() or None
+
+
+def _host_ptr(t: torch.Tensor | None):
+    if t is None:
+        return None
+    if t.is_cuda:
+        raise ValueError("expected a host (CPU) tensor")
     if not t.is_contiguous():
         raise ValueError("expected a contiguous tensor")
     return t.data_ptr() or None
@@ -455,6 +477,28 @@ def moe_route_dispatch_workspace_bytes(T: int, k: int, E: int, R: int) -> int:
 _default_fused_ws: dict[torch.device, Workspace] = {}
 
 
+def _path_outputs(fp8: bool, T: int, k: int, E: int, R: int, H: int, rows: int, x_dtype,
+                  dev) -> dict:
+    """Device outputs of route + layout + dispatch (the layout over E experts
+    and k slots per token)."""
+    out = dict(
+        topk_idx=torch.empty(T, k, dtype=torch.int32, device=dev),
+        topk_w=torch.empty(T, k, dtype=torch.float32, device=dev),
+        expert_counts=torch.empty(E, dtype=torch.int32, device=dev),
+        expert_src_counts=torch.empty(E, R, dtype=torch.int32, device=dev),
+        rank_counts=torch.empty(R, dtype=torch.int32, device=dev),
+        expert_offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
+        dispatch_pos=torch.empty(T, k, dtype=torch.int32, device=dev),
+        recv_src=torch.empty(max(rows, 1), dtype=torch.int32, device=dev),
+    )
+    if fp8:
+        out["recv_q"] = torch.empty(max(rows, 1), H, dtype=torch.uint8, device=dev)
+        out["recv_scale"] = torch.empty(max(rows, 1), H // 128, dtype=torch.float32, device=dev)
+    else:
+        out["recv_x"] = torch.empty(max(rows, 1), H, dtype=x_dtype, device=dev)
+    return out
+
+
 def _route_dispatch(fp8: bool, logits, x, k, R, capacity, rows, renormalize, out, workspace,
                     dev_status, stream, ex: dict | None = None) -> dict:
     assert logits.dtype == torch.float32 and logits.dim() == 2
@@ -472,22 +516,7 @@ def _route_dispatch(fp8: bool, logits, x, k, R, capacity, rows, renormalize, out
     if rows is None:
         rows = T * k if capacity == 0 else E * capacity
     if out is None:
-        out = dict(
-            topk_idx=torch.empty(T, k, dtype=torch.int32, device=dev),
-            topk_w=torch.empty(T, k, dtype=torch.float32, device=dev),
-            expert_counts=torch.empty(E, dtype=torch.int32, device=dev),
-            expert_src_counts=torch.empty(E, R, dtype=torch.int32, device=dev),
-            rank_counts=torch.empty(R, dtype=torch.int32, device=dev),
-            expert_offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
-            dispatch_pos=torch.empty(T, k, dtype=torch.int32, device=dev),
-            recv_src=torch.empty(max(rows, 1), dtype=torch.int32, device=dev),
-        )
-        if fp8:
-            out["recv_q"] = torch.empty(max(rows, 1), H, dtype=torch.uint8, device=dev)
-            out["recv_scale"] = torch.empty(max(rows, 1), H // 128, dtype=torch.float32,
-                                            device=dev)
-        else:
-            out["recv_x"] = torch.empty(max(rows, 1), H, dtype=x.dtype, device=dev)
+        out = _path_outputs(fp8, T, k, E, R, H, rows, x.dtype, dev)
     if workspace is None:
         workspace = _default_fused_ws.setdefault(dev, Workspace(dev))
     nbytes = moe_route_dispatch_workspace_bytes(T, k, E, R)
@@ -582,6 +611,114 @@ def moe_route_dispatch_ex_bf16(logits: torch.Tensor, x: torch.Tensor, k: int, R:
     ex = _ex_spec(logits.shape[1], n_shared, shared_weight, replica_offsets, replica_ids, E_phys)
     return _route_dispatch(False, logits, x, k, R, capacity, rows, renormalize, out, workspace,
                            dev_status, stream, ex)
+
+
+# ---------------------------------------------------------------------------
+# host-buffer entry points: inputs from, and the result to, host memory
+# ---------------------------------------------------------------------------
+
+def _route_dispatch_host(fp8: bool, logits_host, x_host, k, R, capacity, rows, renormalize, fused,
+                         out, workspace, dev_status, stream, device) -> dict:
+    assert logits_host.dtype == torch.float32 and logits_host.dim() == 2
+    x_host = _bits16(x_host)
+    T, E = logits_host.shape
+    H = x_host.shape[1]
+    assert x_host.shape[0] == T
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    if rows is None:
+        rows = T * k if capacity == 0 else E * capacity
+    if out is None:
+        out = _path_outputs(fp8, T, k, E, R, H, rows, x_host.dtype, dev)
+        out["logits"] = torch.empty(T, E, dtype=torch.float32, device=dev)
+        out["x"] = torch.empty(T, H, dtype=x_host.dtype, device=dev)
+    if workspace is None:
+        workspace = (_default_fused_ws if fused else _default_ws).setdefault(dev, Workspace(dev))
+    nbytes = (moe_route_dispatch_workspace_bytes(T, k, E, R) if fused
+              else moe_layout_workspace_bytes(T, k, E, R))
+    if nbytes == 0:
+        raise MoeError(MOE_ERR_INVALID_ARG, "workspace size")
+    ws = workspace.get(nbytes)
+    args = (_host_ptr(logits_host), _host_ptr(x_host), T, E, k, int(renormalize), R, capacity, H,
+            MOE_HOST_FUSED if fused else 0, _ptr(out["logits"]), _ptr(out["x"]),
+            _ptr(out["topk_idx"]), _ptr(out["topk_w"]), _ptr(out["expert_counts"]),
+            _ptr(out["expert_src_counts"]), _ptr(out["rank_counts"]),
+            _ptr(out["expert_offsets"]), _ptr(out["dispatch_pos"]), _ptr(out["recv_src"]))
+    tail = (rows, _ptr(ws), ws.numel(), _ptr(dev_status), _stream(stream))
+    if fp8:
+        _check(lib.moe_route_dispatch_fp8_host(*args, _ptr(out["recv_q"]), _ptr(out["recv_scale"]),
+                                               *tail), "moe_route_dispatch_fp8_host")
+    else:
+        _check(lib.moe_route_dispatch_bf16_host(*args, _ptr(out["recv_x"]), *tail),
+               "moe_route_dispatch_bf16_host")
+    out["rows"] = rows
+    return out
+
+
+def moe_route_dispatch_fp8_host(logits_host: torch.Tensor, x_host: torch.Tensor, k: int, R: int,
+                                capacity: int = 0, rows: int | None = None,
+                                renormalize: bool = False, fused: bool = False,
+                                out: dict | None = None, workspace: Workspace | None = None,
+                                dev_status: torch.Tensor | None = None, stream=None,
+                                device=None) -> dict:
+    """Route + layout + FP8 dispatch of host logits fp32 [T][E] and host x
+    bf16 [T][H]: both are copied (asynchronously when pinned) into device
+    buffers ``out["logits"]``, ``out["x"]``, then the separate kernels run
+    (``fused``: the single launch).  Returns the dict of
+    moe_route_dispatch_fp8 plus those two buffers.  Keep the host tensors
+    unchanged until the stream has passed the copies."""
+    return _route_dispatch_host(True, logits_host, x_host, k, R, capacity, rows, renormalize,
+                                fused, out, workspace, dev_status, stream, device)
+
+
+def moe_route_dispatch_bf16_host(logits_host: torch.Tensor, x_host: torch.Tensor, k: int, R: int,
+                                 capacity: int = 0, rows: int | None = None,
+                                 renormalize: bool = False, fused: bool = False,
+                                 out: dict | None = None, workspace: Workspace | None = None,
+                                 dev_status: torch.Tensor | None = None, stream=None,
+                                 device=None) -> dict:
+    """moe_route_dispatch_fp8_host with the bf16 dispatch (rows in recv_x)."""
+    return _route_dispatch_host(False, logits_host, x_host, k, R, capacity, rows, renormalize,
+                                fused, out, workspace, dev_status, stream, device)
+
+
+def moe_combine_bf16_host(y: torch.Tensor, dispatch_pos: torch.Tensor, topk_w: torch.Tensor,
+                          out_host: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                          dev_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """moe_combine_bf16 into the device buffer ``out``, then copied into the
+    host tensor ``out_host`` (pinned when allocated here), which is returned:
+    read it after the stream has been synchronised."""
+    y = _bits16(y)
+    rows, H = y.shape
+    T, k = dispatch_pos.shape
+    assert topk_w.dtype == torch.float32 and tuple(topk_w.shape) == (T, k)
+    if out is None:
+        out = torch.empty(T, H, dtype=y.dtype, device=y.device)
+    if out_host is None:
+        out_host = torch.empty(T, H, dtype=y.dtype, pin_memory=True)
+    _check(lib.moe_combine_bf16_host(_ptr(y), _ptr(dispatch_pos), _ptr(topk_w), T, H, k, rows,
+                                     _ptr(out), _host_ptr(out_host), _ptr(dev_status),
+                                     _stream(stream)), "moe_combine_bf16_host")
+    return out_host
+
+
+def moe_combine_fp8_host(y_q: torch.Tensor, y_scale: torch.Tensor, dispatch_pos: torch.Tensor,
+                         topk_w: torch.Tensor, out_host: torch.Tensor | None = None,
+                         out: torch.Tensor | None = None, dev_status: torch.Tensor | None = None,
+                         stream=None) -> torch.Tensor:
+    """moe_combine_fp8 into ``out``, then copied into the host tensor
+    ``out_host`` (see moe_combine_bf16_host)."""
+    assert y_q.dtype == torch.uint8 and y_scale.dtype == torch.float32
+    rows, H = y_q.shape
+    T, k = dispatch_pos.shape
+    assert topk_w.dtype == torch.float32 and tuple(topk_w.shape) == (T, k)
+    if out is None:
+        out = torch.empty(T, H, dtype=torch.bfloat16, device=y_q.device)
+    if out_host is None:
+        out_host = torch.empty(T, H, dtype=torch.bfloat16, pin_memory=True)
+    _check(lib.moe_combine_fp8_host(_ptr(y_q), _ptr(y_scale), _ptr(dispatch_pos), _ptr(topk_w), T,
+                                    H, k, rows, _ptr(out), _host_ptr(out_host), _ptr(dev_status),
+                                    _stream(stream)), "moe_combine_fp8_host")
+    return out_host
 
 
 def moe_quantize_e4m3(v: torch.Tensor, q: torch.Tensor | None = None, stream=None) -> torch.Tensor:

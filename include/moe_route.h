@@ -22,9 +22,10 @@
  *     combine kept in BF16.
  *
  * Conventions shared by every entry point
- *   - Every array pointer is a DEVICE pointer owned by the caller.  The
- *     library allocates nothing, keeps no pointer after the call returns and
- *     never synchronises the device.
+ *   - Every array pointer is a DEVICE pointer owned by the caller, except
+ *     the *_host arguments of the host-buffer entry points (near the end of
+ *     this file).  The library allocates nothing, keeps no pointer after the
+ *     call returns and never synchronises the device.
  *   - bf16 data are passed as their 16-bit patterns (uint16_t).
  *   - `stream` is a cudaStream_t (CUstream) passed as void*; NULL is the
  *     legacy default stream.  All device work is enqueued on it and runs
@@ -472,6 +473,85 @@ int moe_combine_bf16(const uint16_t *y, const int32_t *dispatch_pos,
 int moe_combine_fp8(const uint8_t *y_q, const float *y_scale, const int32_t *dispatch_pos,
                     const float *topk_w, int T, int H, int k, int64_t rows, uint16_t *out,
                     int32_t *dev_status, void *stream);
+
+/*
+ * Host-buffer entry points -- the path with the step's inputs and its result
+ * in HOST memory.  The pages have no counterpart: these are deployment
+ * variants of the entry points above, not steps of the method.  A serving
+ * loop whose router logits and hidden states arrive from the host (a
+ * CPU-side scheduler, a test harness, a process without a device allocator
+ * of its own) hands host buffers to the library; each call enqueues, on
+ * `stream` and in this order, the host -> device copies of the step's
+ * inputs, the same kernels as the device-pointer entry points, and (for the
+ * combine) the device -> host copy of the result.  Outputs are bit-identical
+ * to those entry points.
+ *
+ * Every argument of the device-pointer entry point keeps its meaning, layout
+ * and limits; the host buffers come in addition:
+ *   logits_host [T][E] fp32, x_host [T][H] bf16 bits, out_host [T][H] bf16
+ *   bits: host memory owned by the caller, read (written) by the copies.
+ *   logits [T][E], x [T][H], out [T][H]: the DEVICE buffers the copies go
+ *   through, owned by the caller, with the alignment rules above.
+ *
+ * Host memory.  With page-locked memory (cudaHostAlloc, cudaHostRegister,
+ * torch's pin_memory) the copies are asynchronous: the call returns at once
+ * and the copies overlap work on other streams.  The caller must then keep
+ * logits_host / x_host unchanged, and leave out_host unread, until the
+ * stream has passed the copies (an event or a stream synchronise).  Pageable
+ * memory also works, but the runtime stages it and the call may block the
+ * host thread until the copy has been staged (host -> device) or has
+ * completed (device -> host); a stream being captured into a CUDA graph
+ * accepts page-locked memory only (a capture error returns MOE_ERR_CUDA).
+ *
+ * Errors.  Every argument of every step is checked before anything is
+ * enqueued (MOE_ERR_INVALID_ARG / _UNSUPPORTED / _WORKSPACE, as the
+ * device-pointer entry points return them); a host pointer that is NULL
+ * while T > 0 is MOE_ERR_INVALID_ARG.  A failed copy or launch returns
+ * MOE_ERR_CUDA, and the steps before it may already be enqueued.  Kernel-
+ * detected errors go to *dev_status as above.
+ */
+
+/*
+ * moe_route_dispatch_fp8_host / moe_route_dispatch_bf16_host -- copy
+ * logits_host into logits and x_host into x, then route, lay out and
+ * dispatch.  flags = 0: the separate kernels, exactly moe_route_topk(logits,
+ * ...), moe_dispatch_layout(...) with `workspace` of at least
+ * moe_layout_workspace_bytes(T, k, E, R) bytes, and moe_dispatch_fp8 (or
+ * _bf16).  flags = MOE_HOST_FUSED: the single cooperative launch of
+ * moe_route_dispatch_fp8 (or _bf16), with that entry point's workspace rules
+ * (zero-filled before first use, at least moe_route_dispatch_workspace_bytes(
+ * T, k, E, R) bytes, not shared with the layout's).  Other flag bits are
+ * MOE_ERR_INVALID_ARG.  The outputs are those of the entry points named.
+ */
+#define MOE_HOST_FUSED 1
+int moe_route_dispatch_fp8_host(const float *logits_host, const uint16_t *x_host, int T, int E,
+                                int k, int renormalize, int R, int capacity, int H, int flags,
+                                float *logits, uint16_t *x, int32_t *topk_idx, float *topk_w,
+                                int32_t *expert_counts, int32_t *expert_src_counts,
+                                int32_t *rank_counts, int32_t *expert_offsets,
+                                int32_t *dispatch_pos, int32_t *recv_src, uint8_t *recv_q,
+                                float *recv_scale, int64_t rows, void *workspace, size_t ws_bytes,
+                                int32_t *dev_status, void *stream);
+int moe_route_dispatch_bf16_host(const float *logits_host, const uint16_t *x_host, int T, int E,
+                                 int k, int renormalize, int R, int capacity, int H, int flags,
+                                 float *logits, uint16_t *x, int32_t *topk_idx, float *topk_w,
+                                 int32_t *expert_counts, int32_t *expert_src_counts,
+                                 int32_t *rank_counts, int32_t *expert_offsets,
+                                 int32_t *dispatch_pos, int32_t *recv_src, uint16_t *recv_x,
+                                 int64_t rows, void *workspace, size_t ws_bytes,
+                                 int32_t *dev_status, void *stream);
+
+/*
+ * moe_combine_bf16_host / moe_combine_fp8_host -- moe_combine_bf16 (or
+ * _fp8) into the device buffer `out`, then a copy of out [T][H] into
+ * out_host.  T == 0 enqueues nothing.
+ */
+int moe_combine_bf16_host(const uint16_t *y, const int32_t *dispatch_pos, const float *topk_w,
+                          int T, int H, int k, int64_t rows, uint16_t *out, uint16_t *out_host,
+                          int32_t *dev_status, void *stream);
+int moe_combine_fp8_host(const uint8_t *y_q, const float *y_scale, const int32_t *dispatch_pos,
+                         const float *topk_w, int T, int H, int k, int64_t rows, uint16_t *out,
+                         uint16_t *out_host, int32_t *dev_status, void *stream);
 
 /*
  * moe_quantize_e4m3 -- q[i] = e4m3(v[i]) with the converter moe_dispatch_fp8

@@ -230,3 +230,39 @@ def test_layout_launch_count_on_the_host(moe):
     assert moe.moe_dispatch_layout_launches(32768, 8, 256, 8) == 2     # 16 chunks per rank
     assert moe.moe_dispatch_layout_launches(64, 2, 8, 2) in (1, 2)
     assert moe.kernels_per_step(4096, 8, 256, 32) == 5
+
+
+def test_host_buffer_entries_reject_bad_arguments(moe):
+    """Every step's arguments are checked before a copy is enqueued: a bad
+    flag, a NULL host buffer, a bad route, layout, dispatch or workspace
+    argument, and the combine's missing host output."""
+    f8, f16 = moe.lib.moe_route_dispatch_fp8_host, moe.lib.moe_route_dispatch_bf16_host
+    ws = 0x100000
+    wsb = moe.moe_layout_workspace_bytes(64, 2, 8, 2)
+
+    def call8(lh=A16, xh=A16, T=64, E=8, k=2, R=2, cap=0, H=256, flags=0, x=A16, rows=128,
+              wsp=ws, nbytes=wsb, recv_q=A16):
+        return f8(lh, xh, T, E, k, 0, R, cap, H, flags, A4, x, A4, A4, A4, A4, A4, A4, A4, A4,
+                  recv_q, A4, rows, wsp, nbytes, None, None)
+
+    assert call8(flags=2) == moe.MOE_ERR_INVALID_ARG          # unknown flag bit
+    assert call8(lh=None) == moe.MOE_ERR_INVALID_ARG          # no host logits with T > 0
+    assert call8(xh=None) == moe.MOE_ERR_INVALID_ARG
+    assert call8(k=0) == moe.MOE_ERR_INVALID_ARG              # route
+    assert call8(R=3) == moe.MOE_ERR_INVALID_ARG              # layout: E % R != 0
+    assert call8(rows=127) == moe.MOE_ERR_INVALID_ARG         # layout: rows < T*k
+    assert call8(nbytes=wsb - 4) == moe.MOE_ERR_WORKSPACE     # layout workspace short
+    assert call8(wsp=None) == moe.MOE_ERR_WORKSPACE
+    assert call8(H=264) == moe.MOE_ERR_UNSUPPORTED            # fp8 dispatch: H % 128
+    assert call8(x=A16 + 8) == moe.MOE_ERR_INVALID_ARG        # staging x not 16-byte aligned
+    assert call8(recv_q=A16 + 4) == moe.MOE_ERR_INVALID_ARG
+    assert call8(flags=moe.MOE_HOST_FUSED, H=264) == moe.MOE_ERR_UNSUPPORTED
+    assert call8(flags=moe.MOE_HOST_FUSED, wsp=None) == moe.MOE_ERR_WORKSPACE
+    assert f16(A16, A16, 64, 8, 2, 0, 2, 0, 100, 0, A4, A16, A4, A4, A4, A4, A4, A4, A4, A4, A16,
+               128, ws, wsb, None, None) == moe.MOE_ERR_INVALID_ARG   # H % 8
+    c16, c8 = moe.lib.moe_combine_bf16_host, moe.lib.moe_combine_fp8_host
+    assert c16(A16, A4, A4, 4, 256, 2, 8, A16, None, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert c16(A16, A4, A4, 4, 256, 2, 8, A16 + 2, A16, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert c16(None, None, None, 0, 256, 2, 0, None, None, None, None) == moe.MOE_OK  # T = 0
+    assert c8(A16, A4, A4, A4, 4, 200, 2, 8, A16, A16, None, None) == moe.MOE_ERR_UNSUPPORTED
+    assert c8(A16, A4, A4, A4, 4, 256, 2, 8, A16, None, None, None) == moe.MOE_ERR_INVALID_ARG
