@@ -609,6 +609,18 @@ __global__ void __launch_bounds__(kThreads, (NPL <= 12) ? 2 : 1)
         if (t < ntick && ok) {
             const int64_t u0 = static_cast<int64_t>(t) * TU;
             const int64_t u1 = min(u0 + TU, units);
+            // The ticket's units are contiguous in x (32 bytes each for FP8,
+            // 16 for bf16): one bulk L2 prefetch of them, issued before the
+            // waits, so the packers' loads of ticket n + 1 find x in L2.  In
+            // 10-step graphs, same outputs: dsv3 155.4 -> 152.0 us, prefill
+            // 1098.0 -> 1091.8, kimi unchanged (224.4 / 224.9).
+            if (lane == 0) {
+                constexpr int ub = FP8 ? 32 : 16;
+                asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(
+                                 reinterpret_cast<const uint8_t *>(A.x) + u0 * ub),
+                             "r"(static_cast<uint32_t>((u1 - u0) * ub))
+                             : "memory");
+            }
             const int ga = static_cast<int>(u0 / upt), gb = static_cast<int>((u1 - 1) / upt);
             const int ca = chunk_of(G, ga), cb = chunk_of(G, gb);
             for (int c = ca + lane; c <= cb; c += 32)
