@@ -64,6 +64,7 @@ L2_FLUSH_BYTES = 512 << 20
 STEPS_PER_GRAPH = 10           # consecutive steps captured in one CUDA graph (no-flush workloads)
 DEFAULT_CONFIGS = "dsv3,kimi,prefill"
 REGION_TARGET_S = 1.0          # timed work per workload for the step (repeated K-step regions)
+E2E_SETS = 3                   # e2e leg: streams with a device buffer set each, taken in turn
 MIN_REPS, MAX_REPS = 5, 4000
 DTYPES = {"route": "f32 logits -> f32 weights, int32 ids",
           "layout": "int32",
@@ -732,15 +733,16 @@ def measure(cfg: inputs.Config, args, dev, world: int, local: int) -> dict:
     # and its result out to page-locked host memory, inside the timed region.
     # Direct and fused pipelines go through the library's host-buffer entry
     # points (moe_route_dispatch_*_host, moe_combine_*_host), which enqueue
-    # the copies and the kernels on one stream; consecutive steps alternate
-    # between two streams with a device buffer set each, so one step's
-    # copies overlap the other's kernels and copies in the other direction.
+    # the copies and the kernels on one stream; consecutive steps take turns
+    # on E2E_SETS streams with a device buffer set each, so one step's copies
+    # overlap its neighbours' kernels and copies in the other direction.
     # The two-phase and shared-expert pipelines have no host-buffer entry
     # point: their steps are the device-pointer calls between torch copies on
     # two copy streams, double-buffered the same way.
     logits_pin = logits_h.pin_memory()
     x_pin = x_h.pin_memory()
-    out_pins = [torch.empty(T, H, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    nsets = max(2, args.e2e_sets)
+    out_pins = [torch.empty(T, H, dtype=torch.bfloat16).pin_memory() for _ in range(nsets)]
     n_e2e = min(K, 100)
     first, last = max(W, 3), max(W, 3) + n_e2e
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -751,11 +753,11 @@ def measure(cfg: inputs.Config, args, dev, world: int, local: int) -> dict:
                    f"{' with MOE_HOST_FUSED' if args.fused else ''}, moe_combine_"
                    f"{'fp8' if args.combine_fp8 else 'bf16'}_host): every step's inputs copied "
                    "in from page-locked host memory and its result copied out, inside the "
-                   "timed region; steps alternate between two streams and two device buffer "
-                   "sets; no L2 flush")
-        streams = [torch.cuda.Stream(dev) for _ in range(2)]
+                   f"timed region; steps take turns on {nsets} streams with a device buffer "
+                   "set each; no L2 flush")
+        streams = [torch.cuda.Stream(dev) for _ in range(nsets)]
         step_calls = []
-        for q in range(2):
+        for q in range(nsets):
             with torch.cuda.stream(streams[q]):
                 b = dict(logits=torch.empty_like(logits), x=torch.empty_like(x),
                          topk_idx=torch.empty_like(idx), topk_w=torch.empty_like(w),
@@ -791,20 +793,21 @@ def measure(cfg: inputs.Config, args, dev, world: int, local: int) -> dict:
                    + pw) if args.combine_fp8 else (lib.moe_combine_bf16_host, (y.data_ptr(),) + pw))
             step_calls.append(([rd, cb], b))
         ev_start = torch.cuda.Event()
-        ev_end = [torch.cuda.Event() for _ in range(2)]
+        ev_end = [torch.cuda.Event() for _ in range(nsets)]
         torch.cuda.synchronize(dev)
         for i in range(last):
-            q = i % 2
+            q = i % nsets
             if i == first:
-                torch.cuda.synchronize(dev)      # warm-up steps done on both streams
+                torch.cuda.synchronize(dev)      # warm-up steps done on every stream
                 t0.record(streams[0])
                 ev_start.record(streams[0])
-                streams[1].wait_event(ev_start)
+                for sq in streams[1:]:
+                    sq.wait_event(ev_start)
             for fn, a in step_calls[q][0]:
                 rc = fn(*a)
                 if rc != 0:
                     raise moe.MoeError(rc, fn.__name__)
-        for q in range(2):
+        for q in range(nsets):
             ev_end[q].record(streams[q])
             streams[0].wait_event(ev_end[q])
         t1.record(streams[0])
@@ -814,8 +817,8 @@ def measure(cfg: inputs.Config, args, dev, world: int, local: int) -> dict:
         for _, b in step_calls:
             if int(b["status"].item()) not in (moe.MOE_OK, moe.MOE_ERR_CAPACITY):
                 raise moe.MoeError(int(b["status"].item()), "host-buffer step")
-        last_set = step_calls[(last - 1) % 2][1]
-        if not torch.equal(out_pins[(last - 1) % 2].view(torch.int16),
+        last_set = step_calls[(last - 1) % nsets][1]
+        if not torch.equal(out_pins[(last - 1) % nsets].view(torch.int16),
                            last_set["out"].cpu().view(torch.int16)):
             raise RuntimeError("host result differs from the device buffer it was copied from")
         del step_calls, last_set, b
@@ -1006,6 +1009,9 @@ def main(argv=None):
                     help="route + layout + dispatch as one cooperative launch, then combine")
     ap.add_argument("--combine-fp8", action="store_true",
                     help="expert rows come back as E4M3 + 1x128 scales (moe_combine_fp8)")
+    ap.add_argument("--e2e-sets", type=int, default=E2E_SETS,
+                    help="e2e leg: streams (each with its own device buffers) the steps take "
+                         "turns on, so copies of neighbouring steps overlap")
     ap.add_argument("--region-seconds", type=float, default=REGION_TARGET_S,
                     help="timed work per workload: the K-step region repeats (at least 5 times) "
                          "until about this many seconds (dispatch+combine: half of it)")
