@@ -697,6 +697,32 @@ def measure(cfg: inputs.Config, args, dev, world: int, local: int) -> dict:
         stage_how = "one graph per stage, events between the replays"
         del gs
 
+    # the combine kernel alone: G launches back to back in one graph, each
+    # chained to the previous one by programmatic dependent launch, no event
+    # node between them (workloads that move more than 2 x L2 per step only:
+    # every launch then reads its rows from HBM)
+    comb_alone_ms = None
+    if not flush_needed:
+        cfn, cargs = calls[-1]
+
+        def comb_only():
+            rc = cfn(*cargs)
+            if rc != 0:
+                raise moe.MoeError(rc, cfn.__name__)
+        g_c = capture(comb_only, G)
+        n_c = max(3, int(0.1 / max(float(stage_ms[3]) * 1e-3 * G, 1e-6)))
+        with torch.cuda.stream(s):
+            for _ in range(2):
+                g_c.replay()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(s)
+            for _ in range(n_c):
+                g_c.replay()
+            b.record(s)
+            s.synchronize()
+        comb_alone_ms = max_over_ranks([a.elapsed_time(b) / (n_c * G)], world, dev)[0]
+        del g_c
+
     # eager: the same calls launched one by one from Python, no graph -- the
     # cost a caller that does not capture graphs pays (launch latency included)
     K3 = min(K, 200)
@@ -914,7 +940,15 @@ def measure(cfg: inputs.Config, args, dev, world: int, local: int) -> dict:
                      "traffic": combine_traffic(cfg.name, args.combine_fp8),
                      "algorithmic_bytes_per_launch": nb["combine"],
                      "how": "algorithmic bytes of one launch over the combine stage's mean "
-                            "CUDA-event time inside the step graph"},
+                            "CUDA-event time inside the step graph",
+                     "alone": None if comb_alone_ms is None else {
+                         "us": comb_alone_ms * 1e3,
+                         "achieved": nb["combine"] / (comb_alone_ms * 1e-3) / 1e9,
+                         "frac": nb["combine"] / (comb_alone_ms * 1e-3) / 1e9 / peak,
+                         "how": f"the combine launched {G} times back to back in one CUDA graph "
+                                "(programmatic dependent launch between them), events around "
+                                "the replays; the stage time above also holds the launch and "
+                                "ramp that the event nodes between stages expose"}},
         "e2e": {"value": n_gpus * nb["step"] / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
                 "us_per_step": e2e_ms * 1e3, "h2d_bytes_per_step": h2d,
                 "how": e2e_how,
@@ -939,7 +973,7 @@ def summary(res: dict) -> dict:
             "dispatch_combine": {k: dc[k] for k in ["us", "gbs", "frac_of_8tbs", "frac_of_measured",
                                                     "bytes", "repeats", "min_us", "max_us"]},
             "roofline": {k: res["roofline"][k] for k in ["kernel", "achieved", "peak", "frac",
-                                                         "traffic"]},
+                                                         "traffic", "alone"]},
             "e2e_us": res["e2e"]["us_per_step"], "clocks": res["clocks"],
             "capacity": res["capacity"], "rows": res["rows"], "l2": res["l2"]}
 
