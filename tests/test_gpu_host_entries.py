@@ -175,3 +175,62 @@ def test_host_entries_with_no_tokens(moe):
                                       torch.zeros(0, k, dtype=torch.float32, device="cuda"))
     torch.cuda.synchronize()
     assert out_h.shape == (0, H)
+
+
+@pytest.mark.parametrize("T,E,k,R,H,cap,fused", [
+    (7, 8, 2, 1, 256, 0, False),
+    (257, 384, 8, 1, 7168, 0, False),      # ragged against a chunk
+    (520, 1024, 32, 8, 128, 0, False),     # maximum E and k
+    (1200, 24, 6, 3, 512, 120, False),     # padded with drops
+    (96, 16, 4, 2, 16384, 0, False),       # wide rows
+    (1024, 64, 8, 8, 128, 0, False),       # single-launch layout
+    (1200, 24, 6, 3, 512, 120, True),      # the single fused launch, padded with drops
+    (300, 16, 16, 2, 128, 0, True),
+])
+def test_host_entries_equal_device_entries_on_edge_shapes(moe, T, E, k, R, H, cap, fused):
+    """Every output of the host-buffer entry points (FP8 and bf16 dispatch,
+    both combines) equals the device-pointer entry points' bit for bit,
+    status codes included (a capacity drop is reported the same way)."""
+    logits, x = inputs.make_random_case(T, H, E, k, seed=7 * T + E + k + H)
+    rows = T * k if cap == 0 else E * cap
+    dev = torch.device("cuda")
+    for fp8 in ([True, False] if H % 128 == 0 else [False]):
+        st_d, st_h = _status(), _status()
+        if fused:
+            f = moe.moe_route_dispatch_fp8 if fp8 else moe.moe_route_dispatch_bf16
+            want = f(logits.to(dev), x.to(dev), k, R, capacity=cap, rows=rows, dev_status=st_d)
+        else:
+            idx, w = moe.moe_route_topk(logits.to(dev), k)
+            want = moe.moe_dispatch_layout(idx, E, R, capacity=cap, rows=rows, dev_status=st_d)
+            want["topk_idx"], want["topk_w"] = idx, w
+            if fp8:
+                want["recv_q"], want["recv_scale"] = moe.moe_dispatch_fp8(
+                    x.to(dev), want["dispatch_pos"], rows, dev_status=st_d)
+            else:
+                want["recv_x"] = moe.moe_dispatch_bf16(x.to(dev), want["dispatch_pos"], rows,
+                                                       dev_status=st_d)
+        f = moe.moe_route_dispatch_fp8_host if fp8 else moe.moe_route_dispatch_bf16_host
+        got = f(_host(logits, True), _host(x, True), k, R, capacity=cap, rows=rows, fused=fused,
+                dev_status=st_h)
+        torch.cuda.synchronize()
+        assert st_h.item() == st_d.item()
+        filled = want["recv_src"][:rows] >= 0
+        for key in ["topk_idx", "topk_w"] + LAYOUT_KEYS:
+            a, b = got[key], want[key]
+            if key == "recv_src":
+                a, b = a[:rows], b[:rows]
+            assert torch.equal(a.view(torch.int32), b.view(torch.int32)), (key, fp8)
+        for key in (["recv_q", "recv_scale"] if fp8 else ["recv_x"]):
+            a, b = got[key][:rows][filled], want[key][:rows][filled]
+            assert torch.equal(a.contiguous().view(torch.uint8), b.contiguous().view(torch.uint8)), key
+        # combine of the dispatched rows (an identity expert), back to host memory
+        if fp8:
+            out_d = moe.moe_combine_fp8(want["recv_q"], want["recv_scale"], want["dispatch_pos"],
+                                        want["topk_w"])
+            out_h = moe.moe_combine_fp8_host(got["recv_q"], got["recv_scale"], got["dispatch_pos"],
+                                             got["topk_w"])
+        else:
+            out_d = moe.moe_combine_bf16(want["recv_x"], want["dispatch_pos"], want["topk_w"])
+            out_h = moe.moe_combine_bf16_host(got["recv_x"], got["dispatch_pos"], got["topk_w"])
+        torch.cuda.synchronize()
+        assert torch.equal(out_h.view(torch.int16), out_d.cpu().view(torch.int16)), fp8
