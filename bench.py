@@ -1057,6 +1057,10 @@ def main(argv=None):
     if args.region_seconds < 0:
         ap.error("--region-seconds must be >= 0")
     config_names(args.config)
+    world = dist_env()[0]
+    if args.gpus != world:
+        ap.error(f"--gpus {args.gpus} with WORLD_SIZE={world}: launch one rank per GPU with "
+                 "torch.distributed.run --nproc-per-node N")
     if args.impl == "reference":
         run_reference(args)
     else:

@@ -109,3 +109,12 @@ def test_repeated_region_count():
     assert bench.repetitions(0.5, 1.0) == bench.MIN_REPS
     assert bench.repetitions(1e-7, 1.0) == bench.MAX_REPS
     assert bench.repetitions(0.0, 1.0) == bench.MIN_REPS
+
+
+def test_gpus_must_match_the_launched_ranks():
+    """--gpus N without N launched ranks is refused before any work."""
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    p = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2",
+                        "--impl", "reference", "--config", "tiny"],
+                       env=env, capture_output=True, text=True, timeout=300)
+    assert p.returncode != 0 and "WORLD_SIZE=1" in p.stderr
