@@ -932,7 +932,9 @@ def measure(cfg: inputs.Config, args, dev, world: int, local: int) -> dict:
                              "frac_of_measured": dc_gbs / peak},
         "bytes_per_step": nb,
         "roofline": {"bound": "hbm",
-                     "kernel": "k_combine_fp8" if args.combine_fp8 else "k_combine_bf16",
+                     "kernel": "k_combine_fp8" if args.combine_fp8 else (
+                         "k_combine_bf16_w32" if moe.moe_combine_bf16_long_form(T, H, k)
+                         else "k_combine_bf16"),
                      "achieved": comb_gbs,
                      "peak": peak, "unit": "GB/s", "frac": comb_gbs / peak,
                      "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"

@@ -19,6 +19,7 @@ import torch
 __all__ = [
     "MoeError", "lib", "moe_status_string", "moe_route_topk", "moe_route_topk_ex",
     "moe_layout_workspace_bytes", "moe_dispatch_layout_launches", "kernels_per_step",
+    "moe_combine_bf16_long_form",
     "moe_dispatch_layout", "moe_dispatch_bf16", "moe_dispatch_fp8", "moe_combine_bf16",
     "moe_quantize_e4m3", "moe_dispatch_layout_noalloc", "moe_dispatch_fp8_ex", "Workspace",
     "LIB_PATH", "MOE_SCALE_ROW_MAJOR", "MOE_SCALE_COL_MAJOR", "moe_dispatch_layout_private",
@@ -52,6 +53,8 @@ lib.moe_layout_workspace_bytes.argtypes = [_i32, _i32, _i32, _i32]
 lib.moe_layout_workspace_bytes.restype = _sz
 lib.moe_dispatch_layout_launches.argtypes = [_i32, _i32, _i32, _i32]
 lib.moe_dispatch_layout_launches.restype = _i32
+lib.moe_combine_bf16_long_form.argtypes = [_i32, _i32, _i32]
+lib.moe_combine_bf16_long_form.restype = _i32
 lib.moe_dispatch_layout.argtypes = [_P, _i32, _i32, _i32, _i32, _i32, _i64, _P, _P, _P, _P, _P, _P,
                                     _P, _sz, _P, _P]
 lib.moe_dispatch_layout.restype = _i32
@@ -218,6 +221,12 @@ def moe_layout_workspace_bytes(T: int, k: int, E: int, R: int) -> int:
 
 def moe_dispatch_layout_launches(T: int, k: int, E: int, R: int) -> int:
     return int(lib.moe_dispatch_layout_launches(T, k, E, R))
+
+
+def moe_combine_bf16_long_form(T: int, H: int, k: int) -> int:
+    """1 when moe_combine_bf16 runs its long (32-byte load) form for these
+    sizes and 32-byte aligned buffers, else 0."""
+    return int(lib.moe_combine_bf16_long_form(T, H, k))
 
 
 def kernels_per_step(T: int, k: int, E: int, R: int, two_phase: bool = False) -> int:

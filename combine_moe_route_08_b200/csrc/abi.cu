@@ -365,6 +365,13 @@ int moe_combine_bf16(const uint16_t *y, const int32_t *dispatch_pos, const float
                                       as_stream(stream)));
 }
 
+int moe_combine_bf16_long_form(int T, int H, int k)
+{
+    if (!valid_tk(T, k) || H < 8 || H % 8 != 0)
+        return 0;
+    return moe::combine_bf16_long_form(T, H, k) ? 1 : 0;
+}
+
 size_t moe_route_dispatch_workspace_bytes(int T, int k, int E, int R)
 {
     if (!valid_layout_sizes(T, k, E, R))

@@ -9,8 +9,9 @@
 // Gecikmesi": bf16 combine, accumulation only at the receiver.
 //
 // bf16 rows: one CTA per token; a thread owns 8 consecutive channels (16
-// bytes of each row).  FP8 rows: a persistent grid walking the tokens, a
-// thread owning 16 channels.  Either way the token's row indices and weights
+// bytes of each row), or, for long combines with 32-byte aligned buffers, 16
+// channels read 32 bytes at a time.  FP8 rows: a persistent grid walking the
+// tokens, a thread owning 16 channels.  Either way the token's row indices and weights
 // are held in registers, so all k (up to 8) 16-byte loads of a pass issue
 // back to back before any is used; then the sum runs in ascending j with a
 // separate binary32 multiply and add per term (__fmul_rn / __fadd_rn are
@@ -30,6 +31,10 @@ constexpr int kMaxThreads = 512;
 // CTAs fit on an SM with 72 registers per thread, enough to hold 8 rows of 16
 // codes in flight without spilling.
 constexpr int kFp8Threads = 448;
+// Rows read (T * k * H * 2 bytes) from which the bf16 combine takes the
+// 32-byte-load form (k_combine_bf16_w32): between the measured sizes where it
+// lost (0.7 GB) or tied (0.9 GB) and the one where it won (3.8 GB).
+constexpr int64_t kLongCombineBytes = int64_t(2) << 30;
 
 // Lane j of every warp loads the token's j-th row index and weight (no
 // shared memory, no CTA barrier: each warp starts its row loads as soon as its
@@ -259,6 +264,101 @@ __global__ void __launch_bounds__(kFp8Threads, KREG <= 9 ? 2 : 1)
     pdl_trigger();
 }
 
+// 32 bytes of a row in one load (sm_100's 256-bit vector load), bypassing L1.
+struct Words8 {
+    uint32_t w[8];
+};
+__device__ __forceinline__ Words8 ld_stream_v8(const void *p)
+{
+    Words8 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(v.w[0]), "=r"(v.w[1]), "=r"(v.w[2]), "=r"(v.w[3]), "=r"(v.w[4]),
+                   "=r"(v.w[5]), "=r"(v.w[6]), "=r"(v.w[7])
+                 : "l"(p));
+    return v;
+}
+
+// The bf16 combine for long combines (k <= 8, H % 16 == 0, y and out 32-byte
+// aligned): a thread owns 16 channels, reads 32 bytes of a row per load and
+// takes the rows two at a time (40 registers, three CTAs per SM); the same
+// products and sums in the same order as k_combine_bf16, so the same bits.
+// Kernel alone and in whole steps, alternating, at T = 32768, H = 7168,
+// k = 8: 605.5 against 624.9 us, steps 1052.5 against 1075.5 us.  In the
+// decode chains (4096 and 6144 tokens) it made whole steps slower (153.1
+// against 147.3, 218.5 against 215.0 us) with the kernel alone unchanged, so
+// it is used only when the rows read reach kLongCombineBytes.
+__global__ void __launch_bounds__(kMaxThreads, 3)
+    k_combine_bf16_w32(const uint8_t *__restrict__ y, const int32_t *__restrict__ dispatch_pos,
+                       const float *__restrict__ topk_w, int nu, int k, int64_t rows,
+                       uint4 *__restrict__ out, int32_t *__restrict__ dev_status)
+{
+    const int g = blockIdx.x;
+    const int lane = threadIdx.x & 31;
+    pdl_wait();
+    int myr = -1;
+    float myw = 0.0f;
+    if (lane < k) {
+        myr = __ldg(dispatch_pos + static_cast<size_t>(g) * k + lane);
+        myw = __ldg(topk_w + static_cast<size_t>(g) * k + lane);
+        if (myr < -1 || myr >= rows) {
+            if (threadIdx.x < 32)
+                report(dev_status, MOE_ERR_INVALID_ARG);
+            myr = -1;
+        }
+    }
+    int rr[8];
+    float ww[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {  // lanes >= k hold -1
+        rr[j] = __shfl_sync(kFullMask, myr, j);
+        ww[j] = __shfl_sync(kFullMask, myw, j);
+    }
+    for (int v0 = 0; v0 < nu; v0 += blockDim.x) {  // CTA-uniform trips (shuffles)
+        const int v = v0 + threadIdx.x;
+        const bool act = v < nu;
+        float acc[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+            acc[c] = 0.0f;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {  // rows 2q and 2q + 1
+            Words8 d[2];
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj) {
+                const int j = 2 * q + jj;
+                if (act && rr[j] >= 0) {
+                    d[jj] = ld_stream_v8(y + (static_cast<size_t>(rr[j]) * nu + v) * 32);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        d[jj].w[i] = 0u;
+                }
+            }
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj) {
+                const int j = 2 * q + jj;
+                if (rr[j] >= 0) {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        acc[2 * i] = __fadd_rn(acc[2 * i], __fmul_rn(ww[j], bf16_lo(d[jj].w[i])));
+                        acc[2 * i + 1] =
+                            __fadd_rn(acc[2 * i + 1], __fmul_rn(ww[j], bf16_hi(d[jj].w[i])));
+                    }
+                }
+            }
+        }
+        if (act) {
+            uint4 *o = out + static_cast<size_t>(g) * (2 * nu) + 2 * v;
+            st_stream_v4(o, make_uint4(bf16x2_rn(acc[0], acc[1]), bf16x2_rn(acc[2], acc[3]),
+                                       bf16x2_rn(acc[4], acc[5]), bf16x2_rn(acc[6], acc[7])));
+            st_stream_v4(o + 1, make_uint4(bf16x2_rn(acc[8], acc[9]), bf16x2_rn(acc[10], acc[11]),
+                                           bf16x2_rn(acc[12], acc[13]),
+                                           bf16x2_rn(acc[14], acc[15])));
+        }
+    }
+    pdl_trigger();
+}
+
 int threads_for(int units, int max_threads = kMaxThreads)
 {
     const int passes = ceil_div(units, max_threads);
@@ -336,6 +436,11 @@ cudaError_t combine_fp8(const uint8_t *yq, const float *ys, const int32_t *dispa
     return launch_fp8<16, false>(yq, ys, dispatch_pos, topk_w, T, H, k, rows, out, dev_status, s);
 }
 
+bool combine_bf16_long_form(int T, int H, int k)
+{
+    return k <= 8 && H % 16 == 0 && static_cast<int64_t>(T) * k * H * 2 >= kLongCombineBytes;
+}
+
 cudaError_t combine_bf16(const uint16_t *y, const int32_t *dispatch_pos, const float *topk_w,
                          int T, int H, int k, int64_t rows, uint16_t *out, int32_t *dev_status,
                          cudaStream_t s)
@@ -344,6 +449,11 @@ cudaError_t combine_bf16(const uint16_t *y, const int32_t *dispatch_pos, const f
     const dim3 grid(T), block(threads_for(nvec));
     const uint4 *yv = reinterpret_cast<const uint4 *>(y);
     uint4 *ov = reinterpret_cast<uint4 *>(out);
+    if (combine_bf16_long_form(T, H, k) && reinterpret_cast<uintptr_t>(y) % 32 == 0 &&
+        reinterpret_cast<uintptr_t>(out) % 32 == 0)
+        return launch_pdl(k_combine_bf16_w32, grid, dim3(threads_for(H / 16)), 0, s,
+                          reinterpret_cast<const uint8_t *>(y), dispatch_pos, topk_w, H / 16, k,
+                          rows, ov, dev_status);
     if (k <= 2)
         return launch_pdl(k_combine_bf16<2>, grid, block, 0, s, yv, dispatch_pos, topk_w, nvec, k,
                           rows, ov, dev_status);

@@ -71,6 +71,9 @@ cudaError_t dispatch_fp8(const uint16_t *x, int T, int H, int k, const int32_t *
 cudaError_t combine_bf16(const uint16_t *y, const int32_t *dispatch_pos, const float *topk_w,
                          int T, int H, int k, int64_t rows, uint16_t *out, int32_t *dev_status,
                          cudaStream_t s);
+// Whether combine_bf16 takes its long, 32-byte-load form for these sizes when
+// y and out are 32-byte aligned.
+bool combine_bf16_long_form(int T, int H, int k);
 
 // Route + layout + dispatch in one cooperative launch (packed or padded
 // layout).  E, k: the router's experts and routed slots; with ex the layout

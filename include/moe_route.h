@@ -458,6 +458,15 @@ int moe_combine_bf16(const uint16_t *y, const int32_t *dispatch_pos,
                      uint16_t *out, int32_t *dev_status, void *stream);
 
 /*
+ * moe_combine_bf16_long_form -- 1 when moe_combine_bf16 runs its long form
+ * for these sizes (k <= 8, H % 16 == 0 and T*k*H*2 >= 2 GiB of rows read,
+ * with y and out 32-byte aligned: 32-byte row loads, two rows at a time),
+ * 0 otherwise or for invalid sizes.  Both forms give the same bits; this host
+ * query only names the kernel that runs (for profiling and reports).
+ */
+int moe_combine_bf16_long_form(int T, int H, int k);
+
+/*
  * moe_combine_fp8 -- moe_combine_bf16 with the expert rows in the dispatch's
  * FP8 format: E4M3 codes and one fp32 scale per 1x128 block (DeepSeek-V3
  * fragments: activations scaled per token per 128 channels), a payload of

@@ -266,3 +266,15 @@ def test_host_buffer_entries_reject_bad_arguments(moe):
     assert c16(None, None, None, 0, 256, 2, 0, None, None, None, None) == moe.MOE_OK  # T = 0
     assert c8(A16, A4, A4, A4, 4, 200, 2, 8, A16, A16, None, None) == moe.MOE_ERR_UNSUPPORTED
     assert c8(A16, A4, A4, A4, 4, 256, 2, 8, A16, None, None, None) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_combine_long_form_query(moe):
+    """The bf16 combine's long form is chosen from the sizes alone: k <= 8,
+    H % 16 == 0 and at least 2 GiB of rows read."""
+    assert moe.moe_combine_bf16_long_form(32768, 7168, 8) == 1     # 3.76 GB of rows
+    assert moe.moe_combine_bf16_long_form(16384, 8192, 8) == 1     # exactly 2 GiB
+    assert moe.moe_combine_bf16_long_form(16383, 8192, 8) == 0
+    assert moe.moe_combine_bf16_long_form(4096, 7168, 8) == 0      # decode sizes
+    assert moe.moe_combine_bf16_long_form(32768, 7168, 9) == 0     # k > 8
+    assert moe.moe_combine_bf16_long_form(65536, 7160, 8) == 0     # H % 16 != 0
+    assert moe.moe_combine_bf16_long_form(-1, 7168, 8) == 0

@@ -532,6 +532,41 @@ def test_combine_bf16_k_sweep(moe, k, T, H):
     assert st.item() == 0
 
 
+@pytest.mark.parametrize("k,T,H,offset", [(4, 32768, 8192, 0), (8, 16384, 8192, 0),
+                                          (8, 16384, 8192, 16)])
+def test_combine_bf16_long_forms(moe, k, T, H, offset):
+    """Long combines (rows read >= 2 GiB): with y and out 32-byte aligned
+    (offset 0) the 32-byte-load form runs, with y only 16-byte aligned the
+    16-byte form; both equal the oracle within 1 bf16 ulp and bit for bit on
+    sampled tokens (first, last and 254 seeded ones), -1 slots included."""
+    rows = T * k
+    assert rows * H * 2 >= 2 << 30
+    gen = torch.Generator(device="cuda").manual_seed(77 + k + offset)
+    ybuf = torch.empty(rows * H + 16, dtype=torch.bfloat16, device="cuda")
+    y = ybuf[offset // 2: offset // 2 + rows * H].view(rows, H)
+    for r0 in range(0, rows, 8192):  # seeded rows, generated in pieces
+        r1 = min(rows, r0 + 8192)
+        y[r0:r1] = torch.randn(r1 - r0, H, generator=gen, device="cuda").to(torch.bfloat16)
+    rng = np.random.default_rng(5 + k + offset)
+    pos = rng.permutation(rows).astype(np.int32).reshape(T, k)
+    pos[rng.random((T, k)) < 0.05] = -1
+    w = rng.random((T, k)).astype(np.float32)
+    st = _status()
+    out = moe.moe_combine_bf16(y, to_dev(pos), to_dev(w), dev_status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    toks = np.unique(np.concatenate([[0, T - 1], rng.integers(0, T, 254)])).astype(np.int64)
+    used = np.unique(pos[toks][pos[toks] >= 0])
+    remap = np.full(rows, -1, np.int64)
+    remap[used] = np.arange(used.size)
+    y_sub = gpu_bits(y.index_select(0, torch.from_numpy(used).cuda()))
+    pos_sub = np.where(pos[toks] >= 0, remap[np.maximum(pos[toks], 0)], -1).astype(np.int32)
+    acc, out_o = oracle.combine(y_sub, pos_sub, w[toks])
+    got = gpu_bits(out.index_select(0, torch.from_numpy(toks).cuda()))
+    assert check_combine(got, acc, out_o, f"long k={k} offset={offset}") == 1.0
+    del ybuf, y, out
+
+
 @pytest.mark.parametrize("k,T,H", [(1, 37, 128), (3, 37, 128), (8, 37, 128), (9, 37, 128),
                                    (11, 37, 128), (16, 37, 128), (17, 37, 128),
                                    (32, 37, 128), (8, 4099, 128), (2, 9001, 128), (9, 2100, 1024),
