@@ -391,6 +391,43 @@ def test_dispatch_fp8_column_major_scales(moe, name):
                               want_s.view(np.uint32))
 
 
+@pytest.mark.parametrize("T,H,k,offset,colmajor", [(8192, 8192, 8, 0, False),
+                                                    (8192, 7168, 3, 0, True),
+                                                    (8192, 8192, 8, 16, False)])
+def test_dispatch_fp8_when_x_is_read_from_hbm(moe, T, H, k, offset, colmajor):
+    """x larger than three quarters of L2 (not prefetched): with recv_q
+    32-byte aligned (offset 0) the 32-channel, 32-byte-store form runs, with
+    recv_q only 16-byte aligned the 16-channel form; codes and scales equal
+    the oracle's bit for bit (-1 slots, k = 3, column-major scales)."""
+    assert T * H * 2 > 3 * 126 * 2 ** 20 // 4
+    rng = np.random.default_rng(11 + k + offset)
+    rows = T * k
+    x = torch.randn(T, H, generator=torch.Generator().manual_seed(3 + k), dtype=torch.float32)
+    x = x.to(torch.bfloat16)
+    pos = rng.permutation(rows).astype(np.int32).reshape(T, k)
+    pos[rng.random((T, k)) < 0.05] = -1
+    qbuf = torch.zeros(rows * H + 32, dtype=torch.uint8, device="cuda")
+    q = qbuf[offset: offset + rows * H].view(rows, H)
+    S = H // 128
+    st = _status()
+    if colmajor:
+        ld = (rows + 3) // 4 * 4
+        _, sc = moe.moe_dispatch_fp8_ex(to_dev(x), to_dev(pos), rows, moe.MOE_SCALE_COL_MAJOR, ld,
+                                        recv_q=q, dev_status=st)
+        sc = sc[:, :rows].t()
+    else:
+        _, sc = moe.moe_dispatch_fp8(to_dev(x), to_dev(pos), rows, recv_q=q, dev_status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    want_q, want_s = oracle.dispatch_fp8(inputs.bf16_bits(x), pos, rows)
+    filled = np.zeros(rows, bool)
+    filled[pos[pos >= 0]] = True
+    assert np.array_equal(q.cpu().numpy()[filled], want_q[filled])
+    assert np.array_equal(sc.contiguous().cpu().numpy()[filled].view(np.uint32),
+                          want_s[filled].view(np.uint32))
+    del qbuf, q
+
+
 # ------------------------------------------ two-phase dispatch (private regions)
 
 @pytest.mark.parametrize("name", ["dsv3", "kimi", "dsv3_shared"])
