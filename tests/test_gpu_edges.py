@@ -225,6 +225,80 @@ def test_fp8_extreme_values(moe):
     assert np.array_equal(s.cpu().numpy().view(np.uint32), so.view(np.uint32))
 
 
+def test_fp8_nan_and_infinite_inputs(moe):
+    """NaN and infinite inputs, which the pages do not discuss, follow the
+    definition literally on both sides: a NaN never raises the block's amax
+    and quantises to the NaN code 0x7F; an infinity makes s infinite, so
+    finite values give signed zeros and the infinity gives NaN (inf / inf).
+    Codes and scales equal the oracle's bit for bit."""
+    H, T = 512, 6
+    x = torch.randn(T, H, generator=torch.Generator().manual_seed(8), dtype=torch.float32)
+    x[0, 3] = float("nan")                      # one NaN in a block
+    x[1, :128] = float("nan")                   # an all-NaN block: amax 0, s = 1
+    x[2, 7] = float("inf")
+    x[3, 200] = float("-inf")
+    x[4, 130] = float("inf")
+    x[4, 131] = float("-inf")
+    x[4, 300] = float("nan")
+    xb = x.to(torch.bfloat16)
+    pos = np.arange(T * 2, dtype=np.int32).reshape(T, 2)
+    q, s = moe.moe_dispatch_fp8(to_dev(xb), to_dev(pos), T * 2)
+    qo, so = oracle.dispatch_fp8(inputs.bf16_bits(xb), pos, T * 2)
+    torch.cuda.synchronize()
+    assert np.array_equal(q.cpu().numpy(), qo)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), so.view(np.uint32))
+    # token g fills rows 2g and 2g + 1
+    assert qo[0, 3] == 0x7F                                   # the NaN element
+    assert np.all(qo[2, :128] == 0x7F) and so[2, 0] == 1.0    # all-NaN block: s = 1
+    assert qo[4, 7] == 0x7F and np.isinf(so[4, 0])            # inf / inf, s infinite
+    assert np.all(qo[4, :128][np.arange(128) != 7] & 0x7F == 0)  # finite / inf: signed zeros
+
+
+def _same_up_to_nan_payload(got_bits, acc, want_bits, where):
+    """Outputs whose oracle sum is NaN must be NaN (payload and sign are not
+    part of the contract), infinite sums the same infinity, every other
+    output within 1 bf16 ulp and bit-identical."""
+    nan = np.isnan(acc)
+    inf = np.isinf(acc)
+    got_f = bf16_to_f64(got_bits)
+    assert np.all(np.isnan(got_f[nan])), where
+    assert not np.any(np.isnan(got_f[~nan])), where
+    assert np.array_equal(got_bits[inf], want_bits[inf]), where      # signed infinities
+    keep = ~(nan | inf)
+    assert check_combine(got_bits[keep], acc[keep], want_bits[keep], where) == 1.0
+
+
+def test_combine_nan_and_infinite_rows(moe):
+    """bf16 rows holding NaN, +inf and -inf (a token summing +inf and -inf
+    gets NaN), and FP8 rows holding the NaN code: NaN where the oracle's sum
+    is NaN, infinities where it is infinite, everything else bit-identical."""
+    T, k, H = 16, 4, 256
+    rows = T * k
+    rng = np.random.default_rng(21)
+    y = torch.randn(rows, H, generator=torch.Generator().manual_seed(9), dtype=torch.float32)
+    y[1, 0] = float("nan")
+    y[5, 10] = float("inf")
+    y[6, 10] = float("-inf")                    # rows 5 and 6 belong to token 1
+    y[9, 20] = float("inf")
+    yb = y.to(torch.bfloat16)
+    pos = np.arange(rows, dtype=np.int32).reshape(T, k)
+    w = rng.random((T, k)).astype(np.float32)
+    acc, out_o = oracle.combine(inputs.bf16_bits(yb), pos, w)
+    out = moe.moe_combine_bf16(to_dev(yb), to_dev(pos), to_dev(w))
+    torch.cuda.synchronize()
+    _same_up_to_nan_payload(gpu_bits(out), acc, out_o, "bf16 rows")
+    assert np.isnan(acc[1, 10]) and np.isinf(acc[2, 20])
+    # the same rows as E4M3 + scales (each row quantised on its own)
+    qo, so = oracle.dispatch_fp8(inputs.bf16_bits(yb), np.arange(rows, dtype=np.int32)[:, None], rows)
+    qo[3, 40] = 0x7F
+    qo[12, 41] = 0xFF
+    acc8, out8_o = oracle.combine_fp8(qo, so, pos, w)
+    out8 = moe.moe_combine_fp8(to_dev(qo), to_dev(so), to_dev(pos), to_dev(w))
+    torch.cuda.synchronize()
+    _same_up_to_nan_payload(gpu_bits(out8), acc8, out8_o, "fp8 rows")
+    assert np.isnan(acc8[0, 40]) and np.isnan(acc8[3, 41])
+
+
 def test_workspace_reuse_and_determinism(moe):
     ws = moe.Workspace("cuda")
     cfgs = [(4096, 256, 8, 32), (64, 8, 2, 2), (32768, 256, 8, 8), (4096, 256, 8, 32)]
