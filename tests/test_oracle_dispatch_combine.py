@@ -79,6 +79,32 @@ def test_fp8_properties_on_workload_rows(oracle_mod):
     assert np.array_equal(qn, q ^ 0x80)
 
 
+def test_fp8_nan_and_infinity_follow_the_definition(oracle_mod):
+    """The literal reading for inputs the pages do not discuss: the block
+    amax is a maximum a NaN never raises, s = amax / 448 (1 for amax 0), and
+    each code is e4m3(x / s) with NaN -> 0x7F.  So a NaN element gives 0x7F
+    and leaves its neighbours' codes as without it, an all-NaN block has s = 1,
+    and an infinity makes s infinite: finite elements become signed zeros and
+    the infinity itself NaN (inf / inf)."""
+    H = 256
+    base = torch.linspace(-3.0, 3.0, H)
+    x = torch.stack([base, base, base, base]).to(torch.float32)
+    x[1, 5] = float("nan")
+    x[2, :128] = float("nan")
+    x[3, 9] = float("-inf")
+    xb = _bits(x.to(torch.bfloat16))
+    q, s = oracle_mod.dispatch_fp8(xb, np.arange(4, dtype=np.int32)[:, None], 4)
+    assert q[1, 5] == 0x7F
+    keep = np.arange(H) != 5
+    assert np.array_equal(q[1][keep], q[0][keep]) and np.array_equal(s[1], s[0])
+    assert np.all(q[2, :128] == 0x7F) and s[2, 0] == 1.0
+    assert np.array_equal(q[2, 128:], q[0, 128:]) and s[2, 1] == s[0, 1]
+    assert np.isinf(s[3, 0]) and s[3, 0] > 0 and q[3, 9] == 0x7F
+    signs = np.signbit(base[:128].numpy())
+    others = np.arange(128) != 9
+    assert np.array_equal(q[3, :128][others], np.where(signs, 0x80, 0x00)[others].astype(np.uint8))
+
+
 def test_fp8_dispatch_writes_each_token_to_its_k_rows(oracle_mod):
     cfg = inputs.CONFIGS["dsv3"]
     T = 96
