@@ -30,6 +30,24 @@ def test_algorithmic_bytes_dsv3():
     assert abs(nb["combine"] / 1e6 - 528.74) < 0.01
 
 
+def test_algorithmic_bytes_prefill_and_fp8_payload():
+    """Prefill counts only the rows that are filled (padding rows are neither
+    read nor written); the FP8 payload moves H code bytes and H/128 scales per
+    row instead of 2H bytes."""
+    cfg = inputs.CONFIGS["prefill"]
+    T, H, k, S = 32768, 7168, 8, 56
+    kept = T * k
+    rows = 256 * 1105                               # padded: E x capacity
+    nb = bench.algorithmic_bytes(cfg, rows=rows, kept=kept)
+    assert nb["dispatch"] == T * H * 2 + T * k * 4 + kept * H + kept * S * 4    # 2408.6 MB
+    assert nb["combine"] == kept * H * 2 + T * k * 8 + T * H * 2                # 4230.0 MB
+    assert abs(nb["dispatch"] / 1e6 - 2408.58) < 0.01 and abs(nb["combine"] / 1e6 - 4229.96) < 0.01
+    nb8 = bench.algorithmic_bytes(inputs.CONFIGS["dsv3"], rows=32768, kept=32768, combine_fp8=True)
+    assert nb8["combine"] == 32768 * 7168 + 32768 * 56 * 4 + 32768 * 8 + 4096 * 7168 * 2  # 301.1 MB
+    dropped = bench.algorithmic_bytes(cfg, rows=rows, kept=kept - 1000)
+    assert nb["combine"] - dropped["combine"] == 1000 * H * 2
+
+
 def _free_port():
     with socket.socket() as s:
         s.bind(("127.0.0.1", 0))
