@@ -209,29 +209,37 @@ class ClockSampler:
         time.sleep(0.1)
         self.proc.terminate()
         out, _ = self.proc.communicate(timeout=10)
-        rows = []
-        for line in out.strip().splitlines():
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                ts = _dt.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f")
-            except ValueError:
-                continue
-            rows.append((ts, parts))
-        inside = [p for ts, p in rows
-                  if any(a is not None and b is not None and a <= ts <= b for a, b in self.windows)]
-        use = inside or [p for _, p in rows]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({n for p in use for n, v in zip(names, p[5:9]) if v.lower() == "active"})
-        sm = [float(p[1]) for p in use if p[1].replace(".", "").isdigit()]
-        smax = [float(p[2]) for p in use if p[2].replace(".", "").isdigit()]
-        return {"sm_mhz": float(np.median(sm)) if sm else None,
-                "sm_max_mhz": max(smax) if smax else None,
-                "sm_mhz_min": min(sm) if sm else None,
-                "reasons": reasons, "samples": len(rows), "samples_in_timed_region": len(inside),
-                "from": "samples inside the timed regions" if inside else
-                        "no sample fell inside the timed regions: samples around them"}
+        return summarise_clock_samples(out, self.windows)
+
+
+def summarise_clock_samples(out: str, windows: list) -> dict:
+    """nvidia-smi CSV lines (ClockSampler.FIELDS, no header, no units) ->
+    median SM clock, maximum clock, active throttle reasons and sample
+    counts, from the samples inside the [start, end] windows when there are
+    any, else from all of them."""
+    rows = []
+    for line in out.strip().splitlines():
+        parts = [p.strip() for p in line.split(",")]
+        if len(parts) < 9:
+            continue
+        try:
+            ts = _dt.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f")
+        except ValueError:
+            continue
+        rows.append((ts, parts))
+    inside = [p for ts, p in rows
+              if any(a is not None and b is not None and a <= ts <= b for a, b in windows)]
+    use = inside or [p for _, p in rows]
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    reasons = sorted({n for p in use for n, v in zip(names, p[5:9]) if v.lower() == "active"})
+    sm = [float(p[1]) for p in use if p[1].replace(".", "").isdigit()]
+    smax = [float(p[2]) for p in use if p[2].replace(".", "").isdigit()]
+    return {"sm_mhz": float(np.median(sm)) if sm else None,
+            "sm_max_mhz": max(smax) if smax else None,
+            "sm_mhz_min": min(sm) if sm else None,
+            "reasons": reasons, "samples": len(rows), "samples_in_timed_region": len(inside),
+            "from": "samples inside the timed regions" if inside else
+                    "no sample fell inside the timed regions: samples around them"}
 
 
 # --------------------------------------------------------------------------

@@ -136,3 +136,27 @@ def test_gpus_must_match_the_launched_ranks():
                         "--impl", "reference", "--config", "tiny"],
                        env=env, capture_output=True, text=True, timeout=300)
     assert p.returncode != 0 and "WORLD_SIZE=1" in p.stderr
+
+
+def test_clock_summary_uses_the_samples_inside_the_timed_regions():
+    """Samples inside the [start, end] windows decide the clock and the
+    throttle reasons; samples outside count only when none fell inside."""
+    import datetime as dt
+    t0 = dt.datetime(2026, 1, 1, 12, 0, 0)
+
+    def line(sec, mhz, power_cap="Not Active", thermal="Not Active"):
+        ts = (t0 + dt.timedelta(seconds=sec)).strftime("%Y/%m/%d %H:%M:%S.%f")[:-3]
+        return f"{ts}, {mhz}, 1965, 900.0, 0x0, Not Active, Not Active, {thermal}, {power_cap}"
+
+    out = "\n".join([line(0.0, 1965), line(1.0, 1700, power_cap="Active"),
+                     line(1.2, 1720, power_cap="Active"), line(1.4, 1710, power_cap="Active"),
+                     line(3.0, 1965, thermal="Active"), "garbage line"])
+    win = [[t0 + dt.timedelta(seconds=0.9), t0 + dt.timedelta(seconds=1.5)]]
+    got = bench.summarise_clock_samples(out, win)
+    assert got["samples"] == 5 and got["samples_in_timed_region"] == 3
+    assert got["sm_mhz"] == 1710.0 and got["sm_mhz_min"] == 1700.0 and got["sm_max_mhz"] == 1965.0
+    assert got["reasons"] == ["sw_power_cap"]          # the thermal sample lies outside
+    none_inside = bench.summarise_clock_samples(out, [[t0 + dt.timedelta(seconds=5),
+                                                       t0 + dt.timedelta(seconds=6)]])
+    assert none_inside["samples_in_timed_region"] == 0 and none_inside["sm_mhz"] == 1720.0
+    assert none_inside["reasons"] == ["sw_power_cap", "sw_thermal_slowdown"]
