@@ -4,6 +4,8 @@ synchronously, before anything touches the CUDA runtime."""
 import ctypes
 import os
 import re
+import shutil
+import subprocess
 
 import pytest
 import torch
@@ -278,3 +280,13 @@ def test_combine_long_form_query(moe):
     assert moe.moe_combine_bf16_long_form(32768, 7168, 9) == 0     # k > 8
     assert moe.moe_combine_bf16_long_form(65536, 7160, 8) == 0     # H % 16 != 0
     assert moe.moe_combine_bf16_long_form(-1, 7168, 8) == 0
+
+
+@pytest.mark.skipif(shutil.which("gcc") is None, reason="needs a C compiler")
+def test_header_is_plain_c():
+    """include/moe_route.h compiles as C99 on its own (no C++ or CUDA types in
+    the boundary) and as C++17."""
+    for lang, std in (("c", "-std=c99"), ("c++", "-std=c++17")):
+        p = subprocess.run(["gcc", std, "-Wall", "-Wextra", "-Werror", "-fsyntax-only", "-x", lang,
+                            HEADER], capture_output=True, text=True, timeout=60)
+        assert p.returncode == 0, p.stderr
